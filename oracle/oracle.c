@@ -1,0 +1,309 @@
+/*
+ * CPU oracle for QK4V8 mixed-precision attention (test infrastructure only).
+ *
+ * This file is test infrastructure. Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load it. The library path never calls it,
+ * and it shares no code, header or table with the CUDA implementation.
+ *
+ * What it computes (MpFA QK4V8 article, mhpn.cn "MpFA免训练量化：QK4V8混合精度在
+ * Blackwell上的推理加速实践"; MiMo FP4 article, wmrh.cn "MXFP4专家量化"):
+ *  - Q and K are quantized to 4-bit, V to 8-bit (article §1.1, §2.1, §2.2).
+ *  - Scales are computed per block of the data as it is quantized, without any
+ *    calibration set (article §1.2, §3.2). The block is a group of 32 elements
+ *    with one shared power-of-two scale (MiMo article, "MXFP4专家量化": one
+ *    block scale per 32 values). This is OCP Microscaling (MX):
+ *      E2M1 elements (max 6, emax 2) for Q and K, grouped along head_dim;
+ *      E4M3 elements (max 448, emax 8) for V, grouped along the token axis;
+ *      shared exponent X = floor(log2(amax)) - emax, stored as E8M0 (X + 127);
+ *      element code = round-to-nearest-even(x / 2^X) onto the element grid,
+ *      saturating at the largest finite magnitude.
+ *  - Attention then uses the dequantized values (article §2.3, §3.3): scores
+ *    s = scale * q.k, softmax over the allowed keys, output sum_j p_j v_j.
+ *    Here everything after dequantization is done in fp64, which is the exact
+ *    result up to rounding order.
+ *
+ * Readings taken where the articles are silent:
+ *  - amax is the largest |x| of the group's valid elements (the article's
+ *    "min/max" describes an asymmetric integer scheme; MX uses a symmetric
+ *    amax). floor(log2 amax) comes from frexp, exactly. amax = 0 gives X = -127.
+ *  - X is clamped to [-127, 127]; the E8M0 byte 0xFF is never produced.
+ *  - A zero or a value that rounds to zero keeps the input's sign bit.
+ *  - E2M1 codes are packed two per byte, element 2i in the low nibble.
+ *  - V groups of 32 tokens: a trailing partial group takes its amax over the
+ *    valid tokens only; codes past the valid length are 0, and scale bytes of
+ *    groups with no valid token are 0.
+ *  - Causal masking is bottom-right aligned: query i of Sq attends keys
+ *    j <= i + (L - Sq), where L is that sequence's KV length.
+ *  - GQA: query head h uses KV head h / (Hq / Hkv).
+ *  - A row with no allowed key has output 0 and log-sum-exp -inf.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_E2M1 0
+#define ORACLE_E4M3 1
+
+/* Number of magnitude codes (sign bit excluded) that are finite. */
+static int n_finite_mags(int fmt) { return fmt == ORACLE_E2M1 ? 8 : 127; }
+static int sign_bit(int fmt) { return fmt == ORACLE_E2M1 ? 0x8 : 0x80; }
+static int elem_emax(int fmt) { return fmt == ORACLE_E2M1 ? 2 : 8; }
+
+/* Value of a magnitude code, from the format definition:
+ * E2M1: 2 exponent bits (bias 1), 1 mantissa bit, subnormal when the exponent is 0.
+ * E4M3: 4 exponent bits (bias 7), 3 mantissa bits, subnormal when the exponent
+ *       is 0; magnitude code 0x7F is NaN (OCP "FN" variant: no infinities). */
+static double mag_value(int fmt, int m) {
+    if (fmt == ORACLE_E2M1) {
+        int e = (m >> 1) & 3, f = m & 1;
+        if (e == 0) return f * 0.5;
+        return (1.0 + f / 2.0) * ldexp(1.0, e - 1);
+    } else {
+        if (m == 0x7F) return NAN;
+        int e = (m >> 3) & 15, f = m & 7;
+        if (e == 0) return (f / 8.0) * ldexp(1.0, -6);
+        return (1.0 + f / 8.0) * ldexp(1.0, e - 7);
+    }
+}
+
+double oracle_decode(int fmt, int code) {
+    int sb = sign_bit(fmt);
+    double v = mag_value(fmt, code & (sb - 1));
+    return (code & sb) ? -v : v;
+}
+
+/* Round y onto the element grid: nearest finite magnitude, ties to the code
+ * with an even mantissa LSB (bit 0 of the code), magnitudes beyond the largest
+ * finite value saturate to it. The sign bit is copied from y. */
+int oracle_encode(int fmt, double y) {
+    int sb = sign_bit(fmt);
+    int neg = signbit(y) ? 1 : 0;
+    double a = fabs(y);
+    int nmag = n_finite_mags(fmt);
+    int code;
+    if (a >= mag_value(fmt, nmag - 1)) {
+        code = nmag - 1;
+    } else {
+        /* largest magnitude code lo with value(lo) <= a (binary search). */
+        int lo = 0, hi = nmag - 1;
+        while (hi - lo > 1) {
+            int mid = (lo + hi) / 2;
+            if (mag_value(fmt, mid) <= a) lo = mid; else hi = mid;
+        }
+        double dlo = a - mag_value(fmt, lo);
+        double dhi = mag_value(fmt, hi) - a;
+        if (dlo < dhi) code = lo;
+        else if (dhi < dlo) code = hi;
+        else code = (lo & 1) ? hi : lo;
+    }
+    return code | (neg ? sb : 0);
+}
+
+/* Shared exponent X = floor(log2(amax)) - emax, clamped to [-127, 127]. */
+int oracle_shared_exponent(int fmt, double amax) {
+    if (!(amax > 0.0)) return -127;
+    int e;
+    frexp(amax, &e); /* amax = f * 2^e, f in [0.5, 1): floor(log2 amax) = e - 1 */
+    int X = (e - 1) - elem_emax(fmt);
+    if (X < -127) X = -127;
+    if (X > 127) X = 127;
+    return X;
+}
+
+static inline double bf16_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/*
+ * Quantize rows of bf16 values in groups of 32 along the row.
+ * x       [n_rows][n_cols] bf16 bit patterns
+ * valid   per-row number of valid leading elements (NULL: all n_cols)
+ * codes   [n_rows][n_cols]   one element code per byte (unpacked)
+ * scales  [n_rows][ceil(n_cols/32)] E8M0 bytes
+ */
+int oracle_quantize_rows(const uint16_t *x, int64_t n_rows, int64_t n_cols, const int32_t *valid,
+                         int fmt, uint8_t *codes, uint8_t *scales) {
+    if (!x || !codes || !scales || n_cols <= 0 || n_rows < 0) return -1;
+    const int64_t ng = (n_cols + 31) / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const uint16_t *xr = x + r * n_cols;
+        uint8_t *cr = codes + r * n_cols;
+        uint8_t *sr = scales + r * ng;
+        int64_t nv = valid ? (int64_t)valid[r] : n_cols;
+        if (nv > n_cols) nv = n_cols;
+        if (nv < 0) nv = 0;
+        for (int64_t g = 0; g < ng; ++g) {
+            int64_t c0 = g * 32, c1 = c0 + 32 < n_cols ? c0 + 32 : n_cols;
+            int64_t cv = c1 < nv ? c1 : nv; /* valid end within the group */
+            if (cv <= c0) {
+                sr[g] = 0;
+                for (int64_t c = c0; c < c1; ++c) cr[c] = 0;
+                continue;
+            }
+            double amax = 0.0;
+            for (int64_t c = c0; c < cv; ++c) {
+                double a = fabs(bf16_to_double(xr[c]));
+                if (a > amax) amax = a;
+            }
+            int X = oracle_shared_exponent(fmt, amax);
+            sr[g] = (uint8_t)(X + 127);
+            for (int64_t c = c0; c < cv; ++c) cr[c] = (uint8_t)oracle_encode(fmt, ldexp(bf16_to_double(xr[c]), -X));
+            for (int64_t c = cv; c < c1; ++c) cr[c] = 0;
+        }
+    }
+    return 0;
+}
+
+/* Two E2M1 codes per byte, element 2i in the low nibble; n must be even. */
+int oracle_pack_e2m1(const uint8_t *codes, int64_t n, uint8_t *packed) {
+    if (n % 2) return -1;
+    for (int64_t i = 0; i < n / 2; ++i)
+        packed[i] = (uint8_t)((codes[2 * i] & 0xF) | ((codes[2 * i + 1] & 0xF) << 4));
+    return 0;
+}
+
+/* value = decode(code) * 2^(scale - 127) */
+int oracle_dequantize_rows(const uint8_t *codes, const uint8_t *scales, int64_t n_rows, int64_t n_cols,
+                           int fmt, double *out) {
+    const int64_t ng = (n_cols + 31) / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int64_t c = 0; c < n_cols; ++c)
+            out[r * n_cols + c] = ldexp(oracle_decode(fmt, codes[r * n_cols + c]), (int)scales[r * ng + c / 32] - 127);
+    return 0;
+}
+
+/*
+ * Attention over the dequantized tensors, in fp64.
+ *
+ * qc, qs  [B][Hq][Sq][d] codes, [B][Hq][Sq][d/32] scales   (E2M1)
+ * kc, ks  [B][Hkv][Lk][d] codes, [B][Hkv][Lk][d/32] scales (E2M1)
+ * vc, vs  [B][Hkv][d][Lk] codes, [B][Hkv][d][ceil(Lk/32)] scales (E4M3)
+ * seqlens [B] KV length per sequence (NULL: Lk)
+ * sel     [n_sel][3] rows (b, h_q, i) to compute; NULL computes every row in
+ *         (b, i, h_q) order, n_sel = B*Sq*Hq
+ * out     [n_sel][d]; lse [n_sel] natural-log log-sum-exp of the scaled scores
+ */
+int oracle_attention(const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, const uint8_t *ks,
+                     const uint8_t *vc, const uint8_t *vs, const int32_t *seqlens,
+                     int B, int Hq, int Hkv, int Sq, int Lk, int d, int causal, double scale,
+                     const int32_t *sel, int64_t n_sel, double *out, double *lse) {
+    if (d % 32 || Hkv <= 0 || Hq % Hkv) return -1;
+    const int G = Hq / Hkv;
+    const int dg = d / 32;
+    const int64_t lg = (Lk + 31) / 32;
+    if (!sel) n_sel = (int64_t)B * Sq * Hq;
+    /* Rows grouped by KV unit (b, h_kv) so each unit is dequantized once. */
+    const int64_t n_units = (int64_t)B * Hkv;
+    int64_t *cnt = (int64_t *)calloc((size_t)n_units + 1, sizeof(int64_t));
+    int64_t *order = (int64_t *)malloc((size_t)(n_sel > 0 ? n_sel : 1) * sizeof(int64_t));
+    if (!cnt || !order) { free(cnt); free(order); return -2; }
+    for (int64_t r = 0; r < n_sel; ++r) {
+        int b, h;
+        if (sel) { b = sel[3 * r]; h = sel[3 * r + 1]; }
+        else { b = (int)(r / ((int64_t)Sq * Hq)); h = (int)(r % Hq); }
+        cnt[(int64_t)b * Hkv + h / G + 1]++;
+    }
+    for (int64_t u = 0; u < n_units; ++u) cnt[u + 1] += cnt[u];
+    {
+        int64_t *fillp = (int64_t *)malloc((size_t)n_units * sizeof(int64_t));
+        if (!fillp) { free(cnt); free(order); return -2; }
+        memcpy(fillp, cnt, (size_t)n_units * sizeof(int64_t));
+        for (int64_t r = 0; r < n_sel; ++r) {
+            int b, h;
+            if (sel) { b = sel[3 * r]; h = sel[3 * r + 1]; }
+            else { b = (int)(r / ((int64_t)Sq * Hq)); h = (int)(r % Hq); }
+            order[fillp[(int64_t)b * Hkv + h / G]++] = r;
+        }
+        free(fillp);
+    }
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t u = 0; u < n_units; ++u) {
+        if (cnt[u + 1] == cnt[u]) continue;
+        const int b = (int)(u / Hkv), hk = (int)(u % Hkv);
+        int L = seqlens ? seqlens[b] : Lk;
+        if (L > Lk) L = Lk;
+        if (L < 0) L = 0;
+        double *kd = (double *)malloc((size_t)(L > 0 ? L : 1) * d * sizeof(double));
+        double *vd = (double *)malloc((size_t)(L > 0 ? L : 1) * d * sizeof(double));
+        double *qd = (double *)malloc((size_t)d * sizeof(double));
+        double *p = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
+        if (!kd || !vd || !qd || !p) {
+#pragma omp atomic write
+            err = -2;
+            free(kd); free(vd); free(qd); free(p);
+            continue;
+        }
+        const uint8_t *kcu = kc + (int64_t)u * Lk * d, *ksu = ks + (int64_t)u * Lk * dg;
+        for (int j = 0; j < L; ++j)
+            for (int c = 0; c < d; ++c)
+                kd[(int64_t)j * d + c] = ldexp(oracle_decode(ORACLE_E2M1, kcu[(int64_t)j * d + c]),
+                                               (int)ksu[(int64_t)j * dg + c / 32] - 127);
+        const uint8_t *vcu = vc + (int64_t)u * d * Lk, *vsu = vs + (int64_t)u * d * lg;
+        for (int c = 0; c < d; ++c)
+            for (int j = 0; j < L; ++j)
+                vd[(int64_t)j * d + c] = ldexp(oracle_decode(ORACLE_E4M3, vcu[(int64_t)c * Lk + j]),
+                                               (int)vsu[(int64_t)c * lg + j / 32] - 127);
+        for (int64_t oi = cnt[u]; oi < cnt[u + 1]; ++oi) {
+            const int64_t r = order[oi];
+            int h, i;
+            if (sel) { h = sel[3 * r + 1]; i = sel[3 * r + 2]; }
+            else { i = (int)((r / Hq) % Sq); h = (int)(r % Hq); }
+            const int64_t qrow = (((int64_t)b * Hq + h) * Sq + i);
+            for (int c = 0; c < d; ++c)
+                qd[c] = ldexp(oracle_decode(ORACLE_E2M1, qc[qrow * d + c]), (int)qs[qrow * dg + c / 32] - 127);
+            int jmax = L; /* exclusive bound on allowed keys */
+            if (causal) {
+                int lim = i + (L - Sq) + 1;
+                if (lim < jmax) jmax = lim;
+            }
+            if (jmax < 0) jmax = 0;
+            double *o = out + r * d;
+            if (jmax == 0) {
+                for (int c = 0; c < d; ++c) o[c] = 0.0;
+                if (lse) lse[r] = -INFINITY;
+                continue;
+            }
+            double m = -INFINITY;
+            for (int j = 0; j < jmax; ++j) {
+                double s = 0.0;
+                const double *kr = kd + (int64_t)j * d;
+                for (int c = 0; c < d; ++c) s += qd[c] * kr[c];
+                s *= scale;
+                p[j] = s;
+                if (s > m) m = s;
+            }
+            double l = 0.0;
+            for (int j = 0; j < jmax; ++j) { p[j] = exp(p[j] - m); l += p[j]; }
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            for (int j = 0; j < jmax; ++j) {
+                const double w = p[j] / l;
+                const double *vr = vd + (int64_t)j * d;
+                for (int c = 0; c < d; ++c) o[c] += w * vr[c];
+            }
+            if (lse) lse[r] = m + log(l);
+        }
+        free(kd); free(vd); free(qd); free(p);
+    }
+    free(cnt);
+    free(order);
+    return err;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
