@@ -1,0 +1,197 @@
+"""QK4V8 mixed-precision attention for B200 (sm_100a).
+
+This is the Python binding of libqk4v8.so. It marshals arguments only: torch
+provides device memory and the current stream, and every step of the
+computation runs in the library's CUDA kernels. Function names follow the C
+entry points in include/qk4v8.h.
+
+Method (MpFA QK4V8 article, mhpn.cn):
+  - Q and K are quantized to MXFP4 and V to MXFP8-E4M3, with one E8M0 scale
+    per 32 values computed online.
+  - Attention then runs tile by tile with an FP32 online softmax, on
+    block-scaled tcgen05 tensor-core MMAs.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from ._lib import QK4V8Error, check, lib
+
+__all__ = [
+    "MXFP4", "MXFP8V", "QK4V8Error", "lib", "round_cap",
+    "quantize_qk", "quantize_v", "quantize", "attention_prefill", "attention_decode",
+    "decode_workspace_bytes", "decode_default_splits",
+]
+
+D = 128
+
+
+def round_cap(n: int) -> int:
+    """Smallest multiple of 128 that holds n tokens (at least 128)."""
+    return max(128, (int(n) + 127) // 128 * 128)
+
+
+@dataclass
+class MXFP4:
+    """Packed MXFP4 tensor (Q or K): codes uint8 [B][H][cap][64], scales uint8 [B][H][cap/128][512]."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    B: int
+    H: int
+    cap: int
+    length: int
+
+
+@dataclass
+class MXFP8V:
+    """Packed MXFP8-E4M3 V: codes uint8 [B][H][128][cap], scales uint8 [B][H][cap/128][512]."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    B: int
+    H: int
+    cap: int
+    length: int
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_bf16(x: torch.Tensor, name: str):
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 4 or x.shape[-1] != D or x.stride(-1) != 1:
+        raise ValueError(f"{name} must be a CUDA bf16 tensor [B, T, H, 128] with unit channel stride")
+
+
+def _seqlens(seqlens, B, device):
+    if seqlens is None:
+        return None
+    if not torch.is_tensor(seqlens):
+        seqlens = torch.tensor(seqlens, dtype=torch.int32)
+    seqlens = seqlens.to(device=device, dtype=torch.int32).contiguous()
+    if seqlens.numel() != B:
+        raise ValueError("seqlens must have B entries")
+    return seqlens
+
+
+def quantize_qk(x: torch.Tensor, cap: Optional[int] = None, seqlens=None, out: Optional[MXFP4] = None) -> MXFP4:
+    """MXFP4-quantize Q or K ([B, T, H, 128] bf16) into the packed layout."""
+    _check_bf16(x, "x")
+    B, T, H, _ = x.shape
+    cap = round_cap(T) if cap is None else int(cap)
+    sl = _seqlens(seqlens, B, x.device)
+    if out is None:
+        out = MXFP4(torch.empty((B, H, cap, 64), dtype=torch.uint8, device=x.device),
+                    torch.empty((B, H, cap // 128, 512), dtype=torch.uint8, device=x.device), B, H, cap, T)
+    check(lib().qk4v8_quantize_qk(x.data_ptr(), B, T, H, D, x.stride(0), x.stride(1), x.stride(2), _ptr(sl), cap,
+                                  out.codes.data_ptr(), out.scales.data_ptr(), _stream(x.device)), "qk4v8_quantize_qk")
+    out.length = T
+    return out
+
+
+def quantize_v(v: torch.Tensor, cap: Optional[int] = None, seqlens=None, out: Optional[MXFP8V] = None) -> MXFP8V:
+    """MXFP8-E4M3-quantize V ([B, T, H, 128] bf16), groups of 32 along T."""
+    _check_bf16(v, "v")
+    B, T, H, _ = v.shape
+    cap = round_cap(T) if cap is None else int(cap)
+    sl = _seqlens(seqlens, B, v.device)
+    if out is None:
+        out = MXFP8V(torch.empty((B, H, D, cap), dtype=torch.uint8, device=v.device),
+                     torch.empty((B, H, cap // 128, 512), dtype=torch.uint8, device=v.device), B, H, cap, T)
+    check(lib().qk4v8_quantize_v(v.data_ptr(), B, T, H, D, v.stride(0), v.stride(1), v.stride(2), _ptr(sl), cap,
+                                 out.codes.data_ptr(), out.scales.data_ptr(), _stream(v.device)), "qk4v8_quantize_v")
+    out.length = T
+    return out
+
+
+def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seqlens_k=None, q_cap=None, kv_cap=None):
+    """Quantize contiguous Q [B,Sq,Hq,128], K and V [B,Sk,Hkv,128] in one library call."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous for qk4v8_quantize")
+    B, Sq, Hq, _ = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    q_cap = round_cap(Sq) if q_cap is None else int(q_cap)
+    kv_cap = round_cap(Sk) if kv_cap is None else int(kv_cap)
+    dev = q.device
+    sl = _seqlens(seqlens_k, B, dev)
+    qp = MXFP4(torch.empty((B, Hq, q_cap, 64), dtype=torch.uint8, device=dev),
+               torch.empty((B, Hq, q_cap // 128, 512), dtype=torch.uint8, device=dev), B, Hq, q_cap, Sq)
+    kp = MXFP4(torch.empty((B, Hkv, kv_cap, 64), dtype=torch.uint8, device=dev),
+               torch.empty((B, Hkv, kv_cap // 128, 512), dtype=torch.uint8, device=dev), B, Hkv, kv_cap, Sk)
+    vp = MXFP8V(torch.empty((B, Hkv, D, kv_cap), dtype=torch.uint8, device=dev),
+                torch.empty((B, Hkv, kv_cap // 128, 512), dtype=torch.uint8, device=dev), B, Hkv, kv_cap, Sk)
+    check(lib().qk4v8_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Sq, Sk, Hq, Hkv, D, _ptr(sl), q_cap,
+                               kv_cap, qp.codes.data_ptr(), qp.scales.data_ptr(), kp.codes.data_ptr(),
+                               kp.scales.data_ptr(), vp.codes.data_ptr(), vp.scales.data_ptr(), _stream(dev)),
+          "qk4v8_quantize")
+    return qp, kp, vp
+
+
+def attention_prefill(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k=None, causal: bool = True,
+                      softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                      lse: Optional[torch.Tensor] = None, return_lse: bool = False,
+                      dev_status: Optional[torch.Tensor] = None):
+    """QK4V8 prefill attention. Returns out bf16 [B, Sq, Hq, 128] (and lse [B, Hq, Sq])."""
+    dev = q.codes.device
+    B, Hq, Sq = q.B, q.H, q.length
+    sl = _seqlens(seqlens_k, B, dev)
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=torch.bfloat16, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+    check(lib().qk4v8_attention_prefill(q.codes.data_ptr(), q.scales.data_ptr(), B, Hq, Sq, q.cap,
+                                        k.codes.data_ptr(), k.scales.data_ptr(), v.codes.data_ptr(),
+                                        v.scales.data_ptr(), k.H, k.length, k.cap, _ptr(sl), int(bool(causal)),
+                                        float(softmax_scale or 0.0), out.data_ptr(), _ptr(lse), _ptr(dev_status),
+                                        _stream(dev)), "qk4v8_attention_prefill")
+    return (out, lse) if return_lse else out
+
+
+def decode_workspace_bytes(B: int, Hq: int, nq: int, num_splits: int) -> int:
+    return int(lib().qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits))
+
+
+def decode_default_splits(B: int, Hkv: int, max_seqlen: int) -> int:
+    return int(lib().qk4v8_decode_default_splits(B, Hkv, max_seqlen))
+
+
+def attention_decode(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optional[int] = None,
+                     causal_in_block: bool = True, softmax_scale: Optional[float] = None, num_splits: int = 0,
+                     workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, return_lse: bool = False,
+                     dev_status: Optional[torch.Tensor] = None):
+    """Split-KV decode / speculative verify over a packed cache. Returns out bf16 [B, nq, Hq, 128]."""
+    dev = q.codes.device
+    B, Hq, nq = q.B, q.H, q.length
+    sl = _seqlens(seqlens_k, B, dev)
+    if max_seqlen is None:
+        max_seqlen = k.cap
+    splits = num_splits if num_splits > 0 else decode_default_splits(B, k.H, max_seqlen)
+    need = decode_workspace_bytes(B, Hq, nq, splits)
+    if workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((B, nq, Hq, D), dtype=torch.bfloat16, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, nq), dtype=torch.float32, device=dev)
+    check(lib().qk4v8_attention_decode(q.codes.data_ptr(), q.scales.data_ptr(), B, Hq, nq, q.cap,
+                                       k.codes.data_ptr(), k.scales.data_ptr(), v.codes.data_ptr(),
+                                       v.scales.data_ptr(), k.H, k.cap, _ptr(sl), int(max_seqlen),
+                                       int(bool(causal_in_block)), float(softmax_scale or 0.0), int(splits),
+                                       workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                       out.data_ptr(), _ptr(lse), _ptr(dev_status), _stream(dev)),
+          "qk4v8_attention_decode")
+    return (out, lse) if return_lse else out
+
+
+def default_scale() -> float:
+    return 1.0 / math.sqrt(D)

@@ -1,0 +1,327 @@
+// extern "C" entry points of libqk4v8.so: argument validation, TMA descriptor
+// construction and kernel launches. See include/qk4v8.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qk4v8.h"
+#include "../../include/qk4v8_test.h"
+#include "qk4v8_internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+int g_test_stall = 0;
+float *g_test_dump_s = nullptr;
+
+int set_error(int status, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int cuda_error(cudaError_t e, const char *what) {
+    return set_error(QK4V8_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// sm_100 check, cached per device.
+int check_device() {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
+    return qk4v8_device_supported(dev);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// K codes [B*Hkv][cap][64] as a 3-D uint8 tensor, 128-token x 64-byte boxes,
+// 64-byte swizzle (one token row is exactly one swizzle span).
+int make_k_map(CUtensorMap *map, const uint8_t *codes, int BH, int cap) {
+    auto enc = get_encode_fn();
+    if (!enc) return set_error(QK4V8_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(cap), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {64, static_cast<cuuint64_t>(cap) * 64};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(codes), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(QK4V8_ERR_CUDA, "cuTensorMapEncodeTiled(K) failed (%d)", int(r));
+    return QK4V8_OK;
+}
+
+// V codes [B*Hkv][128][cap] as a 3-D uint8 tensor, 128-token x 128-channel
+// boxes, 128-byte swizzle.
+int make_v_map(CUtensorMap *map, const uint8_t *codes, int BH, int cap) {
+    auto enc = get_encode_fn();
+    if (!enc) return set_error(QK4V8_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cap), 128, static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(cap), static_cast<cuuint64_t>(cap) * 128};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(codes), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(QK4V8_ERR_CUDA, "cuTensorMapEncodeTiled(V) failed (%d)", int(r));
+    return QK4V8_OK;
+}
+
+int validate_quant_args(const void *x, int B, int S, int H, int d, int64_t sb, int64_t ss, int64_t sh, int cap,
+                        const uint8_t *codes, const uint8_t *scales) {
+    if (!x || !codes || !scales) return set_error(QK4V8_ERR_INVALID_ARG, "null pointer");
+    if (d != 128) return set_error(QK4V8_ERR_INVALID_ARG, "head_dim must be 128 (got %d)", d);
+    if (B <= 0 || S < 0 || H <= 0) return set_error(QK4V8_ERR_INVALID_ARG, "bad shape B=%d S=%d H=%d", B, S, H);
+    if (cap <= 0 || cap % 128 || cap < S)
+        return set_error(QK4V8_ERR_INVALID_ARG, "cap must be a positive multiple of 128 and >= S (cap=%d S=%d)", cap,
+                         S);
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales))
+        return set_error(QK4V8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    if (sb % 8 || ss % 8 || sh % 8 || sb < 0 || ss < 0 || sh < 0)
+        return set_error(QK4V8_ERR_INVALID_ARG, "strides must be non-negative multiples of 8 elements");
+    return QK4V8_OK;
+}
+
+int validate_packed(const uint8_t *codes, const uint8_t *scales, const char *what) {
+    if (!codes || !scales) return set_error(QK4V8_ERR_INVALID_ARG, "null %s pointer", what);
+    if (!aligned16(codes) || !aligned16(scales))
+        return set_error(QK4V8_ERR_INVALID_ARG, "%s buffers must be 16-byte aligned", what);
+    return QK4V8_OK;
+}
+
+float resolve_scale(float s) { return s > 0.f ? s : 1.0f / std::sqrt(128.0f); }
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace
+
+extern "C" {
+
+const char *qk4v8_status_string(int status) {
+    switch (status) {
+        case QK4V8_OK: return "ok";
+        case QK4V8_ERR_INVALID_ARG: return "invalid argument";
+        case QK4V8_ERR_UNSUPPORTED: return "unsupported device (needs sm_100)";
+        case QK4V8_ERR_CUDA: return "CUDA error";
+        case QK4V8_ERR_TIMEOUT: return "device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+const char *qk4v8_last_error(void) { return g_last_error; }
+
+int qk4v8_device_supported(int device) {
+    int major = 0, minor = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+    if (e != cudaSuccess) return cuda_error(e, "cudaDeviceGetAttribute");
+    e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device);
+    if (e != cudaSuccess) return cuda_error(e, "cudaDeviceGetAttribute");
+    if (major != 10 || minor != 0)
+        return set_error(QK4V8_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", device,
+                         major, minor);
+    return QK4V8_OK;
+}
+
+size_t qk4v8_mxfp4_codes_bytes(int B, int H, int cap) {
+    return static_cast<size_t>(B) * H * cap * 64;
+}
+size_t qk4v8_mxfp8_codes_bytes(int B, int H, int cap) {
+    return static_cast<size_t>(B) * H * 128 * cap;
+}
+size_t qk4v8_scales_bytes(int B, int H, int cap) {
+    return static_cast<size_t>(B) * H * (cap / 128) * 512;
+}
+
+int qk4v8_quantize_qk(const void *x, int B, int S, int H, int d, int64_t stride_b, int64_t stride_s,
+                      int64_t stride_h, const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
+                      void *stream) {
+    int st = validate_quant_args(x, B, S, H, d, stride_b, stride_s, stride_h, cap, codes, scales);
+    if (st) return st;
+    if ((st = check_device())) return st;
+    cudaError_t e = qk4v8::launch_quantize_qk(x, B, S, H, stride_b, stride_s, stride_h, seqlens, cap, codes, scales,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "quantize_qk launch");
+}
+
+int qk4v8_quantize_v(const void *v, int B, int S, int H, int d, int64_t stride_b, int64_t stride_s,
+                     int64_t stride_h, const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
+                     void *stream) {
+    int st = validate_quant_args(v, B, S, H, d, stride_b, stride_s, stride_h, cap, codes, scales);
+    if (st) return st;
+    if ((st = check_device())) return st;
+    cudaError_t e = qk4v8::launch_quantize_v(v, B, S, H, stride_b, stride_s, stride_h, seqlens, cap, codes, scales,
+                                             static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "quantize_v launch");
+}
+
+int qk4v8_quantize(const void *q, const void *k, const void *v, int B, int Sq, int Sk, int Hq, int Hkv, int d,
+                   const int32_t *seqlens_k, int q_cap, int kv_cap, uint8_t *q_codes, uint8_t *q_scales,
+                   uint8_t *k_codes, uint8_t *k_scales, uint8_t *v_codes, uint8_t *v_scales, void *stream) {
+    const int64_t qs = static_cast<int64_t>(Hq) * 128, ks = static_cast<int64_t>(Hkv) * 128;
+    int st = qk4v8_quantize_qk(q, B, Sq, Hq, d, qs * Sq, qs, 128, nullptr, q_cap, q_codes, q_scales, stream);
+    if (st) return st;
+    st = qk4v8_quantize_qk(k, B, Sk, Hkv, d, ks * Sk, ks, 128, seqlens_k, kv_cap, k_codes, k_scales, stream);
+    if (st) return st;
+    return qk4v8_quantize_v(v, B, Sk, Hkv, d, ks * Sk, ks, 128, seqlens_k, kv_cap, v_codes, v_scales, stream);
+}
+
+int qk4v8_attention_prefill(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int Sq, int q_cap,
+                            const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
+                            const uint8_t *v_scales, int Hkv, int Sk, int kv_cap, const int32_t *seqlens_k,
+                            int causal, float softmax_scale, void *out, float *lse, int32_t *dev_status,
+                            void *stream) {
+    int st;
+    if ((st = validate_packed(q_codes, q_scales, "Q")) || (st = validate_packed(k_codes, k_scales, "K")) ||
+        (st = validate_packed(v_codes, v_scales, "V")))
+        return st;
+    if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv)
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad heads B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
+    if (Sq <= 0 || q_cap % 128 || q_cap < Sq || kv_cap <= 0 || kv_cap % 128 || Sk < 0 || Sk > kv_cap)
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad lengths Sq=%d q_cap=%d Sk=%d kv_cap=%d", Sq, q_cap, Sk, kv_cap);
+    if ((st = check_device())) return st;
+    CUtensorMap tk, tv;
+    if ((st = make_k_map(&tk, k_codes, B * Hkv, kv_cap)) || (st = make_v_map(&tv, v_codes, B * Hkv, kv_cap)))
+        return st;
+    qk4v8::AttnParams p{};
+    p.q_codes = q_codes;
+    p.q_scales = q_scales;
+    p.k_scales = k_scales;
+    p.v_scales = v_scales;
+    p.seqlens = seqlens_k;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.Sq = Sq;
+    p.q_cap = q_cap;
+    p.kv_cap = kv_cap;
+    p.Lk = Sk;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = resolve_scale(softmax_scale) * kLog2e;
+    p.decode = 0;
+    p.n_qtiles = (Sq + 127) / 128;
+    p.num_splits = 1;
+    p.split_tiles = 0;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.lse = lse;
+    p.status = dev_status;
+    p.test_stall = g_test_stall;
+    p.test_dump_s = g_test_dump_s;
+    const int grid = B * Hq * p.n_qtiles;
+    cudaError_t e = qk4v8::launch_attention(tk, tv, p, grid, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "attention (prefill) launch");
+}
+
+size_t qk4v8_decode_workspace_bytes(int B, int Hq, int nq, int num_splits) {
+    if (B <= 0 || Hq <= 0 || nq <= 0 || num_splits <= 0) return 0;
+    const size_t rows = static_cast<size_t>(B) * Hq * nq * num_splits;
+    return rows * 128 * sizeof(float) + rows * sizeof(float);
+}
+
+int qk4v8_decode_default_splits(int B, int Hkv, int max_seqlen) {
+    // Enough CTAs for about two waves of 148 SMs, but no split shorter than
+    // 16 tiles of 128 keys.
+    const int units = B > 0 && Hkv > 0 ? B * Hkv : 1;
+    const int tiles = max_seqlen > 0 ? (max_seqlen + 127) / 128 : 1;
+    int splits = (2 * 148 + units - 1) / units;
+    const int max_by_len = tiles / 16 > 0 ? tiles / 16 : 1;
+    if (splits > max_by_len) splits = max_by_len;
+    if (splits < 1) splits = 1;
+    return splits;
+}
+
+int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
+                           const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
+                           const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
+                           int causal_in_block, float softmax_scale, int num_splits, void *workspace,
+                           size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, void *stream) {
+    int st;
+    if ((st = validate_packed(q_codes, q_scales, "Q")) || (st = validate_packed(k_codes, k_scales, "K")) ||
+        (st = validate_packed(v_codes, v_scales, "V")))
+        return st;
+    if (!seqlens_k) return set_error(QK4V8_ERR_INVALID_ARG, "decode needs seqlens_k");
+    if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv)
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad heads B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
+    if (nq < 1 || nq > 8 || (Hq / Hkv) * nq > 128)
+        return set_error(QK4V8_ERR_INVALID_ARG, "need 1 <= nq <= 8 and (Hq/Hkv)*nq <= 128 (nq=%d G=%d)", nq,
+                         Hq / Hkv);
+    if (q_cap <= 0 || q_cap % 128 || q_cap < nq || kv_cap <= 0 || kv_cap % 128 || max_seqlen < 0 ||
+        max_seqlen > kv_cap)
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad lengths q_cap=%d kv_cap=%d max_seqlen=%d", q_cap, kv_cap,
+                         max_seqlen);
+    if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
+    const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hkv, max_seqlen);
+    const size_t need = qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need)
+        return set_error(QK4V8_ERR_INVALID_ARG, "workspace must be 16-byte aligned and >= %zu bytes", need);
+    if ((st = check_device())) return st;
+    CUtensorMap tk, tv;
+    if ((st = make_k_map(&tk, k_codes, B * Hkv, kv_cap)) || (st = make_v_map(&tv, v_codes, B * Hkv, kv_cap)))
+        return st;
+    const int tiles = (max_seqlen + 127) / 128;
+    qk4v8::AttnParams p{};
+    p.q_codes = q_codes;
+    p.q_scales = q_scales;
+    p.k_scales = k_scales;
+    p.v_scales = v_scales;
+    p.seqlens = seqlens_k;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.Sq = nq;
+    p.q_cap = q_cap;
+    p.kv_cap = kv_cap;
+    p.Lk = max_seqlen;
+    p.causal = causal_in_block ? 1 : 0;
+    p.scale_log2 = resolve_scale(softmax_scale) * kLog2e;
+    p.decode = 1;
+    p.n_qtiles = 1;
+    p.num_splits = splits;
+    p.split_tiles = tiles > 0 ? (tiles + splits - 1) / splits : 1;
+    const size_t rows = static_cast<size_t>(B) * Hq * nq * splits;
+    p.ws_o = static_cast<float *>(workspace);
+    p.ws_lse = p.ws_o + rows * 128;
+    p.status = dev_status;
+    p.test_stall = g_test_stall;
+    p.test_dump_s = g_test_dump_s;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = qk4v8::launch_attention(tk, tv, p, B * Hkv * splits, s);
+    if (e != cudaSuccess) return cuda_error(e, "attention (decode) launch");
+    e = qk4v8::launch_decode_merge(p.ws_o, p.ws_lse, B, Hq, nq, splits, static_cast<__nv_bfloat16 *>(out), lse, s);
+    return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "decode merge launch");
+}
+
+// Test hook (declared in include/qk4v8_test.h): while enabled, attention
+// launches withhold the producer's Q-ready signal so the pipeline's bounded
+// waits expire and report QK4V8_ERR_TIMEOUT through dev_status.
+void qk4v8_test_set_stall(int enable) { g_test_stall = enable ? 1 : 0; }
+
+// Test hook (declared in include/qk4v8_test.h): while set, CTA 0 of each
+// attention launch writes its first raw score tile to `dev_ptr`.
+void qk4v8_test_set_dump_scores(float *dev_ptr) { g_test_dump_s = dev_ptr; }
+
+}  // extern "C"

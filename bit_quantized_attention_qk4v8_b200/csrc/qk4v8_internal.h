@@ -1,0 +1,51 @@
+// Internal declarations shared by the CUDA translation units of libqk4v8.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace qk4v8 {
+
+// Limit on any single pipeline wait inside a kernel before it gives up, sets
+// the timeout status and unwinds (nanoseconds).
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;
+
+struct AttnParams {
+    const uint8_t *q_codes;   // [B][Hq][q_cap][64]
+    const uint8_t *q_scales;  // [B][Hq][q_cap/128][512]
+    const uint8_t *k_scales;  // [B][Hkv][kv_cap/128][512]
+    const uint8_t *v_scales;  // [B][Hkv][kv_cap/128][512]
+    const int32_t *seqlens;   // [B] or null
+    int B, Hq, Hkv, G;
+    int Sq;                   // query tokens per sequence (prefill length, or nq when decoding)
+    int q_cap, kv_cap;
+    int Lk;                   // KV length when seqlens is null
+    int causal;
+    float scale_log2;         // softmax_scale * log2(e)
+    int decode;               // 0: units (b, h_q, q tile); 1: units (b, h_kv, split)
+    int n_qtiles;
+    int num_splits, split_tiles;
+    __nv_bfloat16 *out;       // prefill [B][Sq][Hq][128]
+    float *lse;               // prefill [B][Hq][Sq] (natural log), nullable
+    float *ws_o;              // decode partial outputs [B][Hq][nq][splits][128]
+    float *ws_lse;            // decode partial log2-sum-exp [B][Hq][nq][splits]
+    int32_t *status;          // nullable
+    int test_stall;           // test hook: the producer withholds the Q-ready signal
+    float *test_dump_s;       // test hook: CTA 0 writes its first raw score tile [128 lanes][128 keys]
+};
+
+cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
+                               const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
+                               cudaStream_t stream);
+cudaError_t launch_quantize_v(const void *v, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
+                              const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
+                              cudaStream_t stream);
+cudaError_t launch_attention(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p,
+                             int grid, cudaStream_t stream);
+cudaError_t launch_decode_merge(const float *ws_o, const float *ws_lse, int B, int Hq, int nq, int splits,
+                                __nv_bfloat16 *out, float *lse, cudaStream_t stream);
+
+}  // namespace qk4v8

