@@ -24,7 +24,7 @@ from ._lib import QK4V8Error, check, lib
 __all__ = [
     "MXFP4", "MXFP8V", "QK4V8Error", "lib", "round_cap",
     "quantize_qk", "quantize_v", "quantize", "attention_prefill", "attention_decode",
-    "decode_workspace_bytes", "decode_default_splits",
+    "decode_workspace_bytes", "decode_default_splits", "attention_decode_splitkv", "decode_merge",
 ]
 
 D = 128
@@ -191,6 +191,28 @@ def attention_decode(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optio
                                        out.data_ptr(), _ptr(lse), _ptr(dev_status), _stream(dev)),
           "qk4v8_attention_decode")
     return (out, lse) if return_lse else out
+
+
+def attention_decode_splitkv(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k: torch.Tensor, max_seqlen: int,
+                             num_splits: int, workspace: torch.Tensor, causal_in_block: bool = True,
+                             softmax_scale: Optional[float] = None, dev_status: Optional[torch.Tensor] = None):
+    """First decode stage: per-split partial (O, lse2) into `workspace` (num_splits must be > 0)."""
+    dev = q.codes.device
+    check(lib().qk4v8_attention_decode_splitkv(q.codes.data_ptr(), q.scales.data_ptr(), q.B, q.H, q.length, q.cap,
+                                               k.codes.data_ptr(), k.scales.data_ptr(), v.codes.data_ptr(),
+                                               v.scales.data_ptr(), k.H, k.cap, seqlens_k.data_ptr(),
+                                               int(max_seqlen), int(bool(causal_in_block)),
+                                               float(softmax_scale or 0.0), int(num_splits), workspace.data_ptr(),
+                                               workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                                               _stream(dev)), "qk4v8_attention_decode_splitkv")
+
+
+def decode_merge(workspace: torch.Tensor, B: int, Hq: int, nq: int, num_splits: int, out: torch.Tensor,
+                 lse: Optional[torch.Tensor] = None):
+    """Second decode stage: merge the split partials into out bf16 [B, nq, Hq, 128]."""
+    check(lib().qk4v8_decode_merge(workspace.data_ptr(), workspace.numel() * workspace.element_size(), B, Hq, nq,
+                                   num_splits, out.data_ptr(), _ptr(lse), _stream(out.device)), "qk4v8_decode_merge")
+    return out
 
 
 def default_scale() -> float:

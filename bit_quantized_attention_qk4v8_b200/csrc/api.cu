@@ -252,17 +252,22 @@ int qk4v8_decode_default_splits(int B, int Hkv, int max_seqlen) {
     return splits;
 }
 
-int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
-                           const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
-                           const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
-                           int causal_in_block, float softmax_scale, int num_splits, void *workspace,
-                           size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Validates decode arguments, builds the tensor maps and launches the split-KV
+// kernel; the caller decides whether the merge follows.
+int decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
+                   const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes, const uint8_t *v_scales,
+                   int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen, int causal_in_block,
+                   float softmax_scale, int num_splits, void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                   cudaStream_t stream, int *splits_used) {
     int st;
     if ((st = validate_packed(q_codes, q_scales, "Q")) || (st = validate_packed(k_codes, k_scales, "K")) ||
         (st = validate_packed(v_codes, v_scales, "V")))
         return st;
     if (!seqlens_k) return set_error(QK4V8_ERR_INVALID_ARG, "decode needs seqlens_k");
-    if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv)
         return set_error(QK4V8_ERR_INVALID_ARG, "bad heads B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
     if (nq < 1 || nq > 8 || (Hq / Hkv) * nq > 128)
@@ -308,11 +313,59 @@ int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int 
     p.status = dev_status;
     p.test_stall = g_test_stall;
     p.test_dump_s = g_test_dump_s;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = qk4v8::launch_attention(tk, tv, p, B * Hkv * splits, s);
+    cudaError_t e = qk4v8::launch_attention(tk, tv, p, B * Hkv * splits, stream);
     if (e != cudaSuccess) return cuda_error(e, "attention (decode) launch");
-    e = qk4v8::launch_decode_merge(p.ws_o, p.ws_lse, B, Hq, nq, splits, static_cast<__nv_bfloat16 *>(out), lse, s);
+    *splits_used = splits;
+    return QK4V8_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qk4v8_attention_decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
+                                   const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
+                                   const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k,
+                                   int max_seqlen, int causal_in_block, float softmax_scale, int num_splits,
+                                   void *workspace, size_t workspace_bytes, int32_t *dev_status, void *stream) {
+    int splits = 0;
+    return decode_splitkv(q_codes, q_scales, B, Hq, nq, q_cap, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap,
+                          seqlens_k, max_seqlen, causal_in_block, softmax_scale, num_splits, workspace,
+                          workspace_bytes, dev_status, static_cast<cudaStream_t>(stream), &splits);
+}
+
+int qk4v8_decode_merge(const void *workspace, size_t workspace_bytes, int B, int Hq, int nq, int num_splits,
+                       void *out, float *lse, void *stream) {
+    if (!workspace || !aligned16(workspace) || !out || !aligned16(out))
+        return set_error(QK4V8_ERR_INVALID_ARG, "workspace and out must be 16-byte aligned pointers");
+    if (B <= 0 || Hq <= 0 || nq < 1 || nq > 8 || num_splits < 1)
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad merge sizes B=%d Hq=%d nq=%d splits=%d", B, Hq, nq,
+                         num_splits);
+    if (workspace_bytes < qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits))
+        return set_error(QK4V8_ERR_INVALID_ARG, "workspace smaller than %zu bytes",
+                         qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits));
+    int st;
+    if ((st = check_device())) return st;
+    const size_t rows = static_cast<size_t>(B) * Hq * nq * num_splits;
+    const float *ws_o = static_cast<const float *>(workspace);
+    cudaError_t e = qk4v8::launch_decode_merge(ws_o, ws_o + rows * 128, B, Hq, nq, num_splits,
+                                               static_cast<__nv_bfloat16 *>(out), lse,
+                                               static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "decode merge launch");
+}
+
+int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
+                           const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
+                           const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
+                           int causal_in_block, float softmax_scale, int num_splits, void *workspace,
+                           size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, void *stream) {
+    if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
+    int splits = 0;
+    int st = decode_splitkv(q_codes, q_scales, B, Hq, nq, q_cap, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap,
+                            seqlens_k, max_seqlen, causal_in_block, softmax_scale, num_splits, workspace,
+                            workspace_bytes, dev_status, static_cast<cudaStream_t>(stream), &splits);
+    if (st) return st;
+    return qk4v8_decode_merge(workspace, workspace_bytes, B, Hq, nq, splits, out, lse, stream);
 }
 
 // Test hook (declared in include/qk4v8_test.h): while enabled, attention

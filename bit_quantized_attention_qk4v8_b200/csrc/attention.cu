@@ -121,9 +121,10 @@ struct Unit {
     int b, h_kv, h_q, q0, R, L, tile_begin, tile_end, split;
 };
 
+template <bool kDecode>
 __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
     Unit u;
-    if (!p.decode) {
+    if (!kDecode) {
         const int per = p.B * p.Hq;
         const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / per;  // longest (causal) first
         const int rem = static_cast<int>(blockIdx.x) % per;
@@ -164,10 +165,11 @@ struct RowInfo {
     int h, i, limit;
 };
 
+template <bool kDecode>
 __device__ __forceinline__ RowInfo row_info(const AttnParams &p, const Unit &u, int lane) {
     RowInfo r;
     int idx;
-    if (!p.decode) {
+    if (!kDecode) {
         idx = lane;
         r.h = u.h_q;
         r.i = u.q0 + lane;
@@ -190,9 +192,10 @@ __device__ __forceinline__ float exp2_approx(float x) {
 }
 
 // Writes the result of a row that saw no key at all.
+template <bool kDecode>
 __device__ __forceinline__ void write_empty_row(const AttnParams &p, const Unit &u, const RowInfo &r) {
     if (!r.valid) return;
-    if (!p.decode) {
+    if (!kDecode) {
         uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((static_cast<int64_t>(u.b) * p.Sq + r.i) * p.Hq + r.h) * 128);
 #pragma unroll
         for (int q = 0; q < 16; ++q) dst[q] = make_uint4(0, 0, 0, 0);
@@ -208,6 +211,7 @@ __device__ __forceinline__ void write_empty_row(const AttnParams &p, const Unit 
 
 }  // namespace
 
+template <bool kDecode>
 __global__ void __launch_bounds__(kThreads, 1)
     qk4v8_attention_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                            const AttnParams p) {
@@ -216,10 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    const Unit u = decode_unit(p);
+    const Unit u = decode_unit<kDecode>(p);
     const int T = u.tile_end - u.tile_begin;
     if (T <= 0 || (p.status && *reinterpret_cast<const volatile int32_t *>(p.status) != 0)) {
-        if (warp >= 2) write_empty_row(p, u, row_info(p, u, ((warp & 3) << 5) | lane));
+        if (warp >= 2) write_empty_row<kDecode>(p, u, row_info<kDecode>(p, u, ((warp & 3) << 5) | lane));
         return;
     }
 
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *qs = smem + kQOff;
         for (int c = lane; c < 512; c += 32) {
             const int row = c >> 2, j = c & 3;
-            const RowInfo r = row_info(p, u, row);
+            const RowInfo r = row_info<kDecode>(p, u, row);
             uint4 val = make_uint4(0, 0, 0, 0);
             if (r.valid)
                 val = *reinterpret_cast<const uint4 *>(
@@ -285,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4 *>(qs + row * 64 + ((j ^ ((row >> 1) & 3)) << 4)) = val;
         }
         for (int row = lane; row < 128; row += 32) {
-            const RowInfo r = row_info(p, u, row);
+            const RowInfo r = row_info<kDecode>(p, u, row);
             uint32_t sc = 0;
             if (r.valid)
                 sc = *reinterpret_cast<const uint32_t *>(
@@ -419,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------- softmax
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        const RowInfo r = row_info(p, u, row);
+        const RowInfo r = row_info<kDecode>(p, u, row);
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         uint8_t *phi = smem + kPhiOff + row * 128;
         uint8_t *plo = smem + kPloOff + row * 128;
@@ -558,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool any = l > 0.f && m_ref > -INFINITY;
                 const float inv = any ? 1.f / l : 0.f;
                 const float lse2 = any ? m_ref + log2f(l) : -INFINITY;
-                if (!p.decode) {
+                if (!kDecode) {
                     uint4 *dst = reinterpret_cast<uint4 *>(
                         p.out + ((static_cast<int64_t>(u.b) * p.Sq + r.i) * p.Hq + r.h) * 128);
 #pragma unroll
@@ -644,14 +648,25 @@ __global__ void __launch_bounds__(256) qk4v8_decode_merge_kernel(const float *__
 
 cudaError_t launch_attention(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p, int grid,
                              cudaStream_t stream) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(qk4v8_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmemBytes);
+    // The dynamic shared-memory limit is a per-device function attribute.
+    constexpr int kMaxDevices = 64;
+    static bool configured[2][kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int which = p.decode ? 1 : 0;
+    if (dev >= kMaxDevices || !configured[which][dev]) {
+        e = p.decode ? cudaFuncSetAttribute(qk4v8_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            kSmemBytes)
+                     : cudaFuncSetAttribute(qk4v8_attention_kernel<false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
-        configured = true;
+        if (dev < kMaxDevices) configured[which][dev] = true;
     }
-    qk4v8_attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmap_k, tmap_v, p);
+    if (p.decode)
+        qk4v8_attention_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tmap_k, tmap_v, p);
+    else
+        qk4v8_attention_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tmap_k, tmap_v, p);
     return cudaGetLastError();
 }
 

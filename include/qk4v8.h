@@ -155,6 +155,32 @@ QK4V8_API size_t qk4v8_decode_workspace_bytes(int B, int Hq, int nq, int num_spl
 QK4V8_API int qk4v8_decode_default_splits(int B, int Hkv, int max_seqlen);
 
 /*
+ * The two stages of qk4v8_attention_decode, as separate launches.
+ *
+ * qk4v8_attention_decode_splitkv: one CTA per (sequence, KV head, split) runs
+ * the tiled QK4V8 attention over its contiguous slice of the cache. It writes
+ * the split's normalised partial output and log2-sum-exp to `workspace`:
+ *     float O[B][Hq][nq][splits][128], then float lse2[B][Hq][nq][splits].
+ * A split with no key writes O = 0 and lse2 = -inf. Arguments as for
+ * qk4v8_attention_decode.
+ *
+ * qk4v8_decode_merge: combines the splits of each query row,
+ *     O = sum_s 2^(lse2_s - m) O_s / sum_s 2^(lse2_s - m),  m = max_s lse2_s,
+ * into out bf16 [B][nq][Hq][128]. lse (nullable) receives the natural-log
+ * log-sum-exp [B][Hq][nq]. num_splits must be the count the split-KV launch
+ * used (qk4v8_decode_default_splits when it was given 0).
+ */
+QK4V8_API int qk4v8_attention_decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq,
+                                             int q_cap, const uint8_t *k_codes, const uint8_t *k_scales,
+                                             const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap,
+                                             const int32_t *seqlens_k, int max_seqlen, int causal_in_block,
+                                             float softmax_scale, int num_splits, void *workspace,
+                                             size_t workspace_bytes, int32_t *dev_status, void *stream);
+
+QK4V8_API int qk4v8_decode_merge(const void *workspace, size_t workspace_bytes, int B, int Hq, int nq,
+                                 int num_splits, void *out, float *lse, void *stream);
+
+/*
  * Split-KV decode and speculative block verify over a packed KV cache.
  *   q_*      packed MXFP4 Q, [B][Hq][q_cap] with nq (1..8) query tokens
  *   k_*, v_* packed cache, [B][Hkv][kv_cap]
