@@ -35,6 +35,8 @@ SIGNATURES = {
     "qk4v8_attention_decode_splitkv": ([_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _vp,
                                         _i32, _i32, _f32, _i32, _vp, _sz, _vp, _vp], _i32),
     "qk4v8_decode_merge": ([_vp, _sz, _i32, _i32, _i32, _i32, _vp, _vp, _vp], _i32),
+    "qk4v8_attention_decode_noalloc": ([_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _vp,
+                                        _i32, _i32, _f32, _i32, _vp, _vp, _vp, _vp], _i32),
     "qk4v8_test_set_stall": ([_i32], None),
     "qk4v8_test_set_dump_scores": ([_vp], None),
 }

@@ -378,3 +378,68 @@ void qk4v8_test_set_stall(int enable) { g_test_stall = enable ? 1 : 0; }
 void qk4v8_test_set_dump_scores(float *dev_ptr) { g_test_dump_s = dev_ptr; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without any allocation by the caller.
+//
+// Some callers cannot call cudaMalloc. Examples are a plug-in running inside a
+// host application that owns and budgets all device memory (an inference
+// server's pre-reserved pool), and a latency-critical loop where cudaMalloc's
+// implicit device synchronisation is not acceptable. For them, the split-KV
+// scratch lives in this fixed, file-scope device array. Every GPU that loads
+// the library holds it until the process exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char qk4v8_noalloc_scratch[QK4V8_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+constexpr int kNoAllocMaxDevices = 64;
+void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device. In host code the
+// array's name only stands in for the symbol and is not a device address, so
+// the address is looked up once per device, with that device current.
+int noalloc_scratch_address(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return set_error(QK4V8_ERR_UNSUPPORTED, "device index %d too large", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, qk4v8_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_error(e, "cudaGetSymbolAddress(decode scratch)");
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return QK4V8_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qk4v8_attention_decode_noalloc(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq,
+                                   int q_cap, const uint8_t *k_codes, const uint8_t *k_scales,
+                                   const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap,
+                                   const int32_t *seqlens_k, int max_seqlen, int causal_in_block,
+                                   float softmax_scale, int num_splits, void *out, float *lse, int32_t *dev_status,
+                                   void *stream) {
+    if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
+    const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hkv, max_seqlen);
+    const size_t need = qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
+    if (need == 0 || need > QK4V8_NOALLOC_SCRATCH_BYTES)
+        return set_error(QK4V8_ERR_INVALID_ARG,
+                         "decode scratch of %zu bytes (B=%d Hq=%d nq=%d splits=%d) exceeds the fixed %zu-byte "
+                         "array of qk4v8_attention_decode_noalloc; use qk4v8_attention_decode with a workspace",
+                         need, B, Hq, nq, splits, static_cast<size_t>(QK4V8_NOALLOC_SCRATCH_BYTES));
+    void *scratch = nullptr;
+    int st = noalloc_scratch_address(&scratch);
+    if (st) return st;
+    return qk4v8_attention_decode(q_codes, q_scales, B, Hq, nq, q_cap, k_codes, k_scales, v_codes, v_scales, Hkv,
+                                  kv_cap, seqlens_k, max_seqlen, causal_in_block, softmax_scale, splits, scratch,
+                                  need, out, lse, dev_status, stream);
+}
+
+}  // extern "C"

@@ -199,6 +199,40 @@ QK4V8_API int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_sc
                            float softmax_scale, int num_splits, void *workspace, size_t workspace_bytes,
                            void *out, float *lse, int32_t *dev_status, void *stream);
 
+/*
+ * Decode for callers that cannot allocate device memory: qk4v8_attention_decode
+ * with the split-KV scratch taken from a fixed array inside the library
+ * instead of a caller workspace. The paper has no counterpart; this is a
+ * deployment convenience.
+ *
+ * Who needs it: code that may not call cudaMalloc, for example a plug-in whose
+ * host application owns all device memory, or a latency-critical loop that
+ * cannot afford cudaMalloc's implicit device synchronisation.
+ *
+ *   - The scratch is a device array of QK4V8_NOALLOC_SCRATCH_BYTES (8 MiB),
+ *     present on every GPU that loads the library until the process exits.
+ *     Requests that need more (qk4v8_decode_workspace_bytes(B, Hq, nq, splits)
+ *     larger than that) fail with QK4V8_ERR_INVALID_ARG and a message naming
+ *     the size.
+ *   - The first call on each device looks up the array's device address, with
+ *     that device current. Make that first call before any stream capture.
+ *   - Every call shares the one array, and the array keeps the last call's
+ *     contents. Nothing in it has to start at zero: the split-KV kernel writes
+ *     every slot the merge reads. Calls that overlap on the GPU (different
+ *     streams, or different host threads without ordering) race on the array;
+ *     serialise them.
+ *   - It allocates nothing (no cudaMalloc, no cudaFree, no allocating library
+ *     call). Arguments and results as for qk4v8_attention_decode.
+ */
+#define QK4V8_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+QK4V8_API int qk4v8_attention_decode_noalloc(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq,
+                                             int q_cap, const uint8_t *k_codes, const uint8_t *k_scales,
+                                             const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap,
+                                             const int32_t *seqlens_k, int max_seqlen, int causal_in_block,
+                                             float softmax_scale, int num_splits, void *out, float *lse,
+                                             int32_t *dev_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
