@@ -313,7 +313,11 @@ int decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scales, int B, int H
     p.status = dev_status;
     p.test_stall = g_test_stall;
     p.test_dump_s = g_test_dump_s;
-    cudaError_t e = qk4v8::launch_attention(tk, tv, p, B * Hkv * splits, stream);
+    // G*nq <= 64 query rows: the swap-AB decode kernel; larger groups use the
+    // 128-row attention kernel in its decode instantiation.
+    cudaError_t e = (Hq / Hkv) * nq <= qk4v8::kDecodeMaxRows
+                        ? qk4v8::launch_decode(tk, tv, p, B * Hkv * splits, stream)
+                        : qk4v8::launch_attention(tk, tv, p, B * Hkv * splits, stream);
     if (e != cudaSuccess) return cuda_error(e, "attention (decode) launch");
     *splits_used = splits;
     return QK4V8_OK;

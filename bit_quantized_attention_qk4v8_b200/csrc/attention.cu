@@ -28,6 +28,7 @@
 
 #include <cstdint>
 
+#include "pipeline.cuh"
 #include "ptx.cuh"
 #include "qk4v8_internal.h"
 
@@ -89,33 +90,6 @@ constexpr uint32_t kSw128 = 2, kSw64 = 4, kSwNone = 0;
 struct Bars {
     uint64_t *kv_full, *kv_empty, *q_full, *patch, *s_full, *s_free, *p_full, *pv_done, *o_final;
 };
-
-__device__ __forceinline__ bool aborted(volatile uint32_t *flag, const int32_t *status) {
-    if (*flag) return true;
-    if (status && *reinterpret_cast<const volatile int32_t *>(status) != 0) return true;
-    return false;
-}
-
-// Bounded wait on an mbarrier phase. On expiry it records QK4V8_ERR_TIMEOUT (4)
-// and raises the CTA abort flag; every other wait then returns false quickly.
-__device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile uint32_t *flag, int32_t *status) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t n = 1;; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((n & 63) == 0) {
-            if (aborted(flag, status)) return false;
-            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-                *flag = 1;
-                if (status) atomicCAS(status, 0, 4);
-                return false;
-            }
-        }
-    }
-}
-
-__device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
-__device__ __forceinline__ int imax(int a, int b) { return a > b ? a : b; }
 
 struct Unit {
     int b, h_kv, h_q, q0, R, L, tile_begin, tile_end, split;
@@ -185,11 +159,6 @@ __device__ __forceinline__ RowInfo row_info(const AttnParams &p, const Unit &u, 
     return r;
 }
 
-__device__ __forceinline__ float exp2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 // Writes the result of a row that saw no key at all.
 template <bool kDecode>

@@ -45,6 +45,10 @@ cudaError_t launch_quantize_v(const void *v, int B, int S, int H, int64_t sb, in
                               cudaStream_t stream);
 cudaError_t launch_attention(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p,
                              int grid, cudaStream_t stream);
+// Swap-AB split-KV decode kernel; handles G*nq <= kDecodeMaxRows query rows.
+constexpr int kDecodeMaxRows = 64;
+cudaError_t launch_decode(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p, int grid,
+                          cudaStream_t stream);
 cudaError_t launch_decode_merge(const float *ws_o, const float *ws_lse, int B, int Hq, int nq, int splits,
                                 __nv_bfloat16 *out, float *lse, cudaStream_t stream);
 

@@ -29,6 +29,11 @@ def lib():
     return _lib.lib()
 
 
+def test_library_is_not_stale(lib):
+    """The built libqk4v8.so is newer than every source it is built from."""
+    assert not qkbuild._stale()
+
+
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
     assert len(names) >= 15

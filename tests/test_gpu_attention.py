@@ -142,6 +142,8 @@ def test_prefill_softmax_scale_and_peaked_scores():
     (4, 1, 2000, 8, 8, 5, [2000, 1, 33, 129]),
     (2, 8, 1024, 64, 8, 1, [1024, 500]),
     (2, 4, 300, 4, 1, 7, [300, 7]),
+    (1, 8, 600, 16, 1, 2, None),       # G*nq = 128 rows: the 128-row kernel's decode path
+    (2, 3, 900, 12, 4, 3, [900, 400]), # odd row count (G*nq = 9)
 ])
 def test_decode_parity(B, nq, L, Hq, Hkv, splits, lens):
     gen = make_gen(B, nq, L, Hq, Hkv, seed=L + nq, lens=lens, k_out=4)
