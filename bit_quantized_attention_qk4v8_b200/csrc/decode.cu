@@ -36,14 +36,17 @@ namespace qk4v8 {
 
 namespace {
 
-constexpr int kStagesD = 6;
 constexpr float kTauD = 8.0f;
+constexpr int kEMaxD = 64;
+// Stages of the G*nq <= 16 instantiation, small enough for two CTAs per SM.
+constexpr int kDecodeSmallStages = 3;  // largest P scale exponent before O itself is rescaled
 constexpr uint32_t kPhiScaleWord = 0x7F7F7F7Fu;  // E8M0 2^0 for P_hi rows
 constexpr uint32_t kPloScaleWord = 0x7A7A7A7Au;  // E8M0 2^-5 for P_lo rows
 constexpr int kBarVote = 1, kBarSlow = 2, kBarEpi = 3, kBarAbort = 4;
 
-template <int NT, int NC>
+template <int NT, int NC, int ST>
 struct DecodeLayout {
+    static constexpr int kStages = ST;             // K/V pipeline stages
     static constexpr int kCG = NT / NC;            // column groups
     static constexpr int kSoftmaxWarps = 4 * kCG;
     static constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
@@ -51,27 +54,28 @@ struct DecodeLayout {
     static constexpr int kQ = 0;  // NT rows x 64 B, 64-byte swizzle (8 KB reserved)
     static constexpr int kK = 8192;
     static constexpr int kKBytes = 128 * 64;
-    static constexpr int kV = kK + kStagesD * kKBytes;
+    static constexpr int kV = kK + ST * kKBytes;
     static constexpr int kVBytes = 128 * 128;
-    static constexpr int kP = kV + kStagesD * kVBytes;  // 2 buffers of [P_hi rows; P_lo rows] x 128 B
+    static constexpr int kP = kV + ST * kVBytes;  // 2 buffers of [P_hi rows; P_lo rows] x 128 B
     static constexpr int kPBytes = 2 * NT * 128;
     static constexpr int kSfQ = kP + 2 * kPBytes;
     static constexpr int kSfK = kSfQ + 512;
-    static constexpr int kSfV = kSfK + kStagesD * 512;
-    static constexpr int kSfP = kSfV + kStagesD * 512;
-    static constexpr int kRed = kSfP + 512;       // [column group][quarter][NC] floats
+    static constexpr int kSfV = kSfK + ST * 512;
+    static constexpr int kSfP = kSfV + ST * 512;  // one P scale atom per P buffer
+    static constexpr int kRed = kSfP + 1024;      // [column group][quarter][NC] floats
     static constexpr int kLsum = kRed + 2048;     // [column group][quarter][NC] floats
     static constexpr int kAlpha = kLsum + 2048;   // [softmax warp][NC] floats
     static constexpr int kLim = kAlpha + 2048;    // [NT] int: exclusive key bound per query row
-    static constexpr int kBar = kLim + 256;
-    static constexpr int kNumBars = 2 * kStagesD + 11;
+    static constexpr int kEoff = kLim + 256;      // [softmax warp][NC] int: P scale exponent per row
+    static constexpr int kBar = kEoff + 2048;
+    static constexpr int kNumBars = 2 * ST + 11;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16 + 1024;
-    // TMEM columns: S^T x2 [0, 2NT), O^T [2NT, 4NT), scale factors after.
+    // TMEM columns: S^T x2 [0, 2NT), O^T [2NT, 4NT), then scale factors:
+    // Q at 4NT, K x2 at 4NT+4, V x2 at 4NT+12, P x2 at 4NT+20.
     static constexpr uint32_t kColO = 2 * NT;
     static constexpr uint32_t kColSfQ = 4 * NT;
-    static constexpr uint32_t kColSfP = 4 * NT + 20;
-    static constexpr uint32_t kTmemCols = 4 * NT + 24 <= 256 ? 256 : 512;
+    static constexpr uint32_t kTmemCols = 4 * NT + 28 <= 128 ? 128 : (4 * NT + 28 <= 256 ? 256 : 512);
     static_assert(kCG * 4 * NC * 4 <= 2048, "exchange buffers");
     static_assert(kSoftmaxWarps * NC * 4 <= 2048, "rescale buffer");
     static_assert(kBytes <= 227 * 1024, "shared memory budget");
@@ -79,6 +83,7 @@ struct DecodeLayout {
 
 __device__ __forceinline__ uint32_t col_sf_k_d(int nt, int buf) { return static_cast<uint32_t>(4 * nt + 4 + 4 * buf); }
 __device__ __forceinline__ uint32_t col_sf_v_d(int nt, int buf) { return static_cast<uint32_t>(4 * nt + 12 + 4 * buf); }
+__device__ __forceinline__ uint32_t col_sf_p_d(int nt, int buf) { return static_cast<uint32_t>(4 * nt + 20 + 4 * buf); }
 
 constexpr uint32_t idesc_d(uint32_t fmt, uint32_t n) {
     return (fmt << 7) | (fmt << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24);
@@ -122,11 +127,12 @@ __device__ __forceinline__ void st_u8(uint8_t *base, int off, uint32_t v) {
 
 }  // namespace
 
-template <int NT, int NC>
-__global__ void __launch_bounds__(DecodeLayout<NT, NC>::kThreads, 1)
+template <int NT, int NC, int ST, int MINB>
+__global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
     qk4v8_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                         const AttnParams p) {
-    using Lay = DecodeLayout<NT, NC>;
+    using Lay = DecodeLayout<NT, NC, ST>;
+    constexpr int kStagesD = Lay::kStages;
     constexpr int kSoftmaxThreads = Lay::kSoftmaxThreads;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -231,9 +237,11 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC>::kThreads, 1)
                     (t & 31) * 16 + ((t & 127) >> 5) * 4);
             }
             *reinterpret_cast<uint32_t *>(smem + Lay::kSfQ + (n & 31) * 16 + (n >> 5) * 4) = scw;
-            // P scale atom: rows [0, NT) are P_hi (2^0), rows [NT, 2NT) P_lo (2^-5).
-            *reinterpret_cast<uint32_t *>(smem + Lay::kSfP + (n & 31) * 16 + (n >> 5) * 4) =
-                n < NT ? kPhiScaleWord : kPloScaleWord;
+            // P scale atoms: rows [0, NT) are P_hi (2^0), rows [NT, 2NT) P_lo (2^-5);
+            // the softmax raises a row's bytes when its reference max moves.
+            const uint32_t pw = n < NT ? kPhiScaleWord : kPloScaleWord;
+            *reinterpret_cast<uint32_t *>(smem + Lay::kSfP + (n & 31) * 16 + (n >> 5) * 4) = pw;
+            *reinterpret_cast<uint32_t *>(smem + Lay::kSfP + 512 + (n & 31) * 16 + (n >> 5) * 4) = pw;
         }
         // P^T buffers start at zero; rows of absent queries are never written again.
         for (int c = lane; c < 2 * Lay::kPBytes / 16; c += 32)
@@ -307,16 +315,17 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC>::kThreads, 1)
                 const uint64_t dSfK0 = smem_desc(sb + Lay::kSfK, 0, 128, 0);
                 const uint64_t dSfV0 = smem_desc(sb + Lay::kSfV, 0, 128, 0);
                 tc_cp_32x128b_warpx4(tmem + Lay::kColSfQ, smem_desc(sb + Lay::kSfQ, 0, 128, 0));
-                tc_cp_32x128b_warpx4(tmem + Lay::kColSfP, smem_desc(sb + Lay::kSfP, 0, 128, 0));
+                const uint64_t dSfP0 = smem_desc(sb + Lay::kSfP, 0, 128, 0);
                 const uint32_t tO = tmem + Lay::kColO;
                 const uint32_t tSfQ = tmem + Lay::kColSfQ;
-                const uint32_t tSfP = tmem + Lay::kColSfP;
                 auto issue_pv = [&](int j) -> bool {
                     if (!wait_bar(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.status)) return false;
                     tc_fence_after();
                     const int st = j % kStagesD;
                     const uint32_t tSfV = tmem + col_sf_v_d(NT, j & 1);
+                    const uint32_t tSfP = tmem + col_sf_p_d(NT, j & 1);
                     tc_cp_32x128b_warpx4(tSfV, dSfV0 + static_cast<uint64_t>(st * 32));
+                    tc_cp_32x128b_warpx4(tSfP, dSfP0 + static_cast<uint64_t>((j & 1) * 32));
                     const uint64_t dV = dV0 + static_cast<uint64_t>(st * (Lay::kVBytes >> 4));
                     const uint64_t dP = dP0 + static_cast<uint64_t>((j & 1) * (Lay::kPBytes >> 4));
 #pragma unroll
@@ -362,20 +371,29 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC>::kThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         float *red = reinterpret_cast<float *>(smem + Lay::kRed);
         float *lsum = reinterpret_cast<float *>(smem + Lay::kLsum);
-        float *alpha_s = reinterpret_cast<float *>(smem + Lay::kAlpha) + sw * NC;
+        float *alpha_s = reinterpret_cast<float *>(smem + Lay::kAlpha) + sw * NC;  // O rescale factors
         // Byte offset of (row c0 + i, token jt) in a P^T buffer, less i * 128:
         // the 128-byte swizzle puts token jt of row n in chunk (jt/16) ^ (n%8),
         // and c0 is a multiple of 8.
-        int swz[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) swz[k] = c0 * 128 + (((jt >> 4) ^ k) << 4) + (jt & 15);
-        float m_neg[NC];  // -m per row, +inf while the row has seen no key
-        float lacc[NC];   // this thread's share of the row sums
+        const int pbase = c0 * 128 + (jt & 15);
+        const int pchunk = jt >> 4;
+        // Per query row: the reference max m used for p = 2^(s - m) (kept as -m,
+        // +inf while the row has seen no key), and e = m - m_O, the integer
+        // exponent by which m has moved above the reference m_O of the O
+        // accumulator. P's E8M0 row scale carries 2^e, so O never has to be
+        // rescaled while e <= kEMaxD. lacc is this thread's share of the row sum,
+        // relative to m.
+        float m_neg[NC];
+        float lacc[NC];
+        int *e_off = reinterpret_cast<int *>(smem + Lay::kEoff) + sw * NC;  // this warp's copy
 #pragma unroll
         for (int i = 0; i < NC; ++i) {
             m_neg[i] = INFINITY;
             lacc[i] = 0.f;
         }
+        if (lane < NC) e_off[lane] = 0;
+        __syncwarp();
+        int sf_dirty = 0;  // P buffers whose scale atom still holds an old e
         const float sc = p.scale_log2;
         // Key bound of each query row: L, or L - nq + t + 1 for token t of a causal
         // verify block. Tabulated once so the per-tile loop needs no division.
@@ -388,15 +406,13 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC>::kThreads, 1)
             const int sbuf = it & 1;
             ok = wait_bar(&s_full[sbuf], (it >> 1) & 1, abort_flag, p.status);
             ok = __all_sync(0xffffffffu, ok);
+            const uint32_t tS = tmem + lane_base + static_cast<uint32_t>(NT * sbuf + c0);
             uint32_t sraw[NC];
             if (ok) {
                 tc_fence_after();
-                tmem_load_cols<NC>(tmem + lane_base + static_cast<uint32_t>(NT * sbuf + c0), sraw);
+                tmem_load_cols<NC>(tS, sraw);
                 tc_wait_ld();
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[sbuf]);
 
             const int tok = (tile_begin + it) * 128 + jt;
             // Every row may see this key unless it lies past L, or in the last
@@ -423,54 +439,92 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC>::kThreads, 1)
             // slow branch, where a second vote makes the exit collective, so no
             // softmax warp is left waiting at a named barrier.
             const bool need = bar_red_or(kBarVote, kSoftmaxThreads, umax > kTauD || *abort_flag != 0);
-            if (need) {
+            if (!need) {
+                // S buffer `sbuf` is next written by S(it+2), issued after this tile's P.
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[sbuf]);
+            } else {
                 if (bar_red_or(kBarAbort, kSoftmaxThreads, *abort_flag != 0)) {
                     ok = false;
                     break;
                 }
-                // Exact per-row maximum of this tile's scaled scores, then move m.
+                // Exact per-row maximum of this tile's scaled scores (reloaded from
+                // TMEM, so the raw scores need not stay live), then move m.
+                uint32_t sre[NC];
+                tc_fence_after();
+                tmem_load_cols<NC>(tS, sre);
+                tc_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[sbuf]);
 #pragma unroll
                 for (int i = 0; i < NC; ++i) {
-                    const float x = u[i] == -INFINITY ? -INFINITY : __uint_as_float(sraw[i]) * sc;
+                    const float x = u[i] == -INFINITY ? -INFINITY : __uint_as_float(sre[i]) * sc;
                     const float mx = warp_max_f32(x);
                     if (lane == i) red[(cg * 4 + quarter) * NC + i] = mx;
                 }
                 bar_sync(kBarSlow, kSoftmaxThreads);
-                bool moved = false;
+                bool changed = false, over = false;
 #pragma unroll
                 for (int i = 0; i < NC; ++i) {
                     float tmax = red[(cg * 4 + 0) * NC + i];
 #pragma unroll
                     for (int q = 1; q < 4; ++q) tmax = fmaxf(tmax, red[(cg * 4 + q) * NC + i]);
-                    const float m_old = -m_neg[i];
-                    const float m_new = fmaxf(m_old, tmax);
-                    const float a = (m_new == -INFINITY || m_new == m_old) ? 1.f : exp2_approx(m_old - m_new);
-                    moved |= (m_old > -INFINITY && m_new > m_old);
-                    if (m_new > -INFINITY) m_neg[i] = -m_new;
+                    float a = 1.f;
+                    if (m_neg[i] == INFINITY) {
+                        // First key of the row: it fixes m_O = m.
+                        if (tmax > -INFINITY) m_neg[i] = -tmax;
+                    } else if (tmax + m_neg[i] > kTauD) {
+                        // Move m up by a whole number of binades, so the change is
+                        // an exact power of two in P's scale.
+                        const int de = static_cast<int>(ceilf(tmax + m_neg[i]));
+                        m_neg[i] -= static_cast<float>(de);
+                        const int ne = e_off[i] + de;
+                        __syncwarp();
+                        if (lane == 0) e_off[i] = ne;
+                        a = de < 126 ? __uint_as_float(static_cast<uint32_t>(127 - de) << 23) : 0.f;
+                        changed = true;
+                        over |= ne > kEMaxD;
+                    }
                     lacc[i] *= a;
-                    if (lane == 0) alpha_s[i] = a;
-                    if (u[i] != -INFINITY) u[i] = fmaf(__uint_as_float(sraw[i]), sc, m_neg[i]);
+                    if (u[i] != -INFINITY) u[i] = fmaf(__uint_as_float(sre[i]), sc, m_neg[i]);
                 }
                 __syncwarp();
-                // O^T columns of these rows hold PV(it-1); rescale them once it is done.
-                if (it >= 1 && __any_sync(0xffffffffu, moved)) {
-                    bool okw = wait_bar(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag, p.status);
-                    if (__all_sync(0xffffffffu, okw)) {
-                        tc_fence_after();
-                        uint32_t ohi[NC], olo[NC];
-                        tmem_load_cols<NC>(tmem + lane_base + Lay::kColO + c0, ohi);
-                        tmem_load_cols<NC>(tmem + lane_base + Lay::kColO + NT + c0, olo);
-                        tc_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < NC; ++e) {
-                            const float a = alpha_s[e];
-                            ohi[e] = __float_as_uint(__uint_as_float(ohi[e]) * a);
-                            olo[e] = __float_as_uint(__uint_as_float(olo[e]) * a);
+                if (changed) sf_dirty = 2;
+                // Past kEMaxD binades O itself is brought to the current reference:
+                // O *= 2^-e once PV(it-1) is done, and e restarts at 0.
+                if (__any_sync(0xffffffffu, over)) {
+                    __syncwarp();
+                    for (int i = 0; i < NC; ++i) {
+                        const int ee = e_off[i] > kEMaxD ? e_off[i] : 0;
+                        __syncwarp();
+                        if (lane == 0) {
+                            alpha_s[i] = ee < 126 ? __uint_as_float(static_cast<uint32_t>(127 - ee) << 23) : 0.f;
+                            if (ee) e_off[i] = 0;
                         }
-                        tmem_store_cols<NC>(tmem + lane_base + Lay::kColO + c0, ohi);
-                        tmem_store_cols<NC>(tmem + lane_base + Lay::kColO + NT + c0, olo);
-                        tc_wait_st();
                     }
+                    __syncwarp();
+                    if (it >= 1) {
+                        bool okw = wait_bar(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag, p.status);
+                        if (__all_sync(0xffffffffu, okw)) {
+                            tc_fence_after();
+                            uint32_t ohi[NC], olo[NC];
+                            tmem_load_cols<NC>(tmem + lane_base + Lay::kColO + c0, ohi);
+                            tmem_load_cols<NC>(tmem + lane_base + Lay::kColO + NT + c0, olo);
+                            tc_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < NC; ++c) {
+                                const float a = alpha_s[c];
+                                ohi[c] = __float_as_uint(__uint_as_float(ohi[c]) * a);
+                                olo[c] = __float_as_uint(__uint_as_float(olo[c]) * a);
+                            }
+                            tmem_store_cols<NC>(tmem + lane_base + Lay::kColO + c0, ohi);
+                            tmem_store_cols<NC>(tmem + lane_base + Lay::kColO + NT + c0, olo);
+                            tc_wait_st();
+                        }
+                    }
+                    sf_dirty = 2;
                 }
             }
             // P buffer `sbuf` was last read by PV(it-2).
@@ -479,6 +533,20 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC>::kThreads, 1)
                 (void)__all_sync(0xffffffffu, okw);
             }
             uint8_t *pb = smem + Lay::kP + sbuf * Lay::kPBytes;
+            if (sf_dirty > 0) {
+                // This buffer's scale atom: byte `quarter` (this warp's 32 keys) of
+                // rows c0+i (P_hi, 2^e) and NT+c0+i (P_lo, 2^(e-5)).
+                if (lane == 0) {
+                    uint8_t *atom = smem + Lay::kSfP + sbuf * 512;
+#pragma unroll
+                    for (int i = 0; i < NC; ++i) {
+                        const int n = c0 + i, nl = NT + c0 + i;
+                        atom[(n & 31) * 16 + (n >> 5) * 4 + quarter] = static_cast<uint8_t>(127 + e_off[i]);
+                        atom[(nl & 31) * 16 + (nl >> 5) * 4 + quarter] = static_cast<uint8_t>(122 + e_off[i]);
+                    }
+                }
+                --sf_dirty;
+            }
 #pragma unroll
             for (int i = 0; i < NC; i += 2) {
                 if (i >= nv) break;
@@ -496,8 +564,8 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC>::kThreads, 1)
                 const float2 ptf = __half22float2(pt);
                 lacc[i] += ptf.x;
                 lacc[i + 1] += ptf.y;
-                const int o0 = swz[i & 7] + i * 128;
-                const int o1 = swz[(i + 1) & 7] + (i + 1) * 128;
+                const int o0 = pbase + ((pchunk ^ (i & 7)) << 4) + i * 128;
+                const int o1 = pbase + ((pchunk ^ ((i + 1) & 7)) << 4) + (i + 1) * 128;
                 st_u8(pb, o0, h2);
                 st_u8(pb, o0 + NT * 128, l2);
                 if (i + 1 < nv) {
@@ -541,7 +609,9 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC>::kThreads, 1)
                                     lsum[(cg * 4 + 2) * NC + i] + lsum[(cg * 4 + 3) * NC + i];
                     const bool any = l > 0.f && m_neg[i] < INFINITY;
                     const int64_t row = partial_row(c0 + i);
-                    p.ws_o[row * 128 + jt] = any ? (__uint_as_float(ohi[e]) + __uint_as_float(olo[e])) / l : 0.f;
+                    // O is relative to m_O = m - e: divide by l * 2^e.
+                    const float inv = any ? __uint_as_float(static_cast<uint32_t>(127 - e_off[i]) << 23) / l : 0.f;
+                    p.ws_o[row * 128 + jt] = (__uint_as_float(ohi[e]) + __uint_as_float(olo[e])) * inv;
                     if (jt == 0) p.ws_lse[row] = any ? log2f(l) - m_neg[i] : -INFINITY;
                 }
             }
@@ -556,31 +626,31 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC>::kThreads, 1)
     }
 }
 
-template <int NT, int NC>
+template <int NT, int NC, int ST, int MINB>
 static cudaError_t launch_nt(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, int grid,
                              cudaStream_t stream) {
-    using Lay = DecodeLayout<NT, NC>;
+    using Lay = DecodeLayout<NT, NC, ST>;
     constexpr int kMaxDevices = 64;
     static bool configured[kMaxDevices] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= kMaxDevices || !configured[dev]) {
-        e = cudaFuncSetAttribute(qk4v8_decode_kernel<NT, NC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(qk4v8_decode_kernel<NT, NC, ST, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Lay::kBytes);
         if (e != cudaSuccess) return e;
         if (dev < kMaxDevices) configured[dev] = true;
     }
-    qk4v8_decode_kernel<NT, NC><<<grid, Lay::kThreads, Lay::kBytes, stream>>>(tk, tv, p);
+    qk4v8_decode_kernel<NT, NC, ST, MINB><<<grid, Lay::kThreads, Lay::kBytes, stream>>>(tk, tv, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, int grid,
                           cudaStream_t stream) {
     const int R = p.G * p.Sq;
-    if (R <= 16) return launch_nt<16, 16>(tk, tv, p, grid, stream);
-    if (R <= 32) return launch_nt<32, 16>(tk, tv, p, grid, stream);
-    return launch_nt<64, 16>(tk, tv, p, grid, stream);
+    if (R <= 16) return launch_nt<16, 16, kDecodeSmallStages, 2>(tk, tv, p, grid, stream);
+    if (R <= 32) return launch_nt<32, 16, 6, 1>(tk, tv, p, grid, stream);
+    return launch_nt<64, 16, 6, 1>(tk, tv, p, grid, stream);
 }
 
 }  // namespace qk4v8
