@@ -160,8 +160,8 @@ def decode_workspace_bytes(B: int, Hq: int, nq: int, num_splits: int) -> int:
     return int(lib().qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits))
 
 
-def decode_default_splits(B: int, Hkv: int, max_seqlen: int) -> int:
-    return int(lib().qk4v8_decode_default_splits(B, Hkv, max_seqlen))
+def decode_default_splits(B: int, Hq: int, Hkv: int, nq: int, max_seqlen: int) -> int:
+    return int(lib().qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen))
 
 
 def attention_decode(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optional[int] = None,
@@ -175,7 +175,7 @@ def attention_decode(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optio
     sl = _seqlens(seqlens_k, B, dev)
     if max_seqlen is None:
         max_seqlen = k.cap
-    splits = num_splits if num_splits > 0 else decode_default_splits(B, k.H, max_seqlen)
+    splits = num_splits if num_splits > 0 else decode_default_splits(B, Hq, k.H, nq, max_seqlen)
     need = decode_workspace_bytes(B, Hq, nq, splits)
     if workspace is None:
         workspace = torch.empty((need,), dtype=torch.uint8, device=dev)

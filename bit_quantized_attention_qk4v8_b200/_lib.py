@@ -29,7 +29,7 @@ SIGNATURES = {
     "qk4v8_attention_prefill": ([_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                                  _vp, _i32, _f32, _vp, _vp, _vp, _vp], _i32),
     "qk4v8_decode_workspace_bytes": ([_i32, _i32, _i32, _i32], _sz),
-    "qk4v8_decode_default_splits": ([_i32, _i32, _i32], _i32),
+    "qk4v8_decode_default_splits": ([_i32, _i32, _i32, _i32, _i32], _i32),
     "qk4v8_attention_decode": ([_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32,
                                 _i32, _f32, _i32, _vp, _sz, _vp, _vp, _vp, _vp], _i32),
     "qk4v8_attention_decode_splitkv": ([_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _vp,

@@ -240,16 +240,36 @@ size_t qk4v8_decode_workspace_bytes(int B, int Hq, int nq, int num_splits) {
     return rows * 128 * sizeof(float) + rows * sizeof(float);
 }
 
-int qk4v8_decode_default_splits(int B, int Hkv, int max_seqlen) {
-    // Enough CTAs for about two waves of 148 SMs, but no split shorter than
-    // 16 tiles of 128 keys.
-    const int units = B > 0 && Hkv > 0 ? B * Hkv : 1;
+int qk4v8_decode_default_splits(int B, int Hq, int Hkv, int nq, int max_seqlen) {
+    // Wave cost model: a launch of units * s CTAs over `slots` resident CTA
+    // slots takes ceil(units * s / slots) waves, each as long as one split
+    // (ceil(tiles / s) key tiles of 128) plus a fixed cost of about
+    // kSplitOverheadTiles tiles for the prologue, pipeline fill and epilogue.
+    // Pick the cheapest s, the smallest on ties.
+    constexpr int kSplitOverheadTiles = 3;
+    constexpr int kMaxSplits = 64;
+    if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv || nq <= 0) return 1;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+        sms = 148;
+        (void)cudaGetLastError();
+    }
+    const int rows = (Hq / Hkv) * nq;
+    const int64_t slots = static_cast<int64_t>(sms) * (rows <= 16 ? 2 : 1);
+    const int64_t units = static_cast<int64_t>(B) * Hkv;
     const int tiles = max_seqlen > 0 ? (max_seqlen + 127) / 128 : 1;
-    int splits = (2 * 148 + units - 1) / units;
-    const int max_by_len = tiles / 16 > 0 ? tiles / 16 : 1;
-    if (splits > max_by_len) splits = max_by_len;
-    if (splits < 1) splits = 1;
-    return splits;
+    int best = 1;
+    int64_t best_cost = INT64_MAX;
+    for (int s = 1; s <= kMaxSplits && s <= tiles; ++s) {
+        const int64_t waves = (units * s + slots - 1) / slots;
+        const int64_t cost = waves * ((tiles + s - 1) / s + kSplitOverheadTiles);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
 }
 
 }  // extern "C"
@@ -278,7 +298,7 @@ int decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scales, int B, int H
         return set_error(QK4V8_ERR_INVALID_ARG, "bad lengths q_cap=%d kv_cap=%d max_seqlen=%d", q_cap, kv_cap,
                          max_seqlen);
     if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
-    const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hkv, max_seqlen);
+    const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen);
     const size_t need = qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
     if (!workspace || !aligned16(workspace) || workspace_bytes < need)
         return set_error(QK4V8_ERR_INVALID_ARG, "workspace must be 16-byte aligned and >= %zu bytes", need);
@@ -431,7 +451,7 @@ int qk4v8_attention_decode_noalloc(const uint8_t *q_codes, const uint8_t *q_scal
                                    float softmax_scale, int num_splits, void *out, float *lse, int32_t *dev_status,
                                    void *stream) {
     if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
-    const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hkv, max_seqlen);
+    const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen);
     const size_t need = qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
     if (need == 0 || need > QK4V8_NOALLOC_SCRATCH_BYTES)
         return set_error(QK4V8_ERR_INVALID_ARG,

@@ -14,11 +14,16 @@
 // hold the P_hi part and [NT, 2NT) the P_lo part, summed in the epilogue.
 //
 // Softmax: thread (lane quarter q, lane l) owns token 32q + l of the tile; a
-// warp covers NC query rows. Rows share a reference max m that moves only when
-// a score exceeds it by 2^8 (one barrier vote of the softmax threads per tile).
-// So the common path needs no reduction, and p = 2^(s - m) <= 256.
-// P_hi = E4M3(p), P_lo = E4M3((p - P_hi) * 32): about 8 significant bits. The
-// denominator sums P_hi + P_lo exactly as the MMA sees them.
+// warp covers NC query rows, and the four warps of a column group cover the
+// tile's four 32-key blocks. The P operand carries one E8M0 scale per (row,
+// 32-key block), so every warp keeps its own reference max m per row: p =
+// 2^(s - m) <= 2^8, and the block's scale byte holds the integer offset e =
+// m - m_O from the reference m_O of the O accumulator. A warp moves its m (by
+// whole binades, only when a score passes it by 2^8) without talking to the
+// other warps; the group agrees on m_O once, on its first tile, and moves it
+// only when some offset passes 2^64 (an mbarrier vote posted early in the tile
+// and collected after the encode, so it rarely waits).
+// P_hi = E4M3(p), P_lo = E4M3((p - P_hi) * 32): about 8 significant bits.
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer,
 // warps 2.. softmax and epilogue (4 per column group of NC rows).
@@ -36,13 +41,19 @@ namespace qk4v8 {
 
 namespace {
 
-constexpr float kTauD = 8.0f;
-constexpr int kEMaxD = 64;
+constexpr float kTauD = 8.0f;      // a warp moves m once a score passes it by 2^kTauD
+constexpr int kEMaxD = 64;         // largest offset e = m - m_O before O itself is rescaled
+constexpr float kMaxMoveD = 16777216.0f;  // cap on one move of m (binades), keeps it an exact integer
 // Stages of the G*nq <= 16 instantiation, small enough for two CTAs per SM.
-constexpr int kDecodeSmallStages = 3;  // largest P scale exponent before O itself is rescaled
+constexpr int kDecodeSmallStages = 3;
 constexpr uint32_t kPhiScaleWord = 0x7F7F7F7Fu;  // E8M0 2^0 for P_hi rows
 constexpr uint32_t kPloScaleWord = 0x7A7A7A7Au;  // E8M0 2^-5 for P_lo rows
-constexpr int kBarVote = 1, kBarSlow = 2, kBarEpi = 3, kBarAbort = 4;
+// Named barriers: one per column group (ids 1..4), and one over all softmax warps.
+constexpr int kBarGroup0 = 1, kBarAllSoftmax = 5;
+// Limit on the vote wait, which ignores the abort flag so that a column group
+// always takes the same branch (nanoseconds; above any bounded wait a peer may
+// be sitting in).
+constexpr uint64_t kVoteTimeoutNs = 4 * kWaitTimeoutNs;
 
 template <int NT, int NC, int ST>
 struct DecodeLayout {
@@ -62,13 +73,18 @@ struct DecodeLayout {
     static constexpr int kSfK = kSfQ + 512;
     static constexpr int kSfV = kSfK + ST * 512;
     static constexpr int kSfP = kSfV + ST * 512;  // one P scale atom per P buffer
-    static constexpr int kRed = kSfP + 1024;      // [column group][quarter][NC] floats
-    static constexpr int kLsum = kRed + 2048;     // [column group][quarter][NC] floats
-    static constexpr int kAlpha = kLsum + 2048;   // [softmax warp][NC] floats
-    static constexpr int kLim = kAlpha + 2048;    // [NT] int: exclusive key bound per query row
-    static constexpr int kEoff = kLim + 256;      // [softmax warp][NC] int: P scale exponent per row
-    static constexpr int kBar = kEoff + 2048;
-    static constexpr int kNumBars = 2 * ST + 11;
+    // Exchange buffers, each [column group][quarter][NC] 32-bit words.
+    static constexpr int kXmax = kSfP + 1024;  // first-tile row maxima
+    static constexpr int kXe = kXmax + 1024;    // offsets e, when O is rescaled
+    static constexpr int kLsum = kXe + 1024;    // epilogue row sums
+    static constexpr int kEsum = kLsum + 1024;  // epilogue offsets e
+    static constexpr int kLim = kEsum + 1024;   // [NT] int: exclusive key bound per query row
+    static constexpr int kVote = kLim + 256;    // [column group][tile parity][quarter] u32 vote words
+    static constexpr int kMneg = kVote + 128;   // [softmax warp][NC] float: -m of each row
+    static constexpr int kBar = kMneg + 1024;
+    // kv_full/empty per stage, q_full, patch, s_full/free x2, p_full x2,
+    // pv_done x2, o_final, vote x2 and e exchange per column group.
+    static constexpr int kNumBars = 2 * ST + 11 + 3 * kCG;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16 + 1024;
     // TMEM columns: S^T x2 [0, 2NT), O^T [2NT, 4NT), then scale factors:
@@ -76,8 +92,9 @@ struct DecodeLayout {
     static constexpr uint32_t kColO = 2 * NT;
     static constexpr uint32_t kColSfQ = 4 * NT;
     static constexpr uint32_t kTmemCols = 4 * NT + 28 <= 128 ? 128 : (4 * NT + 28 <= 256 ? 256 : 512);
-    static_assert(kCG * 4 * NC * 4 <= 2048, "exchange buffers");
-    static_assert(kSoftmaxWarps * NC * 4 <= 2048, "rescale buffer");
+    static_assert(kCG * 4 * NC * 4 <= 1024, "exchange buffers");
+    static_assert(kSoftmaxWarps * NC * 4 <= 1024 && kMneg % 16 == 0, "row references");
+    static_assert(NC <= 32 && NT <= 64, "one lane per row of a warp");
     static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -115,14 +132,27 @@ __device__ __forceinline__ void tmem_store_cols(uint32_t taddr, const uint32_t (
     }
 }
 
-__device__ __forceinline__ uint16_t cvt_e4m3x2_from_h2(uint32_t h2) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(h2));
-    return r;
-}
-
 __device__ __forceinline__ void st_u8(uint8_t *base, int off, uint32_t v) {
     base[off] = static_cast<uint8_t>(v);
+}
+
+// Wait on an mbarrier phase that every peer reaches within its own bounded
+// waits. Unlike wait_bar it does not give up on the abort flag, so all waiters
+// see the same phase and take the same branch afterwards.
+__device__ __noinline__ bool wait_bar_peers_slow(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_sleep(bar, parity, 20000))
+        if (globaltimer_ns() - t0 > kVoteTimeoutNs) return false;
+    return true;
+}
+
+__device__ __forceinline__ bool wait_bar_peers(uint64_t *bar, uint32_t parity) {
+    return mbar_try_wait(bar, parity) || wait_bar_peers_slow(bar, parity);
+}
+
+// 2^-k as a float for an integer k >= 0 (0 once it would be subnormal).
+__device__ __forceinline__ float exp2_neg_int(int k) {
+    return k < 126 ? __uint_as_float(static_cast<uint32_t>(127 - k) << 23) : 0.f;
 }
 
 }  // namespace
@@ -180,6 +210,8 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
     uint64_t *p_full = q_full + 6;   // [2]
     uint64_t *pv_done = q_full + 8;  // [2]
     uint64_t *o_final = q_full + 10;
+    uint64_t *vote_bar = q_full + 11;            // [column group][tile parity]: one arrival per warp
+    uint64_t *xe_bar = vote_bar + 2 * Lay::kCG;  // [column group]: offsets posted for an O rescale
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::kMisc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + Lay::kMisc + 4);
 
@@ -197,6 +229,11 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
             mbar_init(&pv_done[s], 1);
         }
         mbar_init(o_final, 1);
+        for (int g = 0; g < Lay::kCG; ++g) {
+            mbar_init(&vote_bar[2 * g], 4);
+            mbar_init(&vote_bar[2 * g + 1], 4);
+            mbar_init(&xe_bar[g], 4);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -369,203 +406,156 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
         const int nv = imax(0, imin(R - c0, NC));
         const int jt = quarter * 32 + lane;  // token within the tile, and channel in the epilogue
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        float *red = reinterpret_cast<float *>(smem + Lay::kRed);
-        float *lsum = reinterpret_cast<float *>(smem + Lay::kLsum);
-        float *alpha_s = reinterpret_cast<float *>(smem + Lay::kAlpha) + sw * NC;  // O rescale factors
-        // Byte offset of (row c0 + i, token jt) in a P^T buffer, less i * 128:
-        // the 128-byte swizzle puts token jt of row n in chunk (jt/16) ^ (n%8),
-        // and c0 is a multiple of 8.
-        const int pbase = c0 * 128 + (jt & 15);
-        const int pchunk = jt >> 4;
-        // Per query row: the reference max m used for p = 2^(s - m) (kept as -m,
-        // +inf while the row has seen no key), and e = m - m_O, the integer
-        // exponent by which m has moved above the reference m_O of the O
-        // accumulator. P's E8M0 row scale carries 2^e, so O never has to be
-        // rescaled while e <= kEMaxD. lacc is this thread's share of the row sum,
-        // relative to m.
-        float m_neg[NC];
+        const int gbar = kBarGroup0 + cg;
+        // Exchange slots of this column group, [quarter][NC].
+        float *xmax = reinterpret_cast<float *>(smem + Lay::kXmax) + cg * 4 * NC;
+        int *xe = reinterpret_cast<int *>(smem + Lay::kXe) + cg * 4 * NC;
+        float *lsum = reinterpret_cast<float *>(smem + Lay::kLsum) + cg * 4 * NC;
+        int *esum = reinterpret_cast<int *>(smem + Lay::kEsum) + cg * 4 * NC;
+        volatile uint32_t *votes = reinterpret_cast<volatile uint32_t *>(smem + Lay::kVote) + cg * 8;
+        // Byte offset of (row c0 + i, token jt) in a P^T buffer is
+        // pofs ^ ((i & 7) << 4) plus i * 128: the 128-byte swizzle puts token jt
+        // of row n in 16-byte chunk (jt / 16) ^ (n % 8), and c0 is a multiple of 8.
+        const int pofs = c0 * 128 + ((jt >> 4) << 4) + (jt & 15);
+        // Per query row: -m, this warp's reference max (log2 units, so p =
+        // 2^(s * scale - m)), kept in shared memory as it is the same for all
+        // lanes; lacc, this thread's share of the row sum relative to m. Lane
+        // i < NC also holds e_mine = m - m_O for row c0 + i, the exponent this
+        // warp's scale byte gives its P block.
+        float *m_neg = reinterpret_cast<float *>(smem + Lay::kMneg) + sw * NC;
         float lacc[NC];
-        int *e_off = reinterpret_cast<int *>(smem + Lay::kEoff) + sw * NC;  // this warp's copy
 #pragma unroll
-        for (int i = 0; i < NC; ++i) {
-            m_neg[i] = INFINITY;
-            lacc[i] = 0.f;
-        }
-        if (lane < NC) e_off[lane] = 0;
+        for (int i = 0; i < NC; ++i) lacc[i] = 0.f;
+        if (lane < NC) m_neg[lane] = 0.f;
         __syncwarp();
-        int sf_dirty = 0;  // P buffers whose scale atom still holds an old e
+        int e_mine = 0;
+        uint32_t n_rescales = 0;
         const float sc = p.scale_log2;
         // Key bound of each query row: L, or L - nq + t + 1 for token t of a causal
         // verify block. Tabulated once so the per-tile loop needs no division.
         int *lim_s = reinterpret_cast<int *>(smem + Lay::kLim);
         if (sw == 0)
             for (int n = lane; n < NT; n += 32) lim_s[n] = p.causal ? imin(L, L - nq + (n % nq) + 1) : L;
-        bar_sync(kBarEpi, kSoftmaxThreads);
-        bool ok = true;
+        bar_sync(kBarAllSoftmax, kSoftmaxThreads);
         for (int it = 0; it < T; ++it) {
             const int sbuf = it & 1;
-            ok = wait_bar(&s_full[sbuf], (it >> 1) & 1, abort_flag, p.status);
+            bool ok = wait_bar(&s_full[sbuf], (it >> 1) & 1, abort_flag, p.status);
             ok = __all_sync(0xffffffffu, ok);
-            const uint32_t tS = tmem + lane_base + static_cast<uint32_t>(NT * sbuf + c0);
             uint32_t sraw[NC];
             if (ok) {
                 tc_fence_after();
-                tmem_load_cols<NC>(tS, sraw);
+                tmem_load_cols<NC>(tmem + lane_base + static_cast<uint32_t>(NT * sbuf + c0), sraw);
                 tc_wait_ld();
             }
+            // S buffer `sbuf` is next written by S(it+2), issued after this tile's P.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[sbuf]);
 
+            // u = s * scale - m (log2 units); -inf where the key is masked. Every row
+            // may see this key unless it lies past L, or in the last nq-1 positions
+            // where query t of the verify block stops at L - nq + t.
             const int tok = (tile_begin + it) * 128 + jt;
-            // Every row may see this key unless it lies past L, or in the last
-            // nq-1 positions where query t of the verify block stops at L - nq + t.
-            const bool all_rows = ok && tok < L - (p.causal ? nq - 1 : 0);
-            float u[NC];  // s * scale - m (log2 units); -inf when the key is masked
-            float umax = -INFINITY;
-            if (all_rows) {
+            float mrow[NC];
 #pragma unroll
-                for (int i = 0; i < NC; ++i) {
-                    u[i] = i < nv ? fmaf(__uint_as_float(sraw[i]), sc, m_neg[i]) : -INFINITY;
-                    umax = fmaxf(umax, u[i]);
-                }
+            for (int i = 0; i < NC; i += 4) {
+                const float4 m4 = *reinterpret_cast<const float4 *>(m_neg + i);
+                mrow[i] = m4.x;
+                mrow[i + 1] = m4.y;
+                mrow[i + 2] = m4.z;
+                mrow[i + 3] = m4.w;
+            }
+            float u[NC];
+            if (it > 0 && ok && tok < L - (p.causal ? nq - 1 : 0)) {
+#pragma unroll
+                for (int i = 0; i < NC; ++i)
+                    u[i] = i < nv ? fmaf(__uint_as_float(sraw[i]), sc, mrow[i]) : -INFINITY;
             } else {
                 const bool any_key = ok && tok < L;
 #pragma unroll
                 for (int i = 0; i < NC; ++i) {
                     const bool valid = any_key && i < nv && tok < lim_s[c0 + i];
-                    u[i] = valid ? fmaf(__uint_as_float(sraw[i]), sc, m_neg[i]) : -INFINITY;
-                    umax = fmaxf(umax, u[i]);
+                    u[i] = valid ? fmaf(__uint_as_float(sraw[i]), sc, mrow[i]) : -INFINITY;
                 }
             }
-            // One vote per tile. An abort raised anywhere in the CTA also takes the
-            // slow branch, where a second vote makes the exit collective, so no
-            // softmax warp is left waiting at a named barrier.
-            const bool need = bar_red_or(kBarVote, kSoftmaxThreads, umax > kTauD || *abort_flag != 0);
-            if (!need) {
-                // S buffer `sbuf` is next written by S(it+2), issued after this tile's P.
-                tc_fence_before();
+            if (it == 0) {
+                // The group's first tile fixes m_O = m of each row: the row's largest
+                // scaled score over the tile's 128 keys. A row with no key here has
+                // no key in any later tile of the split (keys only grow), and keeps
+                // m = 0 with a zero sum.
+#pragma unroll
+                for (int i = 0; i < NC; ++i) {
+                    const float mx = warp_max_f32(u[i]);
+                    if (lane == i) xmax[quarter * NC + i] = mx;
+                }
+                bar_sync(gbar, 128);
+#pragma unroll
+                for (int i = 0; i < NC; ++i) {
+                    const float t = fmaxf(fmaxf(xmax[i], xmax[NC + i]), fmaxf(xmax[2 * NC + i], xmax[3 * NC + i]));
+                    if (t > -INFINITY) {
+                        if (lane == i) m_neg[i] = -t;
+                        u[i] -= t;
+                    }
+                }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s_free[sbuf]);
             } else {
-                if (bar_red_or(kBarAbort, kSoftmaxThreads, *abort_flag != 0)) {
-                    ok = false;
-                    break;
-                }
-                // Exact per-row maximum of this tile's scaled scores (reloaded from
-                // TMEM, so the raw scores need not stay live), then move m.
-                uint32_t sre[NC];
-                tc_fence_after();
-                tmem_load_cols<NC>(tS, sre);
-                tc_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_free[sbuf]);
+                // This warp's own moves: a row whose scores pass m by more than 2^kTauD
+                // moves m up to the next whole binade above its maximum, so the offset
+                // e in the scale byte stays an integer.
+                float umax = u[0];
 #pragma unroll
-                for (int i = 0; i < NC; ++i) {
-                    const float x = u[i] == -INFINITY ? -INFINITY : __uint_as_float(sre[i]) * sc;
-                    const float mx = warp_max_f32(x);
-                    if (lane == i) red[(cg * 4 + quarter) * NC + i] = mx;
-                }
-                bar_sync(kBarSlow, kSoftmaxThreads);
-                bool changed = false, over = false;
+                for (int i = 1; i < NC; ++i) umax = fmaxf(umax, u[i]);
+                if (__any_sync(0xffffffffu, umax > kTauD)) {
 #pragma unroll
-                for (int i = 0; i < NC; ++i) {
-                    float tmax = red[(cg * 4 + 0) * NC + i];
-#pragma unroll
-                    for (int q = 1; q < 4; ++q) tmax = fmaxf(tmax, red[(cg * 4 + q) * NC + i]);
-                    float a = 1.f;
-                    if (m_neg[i] == INFINITY) {
-                        // First key of the row: it fixes m_O = m.
-                        if (tmax > -INFINITY) m_neg[i] = -tmax;
-                    } else if (tmax + m_neg[i] > kTauD) {
-                        // Move m up by a whole number of binades, so the change is
-                        // an exact power of two in P's scale.
-                        const int de = static_cast<int>(ceilf(tmax + m_neg[i]));
-                        m_neg[i] -= static_cast<float>(de);
-                        const int ne = e_off[i] + de;
-                        __syncwarp();
-                        if (lane == 0) e_off[i] = ne;
-                        a = de < 126 ? __uint_as_float(static_cast<uint32_t>(127 - de) << 23) : 0.f;
-                        changed = true;
-                        over |= ne > kEMaxD;
-                    }
-                    lacc[i] *= a;
-                    if (u[i] != -INFINITY) u[i] = fmaf(__uint_as_float(sre[i]), sc, m_neg[i]);
-                }
-                __syncwarp();
-                if (changed) sf_dirty = 2;
-                // Past kEMaxD binades O itself is brought to the current reference:
-                // O *= 2^-e once PV(it-1) is done, and e restarts at 0.
-                if (__any_sync(0xffffffffu, over)) {
-                    __syncwarp();
                     for (int i = 0; i < NC; ++i) {
-                        const int ee = e_off[i] > kEMaxD ? e_off[i] : 0;
-                        __syncwarp();
-                        if (lane == 0) {
-                            alpha_s[i] = ee < 126 ? __uint_as_float(static_cast<uint32_t>(127 - ee) << 23) : 0.f;
-                            if (ee) e_off[i] = 0;
+                        if (i >= nv) break;
+                        const float mx = warp_max_f32(u[i]);
+                        if (mx > kTauD) {
+                            const float de = ceilf(fminf(mx, kMaxMoveD));
+                            u[i] -= de;
+                            const int dei = static_cast<int>(de);
+                            lacc[i] *= exp2_neg_int(dei);
+                            if (lane == i) {
+                                m_neg[i] -= de;
+                                e_mine += dei;
+                            }
                         }
                     }
                     __syncwarp();
-                    if (it >= 1) {
-                        bool okw = wait_bar(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag, p.status);
-                        if (__all_sync(0xffffffffu, okw)) {
-                            tc_fence_after();
-                            uint32_t ohi[NC], olo[NC];
-                            tmem_load_cols<NC>(tmem + lane_base + Lay::kColO + c0, ohi);
-                            tmem_load_cols<NC>(tmem + lane_base + Lay::kColO + NT + c0, olo);
-                            tc_wait_ld();
-#pragma unroll
-                            for (int c = 0; c < NC; ++c) {
-                                const float a = alpha_s[c];
-                                ohi[c] = __float_as_uint(__uint_as_float(ohi[c]) * a);
-                                olo[c] = __float_as_uint(__uint_as_float(olo[c]) * a);
-                            }
-                            tmem_store_cols<NC>(tmem + lane_base + Lay::kColO + c0, ohi);
-                            tmem_store_cols<NC>(tmem + lane_base + Lay::kColO + NT + c0, olo);
-                            tc_wait_st();
-                        }
-                    }
-                    sf_dirty = 2;
                 }
+            }
+            // Post this warp's vote for the tile: bit 0, an offset past kEMaxD (O must
+            // be rescaled before PV of this tile); bit 1, the CTA is unwinding.
+            const bool over = __any_sync(0xffffffffu, lane < NC && e_mine > kEMaxD);
+            if (lane == 0) {
+                votes[sbuf * 4 + quarter] = (over ? 1u : 0u) | (*abort_flag ? 2u : 0u);
+                mbar_arrive(&vote_bar[2 * cg + sbuf]);
             }
             // P buffer `sbuf` was last read by PV(it-2).
             if (it >= 2) {
                 bool okw = wait_bar(&pv_done[sbuf], ((it >> 1) & 1) ^ 1, abort_flag, p.status);
                 (void)__all_sync(0xffffffffu, okw);
             }
+            // Encode P^T bytes. P_hi = E4M3(p). Its value comes back exactly from the
+            // code's 7 magnitude bits placed at bit 20 of a float, times 2^120: f32
+            // and E4M3 treat their lowest exponent alike, so subnormal codes decode
+            // the same way. P_lo = E4M3(32 (p - P_hi)) carries the next bits.
             uint8_t *pb = smem + Lay::kP + sbuf * Lay::kPBytes;
-            if (sf_dirty > 0) {
-                // This buffer's scale atom: byte `quarter` (this warp's 32 keys) of
-                // rows c0+i (P_hi, 2^e) and NT+c0+i (P_lo, 2^(e-5)).
-                if (lane == 0) {
-                    uint8_t *atom = smem + Lay::kSfP + sbuf * 512;
-#pragma unroll
-                    for (int i = 0; i < NC; ++i) {
-                        const int n = c0 + i, nl = NT + c0 + i;
-                        atom[(n & 31) * 16 + (n >> 5) * 4 + quarter] = static_cast<uint8_t>(127 + e_off[i]);
-                        atom[(nl & 31) * 16 + (nl >> 5) * 4 + quarter] = static_cast<uint8_t>(122 + e_off[i]);
-                    }
-                }
-                --sf_dirty;
-            }
 #pragma unroll
             for (int i = 0; i < NC; i += 2) {
                 if (i >= nv) break;
                 const float p0 = exp2_approx(u[i]);
                 const float p1 = exp2_approx(u[i + 1]);
-                const uint16_t h2 = cvt_e4m3x2(p0, p1);
-                const uint32_t hv = cvt_e4m3x2_to_f16x2(h2);
-                const __half2 ph = __floats2half2_rn(p0, p1);
-                const __half2 r = __hmul2(__hsub2(ph, *reinterpret_cast<const __half2 *>(&hv)),
-                                          __float2half2_rn(32.f));
-                const uint16_t l2 = cvt_e4m3x2_from_h2(*reinterpret_cast<const uint32_t *>(&r));
-                const uint32_t lv = cvt_e4m3x2_to_f16x2(l2);
-                const __half2 pt = __hfma2(*reinterpret_cast<const __half2 *>(&lv), __float2half2_rn(0.03125f),
-                                           *reinterpret_cast<const __half2 *>(&hv));
-                const float2 ptf = __half22float2(pt);
-                lacc[i] += ptf.x;
-                lacc[i + 1] += ptf.y;
-                const int o0 = pbase + ((pchunk ^ (i & 7)) << 4) + i * 128;
-                const int o1 = pbase + ((pchunk ^ ((i + 1) & 7)) << 4) + (i + 1) * 128;
+                lacc[i] += p0;
+                lacc[i + 1] += p1;
+                const uint32_t h2 = cvt_e4m3x2(p0, p1);
+                const float hv0 = __uint_as_float((h2 << 20) & 0x0FF00000u);
+                const float hv1 = __uint_as_float((h2 << 12) & 0x0FF00000u);
+                const float d0 = fmaf(hv0, -0x1p125f, p0 * 32.f);
+                const float d1 = fmaf(hv1, -0x1p125f, p1 * 32.f);
+                const uint32_t l2 = cvt_e4m3x2(d0, d1);
+                const int o0 = (pofs ^ ((i & 7) << 4)) + i * 128;
+                const int o1 = (pofs ^ (((i + 1) & 7) << 4)) + (i + 1) * 128;
                 st_u8(pb, o0, h2);
                 st_u8(pb, o0 + NT * 128, l2);
                 if (i + 1 < nv) {
@@ -573,25 +563,81 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
                     st_u8(pb, o1 + NT * 128, l2 >> 8);
                 }
             }
+            // Collect the vote. Every warp of the group reads the same four words.
+            const bool okv = wait_bar_peers(&vote_bar[2 * cg + sbuf], (it >> 1) & 1);
+            const uint32_t flags = okv ? (votes[sbuf * 4] | votes[sbuf * 4 + 1] | votes[sbuf * 4 + 2] |
+                                          votes[sbuf * 4 + 3])
+                                       : 2u;
+            if (flags & 2u) break;
+            if (flags & 1u) {
+                // Some warp's offset passed kEMaxD: move m_O of each such row up by the
+                // largest offset E among the group's warps. O (which holds PV up to
+                // tile it-1) is scaled by 2^-E, every warp's offset drops by E, and
+                // P bytes, being relative to each warp's own m, stay as they are.
+                if (lane < NC) xe[quarter * NC + lane] = e_mine;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xe_bar[cg]);
+                const bool okx = wait_bar_peers(&xe_bar[cg], n_rescales & 1);
+                ++n_rescales;
+                int E = 0;
+                if (okx && lane < NC) {
+                    E = imax(imax(xe[lane], xe[NC + lane]), imax(xe[2 * NC + lane], xe[3 * NC + lane]));
+                    if (E <= kEMaxD) E = 0;
+                    e_mine -= E;
+                }
+                if (okx && it >= 1) {
+                    bool okw = wait_bar(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag, p.status);
+                    if (__all_sync(0xffffffffu, okw)) {
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int c8 = 0; c8 < NC; c8 += 8) {
+                            uint32_t ohi[8], olo[8];
+                            tmem_load_cols<8>(tmem + lane_base + Lay::kColO + c0 + c8, ohi);
+                            tmem_load_cols<8>(tmem + lane_base + Lay::kColO + NT + c0 + c8, olo);
+                            tc_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const float a = exp2_neg_int(__shfl_sync(0xffffffffu, E, c8 + c));
+                                ohi[c] = __float_as_uint(__uint_as_float(ohi[c]) * a);
+                                olo[c] = __float_as_uint(__uint_as_float(olo[c]) * a);
+                            }
+                            tmem_store_cols<8>(tmem + lane_base + Lay::kColO + c0 + c8, ohi);
+                            tmem_store_cols<8>(tmem + lane_base + Lay::kColO + NT + c0 + c8, olo);
+                        }
+                        tc_wait_st();
+                    }
+                }
+            }
+            // Scale bytes of this warp's key block (byte `quarter`) in the buffer's
+            // atom: row c0+i (P_hi) gets 2^e, row NT+c0+i (P_lo) 2^(e-5). An offset
+            // far below m_O clamps at the smallest E8M0 value; such a block is
+            // negligible against the row's maximum.
+            if (lane < NC) {
+                uint8_t *atom = smem + Lay::kSfP + sbuf * 512;
+                const int n = c0 + lane, nl = NT + c0 + lane;
+                atom[(n & 31) * 16 + (n >> 5) * 4 + quarter] = static_cast<uint8_t>(imax(0, 127 + e_mine));
+                atom[(nl & 31) * 16 + (nl >> 5) * 4 + quarter] = static_cast<uint8_t>(imax(0, 122 + e_mine));
+            }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[sbuf]);
         }
         // ----------------------------------------------------------------- epilogue
-        if (ok) {
-            ok = wait_bar(o_final, 0, abort_flag, p.status);
-            ok = __all_sync(0xffffffffu, ok);
-        }
-        // Row denominators: sum the per-token partial sums over the 128 lanes.
+        bool ok = !*abort_flag;
+        if (ok) ok = wait_bar(o_final, 0, abort_flag, p.status);
+        ok = __all_sync(0xffffffffu, ok);
+        // Row sums: over this warp's lanes, then over the group's four warps, each
+        // scaled from its own m to m_O by 2^e.
 #pragma unroll
         for (int i = 0; i < NC; ++i) {
             float v = lacc[i];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) lsum[(cg * 4 + quarter) * NC + i] = v;
+            if (lane == 0) lsum[quarter * NC + i] = v;
         }
-        bar_sync(kBarEpi, kSoftmaxThreads);
+        if (lane < NC) esum[quarter * NC + lane] = e_mine;
+        bar_sync(gbar, 128);
         if (ok && !*abort_flag) {
             tc_fence_after();
 #pragma unroll
@@ -605,19 +651,20 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
                 for (int e = 0; e < 4; ++e) {
                     const int i = c + e;
                     if (i >= nv) break;
-                    const float l = lsum[(cg * 4 + 0) * NC + i] + lsum[(cg * 4 + 1) * NC + i] +
-                                    lsum[(cg * 4 + 2) * NC + i] + lsum[(cg * 4 + 3) * NC + i];
-                    const bool any = l > 0.f && m_neg[i] < INFINITY;
+                    float l = 0.f;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) l += ldexpf(lsum[q * NC + i], esum[q * NC + i]);
+                    const bool any = l > 0.f;
                     const int64_t row = partial_row(c0 + i);
-                    // O is relative to m_O = m - e: divide by l * 2^e.
-                    const float inv = any ? __uint_as_float(static_cast<uint32_t>(127 - e_off[i]) << 23) / l : 0.f;
-                    p.ws_o[row * 128 + jt] = (__uint_as_float(ohi[e]) + __uint_as_float(olo[e])) * inv;
-                    if (jt == 0) p.ws_lse[row] = any ? log2f(l) - m_neg[i] : -INFINITY;
+                    // O and l are both relative to m_O = m - e.
+                    p.ws_o[row * 128 + jt] = any ? (__uint_as_float(ohi[e]) + __uint_as_float(olo[e])) / l : 0.f;
+                    if (jt == 0)
+                        p.ws_lse[row] = any ? log2f(l) - m_neg[i] - static_cast<float>(esum[quarter * NC + i])
+                                            : -INFINITY;
                 }
             }
         }
     }
-
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -650,7 +697,7 @@ cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const At
     const int R = p.G * p.Sq;
     if (R <= 16) return launch_nt<16, 16, kDecodeSmallStages, 2>(tk, tv, p, grid, stream);
     if (R <= 32) return launch_nt<32, 16, 6, 1>(tk, tv, p, grid, stream);
-    return launch_nt<64, 16, 6, 1>(tk, tv, p, grid, stream);
+    return launch_nt<64, 32, 6, 1>(tk, tv, p, grid, stream);
 }
 
 }  // namespace qk4v8

@@ -151,8 +151,14 @@ QK4V8_API int qk4v8_attention_prefill(const uint8_t *q_codes, const uint8_t *q_s
 /* Workspace bytes for qk4v8_attention_decode with these sizes. */
 QK4V8_API size_t qk4v8_decode_workspace_bytes(int B, int Hq, int nq, int num_splits);
 
-/* The split count qk4v8_attention_decode picks when given num_splits = 0. */
-QK4V8_API int qk4v8_decode_default_splits(int B, int Hkv, int max_seqlen);
+/*
+ * The split count qk4v8_attention_decode picks when given num_splits = 0 for
+ * B sequences of Hkv KV heads, (Hq / Hkv) * nq query rows per KV head and keys
+ * up to max_seqlen: the count that minimises the modelled time of the waves of
+ * CTAs on the current device (148 SMs when no device can be queried). Returns
+ * 1 for invalid sizes.
+ */
+QK4V8_API int qk4v8_decode_default_splits(int B, int Hq, int Hkv, int nq, int max_seqlen);
 
 /*
  * The two stages of qk4v8_attention_decode, as separate launches.
