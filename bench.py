@@ -3,11 +3,12 @@
 
 One step is one pass of the decode hot path over one batch of the GQA decode
 workload: B=32, Hq=32, Hkv=8, one query token, KV length 8192, d=128, four
-outlier channels x16 in Q and K. The step has three launches:
-  1. MXFP4 quantization of the step's query tokens;
-  2. the split-KV block-scaled tcgen05 attention over the pre-quantized
-     MXFP4-K / MXFP8-V cache;
-  3. the merge of the split partials.
+outlier channels x16 in Q and K. The step is one library call,
+qk4v8_attention_decode_bf16: the split-KV block-scaled tcgen05 attention over
+the pre-quantized MXFP4-K / MXFP8-V cache, which MXFP4-quantizes the step's
+bf16 query rows itself. With one KV split (the library's choice for this
+workload) that is a single launch that also writes the bf16 output; with
+more splits a merge launch follows.
 `value` is the packed KV bytes streamed per second, summed over all ranks
 (weak scaling: every rank runs its own copy of the workload, with no
 collective on the data path).
@@ -164,6 +165,17 @@ def to_dev(bits):
 
 # ----------------------------------------------------------------------------- decode
 
+def decode_kernel_name(rows: int) -> str:
+    """The split-KV kernel the library launches for `rows` = (Hq / Hkv) * nq query rows per KV head."""
+    if rows <= 16:
+        return "qk4v8_decode_kernel<16,16,3,2> (swap-AB split-KV decode)"
+    if rows <= 32:
+        return "qk4v8_decode_kernel<32,16,6,1> (swap-AB split-KV decode)"
+    if rows <= 64:
+        return "qk4v8_decode_kernel<64,32,6,1> (swap-AB split-KV decode)"
+    return "qk4v8_attention_kernel<true> (128-row split-KV decode)"
+
+
 def run_decode(args, world, rank):
     import torch
     import bit_quantized_attention_qk4v8_b200 as qk
@@ -175,40 +187,47 @@ def run_decode(args, world, rank):
     sl = torch.from_numpy(gen["seqlens"]).cuda()
     kp = qk.quantize_qk(to_dev(gen["k"]), seqlens=sl)      # the cache: quantized once, outside the timing
     vp = qk.quantize_v(to_dev(gen["v"]), seqlens=sl)
-    qp = qk.quantize_qk(q)
-    splits = args.splits if args.splits > 0 else qk.decode_default_splits(wl.B, wl.Hkv, wl.Lk)
-    ws = torch.empty((qk.decode_workspace_bytes(wl.B, wl.Hq, wl.Sq, splits),), dtype=torch.uint8, device="cuda")
+    splits = args.splits if args.splits > 0 else qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, wl.Lk)
+    ws_bytes = qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device="cuda") if ws_bytes else None
     out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
     kv_bytes = wl.B * wl.Hkv * wl.Lk * KV_BYTES_PER_TOKEN_HEAD
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-
-    def step(i=None):
-        qk.quantize_qk(q, out=qp)
-        if i is not None:
-            ev[i][0].record(stream)
-        qk.attention_decode_splitkv(qp, kp, vp, sl, wl.Lk, splits, ws)
-        if i is not None:
-            ev[i][1].record(stream)
-        qk.decode_merge(ws, wl.B, wl.Hq, wl.Sq, splits, out)
+    def step():
+        qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=wl.Lk, num_splits=splits, workspace=ws, out=out)
 
     for _ in range(args.warmup):
         step()
+    torch.cuda.synchronize()
+    # The K timed steps run as one CUDA graph, so host launch overhead does not
+    # pace the device. An event pair (graph event-record nodes) brackets each
+    # step's attention call for the kernel's own duration (with one split the
+    # call is that one kernel; with more, the merge is inside the pair too).
+    ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+          for _ in range(args.steps)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cap = torch.cuda.current_stream()
+        for i in range(args.steps):
+            ev[i][0].record(cap)
+            qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=wl.Lk, num_splits=splits, workspace=ws, out=out)
+            ev[i][1].record(cap)
+    graph.replay()          # untimed first replay uploads the graph
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
         t0.record(stream)
-        for i in range(args.steps):
-            step(i)
+        graph.replay()
         t1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world)
     attn_ms = [a.elapsed_time(b) for a, b in ev]
     attn_avg_ms = statistics.fmean(attn_ms)
+    del graph
 
     # e2e: the public API with host buffers; the step's query is copied in and
     # its output copied back every step.
@@ -217,8 +236,7 @@ def run_decode(args, world, rank):
 
     def e2e_step():
         q.copy_(q_host, non_blocking=True)
-        qk.quantize_qk(q, out=qp)
-        qk.attention_decode(qp, kp, vp, sl, max_seqlen=wl.Lk, num_splits=splits, workspace=ws, out=out)
+        qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=wl.Lk, num_splits=splits, workspace=ws, out=out)
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(min(args.warmup, 5)):
@@ -234,7 +252,10 @@ def run_decode(args, world, rank):
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
 
+    rows = wl.G * wl.Sq
+    launches = (1 if rows <= 64 else 2) + (0 if splits == 1 and rows <= 64 else 1)
     return dict(wl=wl, gen=gen, kv_bytes=kv_bytes, splits=splits, elapsed_ms=elapsed_ms, attn_avg_ms=attn_avg_ms,
+                launches_per_step=launches,
                 clocks=clk.summary(), e2e_ms=e2e_ms, e2e_steps=e2e_steps,
                 h2d=q_host.numel() * 2, d2h=out_host.numel() * 2)
 
@@ -410,14 +431,14 @@ def main():
             "tokens_per_s": wl.B * wl.Sq * steps * world / (d["elapsed_ms"] * 1e-3),
         },
         "roofline": {
-            "bound": "hbm", "kernel": "qk4v8_attention_kernel<true> (split-KV decode)",
+            "bound": "hbm", "kernel": decode_kernel_name(wl.G * wl.Sq),
             "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
             "peak_source": f"{peak_src} hbm_gbs", "traffic": None,
             "algorithmic_bytes_per_launch": d["kv_bytes"], "avg_launch_ms": d["attn_avg_ms"],
         },
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": d["h2d"], "d2h_bytes_per_step": d["d2h"],
                 "steps": d["e2e_steps"]},
-        "gpu_launches": 3 * steps,
+        "gpu_launches": d["launches_per_step"] * steps,
         "clocks": d["clocks"],
     }
 

@@ -25,6 +25,7 @@ __all__ = [
     "MXFP4", "MXFP8V", "QK4V8Error", "lib", "round_cap",
     "quantize_qk", "quantize_v", "quantize", "attention_prefill", "attention_decode",
     "decode_workspace_bytes", "decode_default_splits", "attention_decode_splitkv", "decode_merge",
+    "attention_decode_bf16", "decode_bf16_workspace_bytes",
 ]
 
 D = 128
@@ -190,6 +191,41 @@ def attention_decode(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optio
                                        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                        out.data_ptr(), _ptr(lse), _ptr(dev_status), _stream(dev)),
           "qk4v8_attention_decode")
+    return (out, lse) if return_lse else out
+
+
+def decode_bf16_workspace_bytes(B: int, Hq: int, Hkv: int, nq: int, num_splits: int) -> int:
+    return int(lib().qk4v8_decode_bf16_workspace_bytes(B, Hq, Hkv, nq, num_splits))
+
+
+def attention_decode_bf16(q: torch.Tensor, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optional[int] = None,
+                          causal_in_block: bool = True, softmax_scale: Optional[float] = None, num_splits: int = 0,
+                          workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                          lse: Optional[torch.Tensor] = None, return_lse: bool = False,
+                          dev_status: Optional[torch.Tensor] = None):
+    """Decode step from bf16 queries q [B, nq, Hq, 128]; the query is MXFP4-quantized inside the call.
+    Returns out bf16 [B, nq, Hq, 128] (and lse [B, Hq, nq])."""
+    _check_bf16(q, "q")
+    dev = q.device
+    B, nq, Hq, _ = q.shape
+    sl = _seqlens(seqlens_k, B, dev)
+    if max_seqlen is None:
+        max_seqlen = k.cap
+    splits = num_splits if num_splits > 0 else decode_default_splits(B, Hq, k.H, nq, max_seqlen)
+    need = decode_bf16_workspace_bytes(B, Hq, k.H, nq, splits)
+    if workspace is None and need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((B, nq, Hq, D), dtype=torch.bfloat16, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, nq), dtype=torch.float32, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib().qk4v8_attention_decode_bf16(q.data_ptr(), B, Hq, nq, q.stride(0), q.stride(1), q.stride(2),
+                                            k.codes.data_ptr(), k.scales.data_ptr(), v.codes.data_ptr(),
+                                            v.scales.data_ptr(), k.H, k.cap, _ptr(sl), int(max_seqlen),
+                                            int(bool(causal_in_block)), float(softmax_scale or 0.0), int(splits),
+                                            _ptr(workspace), ws_bytes, out.data_ptr(), _ptr(lse), _ptr(dev_status),
+                                            _stream(dev)), "qk4v8_attention_decode_bf16")
     return (out, lse) if return_lse else out
 
 

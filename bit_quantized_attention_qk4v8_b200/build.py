@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqk4v8.so")
 SOURCES = ["quantize.cu", "attention.cu", "decode.cu", "api.cu"]
-HEADERS = ["ptx.cuh", "pipeline.cuh", "qk4v8_internal.h"]
+HEADERS = ["ptx.cuh", "pipeline.cuh", "mx_encode.cuh", "qk4v8_internal.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -276,31 +276,55 @@ int qk4v8_decode_default_splits(int B, int Hq, int Hkv, int nq, int max_seqlen) 
 
 namespace {
 
+// Query of a decode call: packed MXFP4 (codes, scales, cap) or bf16 rows
+// [b][t][h][128] with element strides, quantized inside the kernel.
+struct DecodeQuery {
+    const uint8_t *codes = nullptr;
+    const uint8_t *scales = nullptr;
+    int cap = 0;
+    const __nv_bfloat16 *bf16 = nullptr;
+    int64_t sb = 0, st = 0, sh = 0;
+};
+
+bool swap_ab_rows(int Hq, int Hkv, int nq) { return (Hq / Hkv) * nq <= qk4v8::kDecodeMaxRows; }
+
 // Validates decode arguments, builds the tensor maps and launches the split-KV
-// kernel; the caller decides whether the merge follows.
-int decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
-                   const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes, const uint8_t *v_scales,
-                   int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen, int causal_in_block,
-                   float softmax_scale, int num_splits, void *workspace, size_t workspace_bytes, int32_t *dev_status,
-                   cudaStream_t stream, int *splits_used) {
+// kernel. With `out` given and a single split on the swap-AB kernel, the kernel
+// writes out (and lse) itself and *direct is set; otherwise it writes the split
+// partials to the workspace and the caller runs the merge.
+int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k_codes, const uint8_t *k_scales,
+                   const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k,
+                   int max_seqlen, int causal_in_block, float softmax_scale, int num_splits, void *workspace,
+                   size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, cudaStream_t stream,
+                   int *splits_used, bool *direct) {
     int st;
-    if ((st = validate_packed(q_codes, q_scales, "Q")) || (st = validate_packed(k_codes, k_scales, "K")) ||
-        (st = validate_packed(v_codes, v_scales, "V")))
+    if (q.bf16) {
+        if (!aligned16(q.bf16) || q.sb % 8 || q.st % 8 || q.sh % 8 || q.sb < 0 || q.st < 0 || q.sh < 0)
+            return set_error(QK4V8_ERR_INVALID_ARG, "bf16 Q must be 16-byte aligned with strides of whole 8-element "
+                                                    "(16-byte) units");
+    } else if ((st = validate_packed(q.codes, q.scales, "Q"))) {
         return st;
+    }
+    if ((st = validate_packed(k_codes, k_scales, "K")) || (st = validate_packed(v_codes, v_scales, "V"))) return st;
     if (!seqlens_k) return set_error(QK4V8_ERR_INVALID_ARG, "decode needs seqlens_k");
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv)
         return set_error(QK4V8_ERR_INVALID_ARG, "bad heads B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
     if (nq < 1 || nq > 8 || (Hq / Hkv) * nq > 128)
         return set_error(QK4V8_ERR_INVALID_ARG, "need 1 <= nq <= 8 and (Hq/Hkv)*nq <= 128 (nq=%d G=%d)", nq,
                          Hq / Hkv);
-    if (q_cap <= 0 || q_cap % 128 || q_cap < nq || kv_cap <= 0 || kv_cap % 128 || max_seqlen < 0 ||
+    if ((!q.bf16 && (q.cap <= 0 || q.cap % 128 || q.cap < nq)) || kv_cap <= 0 || kv_cap % 128 || max_seqlen < 0 ||
         max_seqlen > kv_cap)
-        return set_error(QK4V8_ERR_INVALID_ARG, "bad lengths q_cap=%d kv_cap=%d max_seqlen=%d", q_cap, kv_cap,
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad lengths q_cap=%d kv_cap=%d max_seqlen=%d", q.cap, kv_cap,
                          max_seqlen);
+    if (q.bf16 && !swap_ab_rows(Hq, Hkv, nq))
+        return set_error(QK4V8_ERR_INVALID_ARG, "bf16 Q in the split kernel needs (Hq/Hkv)*nq <= %d",
+                         qk4v8::kDecodeMaxRows);
     if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
     const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen);
-    const size_t need = qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
-    if (!workspace || !aligned16(workspace) || workspace_bytes < need)
+    const bool direct_out = out && splits == 1 && swap_ab_rows(Hq, Hkv, nq);
+    if (out && !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
+    const size_t need = direct_out ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
+    if (need && (!workspace || !aligned16(workspace) || workspace_bytes < need))
         return set_error(QK4V8_ERR_INVALID_ARG, "workspace must be 16-byte aligned and >= %zu bytes", need);
     if ((st = check_device())) return st;
     CUtensorMap tk, tv;
@@ -308,8 +332,12 @@ int decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scales, int B, int H
         return st;
     const int tiles = (max_seqlen + 127) / 128;
     qk4v8::AttnParams p{};
-    p.q_codes = q_codes;
-    p.q_scales = q_scales;
+    p.q_codes = q.codes;
+    p.q_scales = q.scales;
+    p.q_bf16 = q.bf16;
+    p.q_sb = q.sb;
+    p.q_st = q.st;
+    p.q_sh = q.sh;
     p.k_scales = k_scales;
     p.v_scales = v_scales;
     p.seqlens = seqlens_k;
@@ -318,7 +346,7 @@ int decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scales, int B, int H
     p.Hkv = Hkv;
     p.G = Hq / Hkv;
     p.Sq = nq;
-    p.q_cap = q_cap;
+    p.q_cap = q.cap;
     p.kv_cap = kv_cap;
     p.Lk = max_seqlen;
     p.causal = causal_in_block ? 1 : 0;
@@ -327,19 +355,25 @@ int decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scales, int B, int H
     p.n_qtiles = 1;
     p.num_splits = splits;
     p.split_tiles = tiles > 0 ? (tiles + splits - 1) / splits : 1;
-    const size_t rows = static_cast<size_t>(B) * Hq * nq * splits;
-    p.ws_o = static_cast<float *>(workspace);
-    p.ws_lse = p.ws_o + rows * 128;
+    if (direct_out) {
+        p.direct_out = 1;
+        p.out = static_cast<__nv_bfloat16 *>(out);
+        p.lse = lse;
+    } else {
+        const size_t rows = static_cast<size_t>(B) * Hq * nq * splits;
+        p.ws_o = static_cast<float *>(workspace);
+        p.ws_lse = p.ws_o + rows * 128;
+    }
     p.status = dev_status;
     p.test_stall = g_test_stall;
     p.test_dump_s = g_test_dump_s;
     // G*nq <= 64 query rows: the swap-AB decode kernel; larger groups use the
     // 128-row attention kernel in its decode instantiation.
-    cudaError_t e = (Hq / Hkv) * nq <= qk4v8::kDecodeMaxRows
-                        ? qk4v8::launch_decode(tk, tv, p, B * Hkv * splits, stream)
-                        : qk4v8::launch_attention(tk, tv, p, B * Hkv * splits, stream);
+    cudaError_t e = swap_ab_rows(Hq, Hkv, nq) ? qk4v8::launch_decode(tk, tv, p, B * Hkv * splits, stream)
+                                              : qk4v8::launch_attention(tk, tv, p, B * Hkv * splits, stream);
     if (e != cudaSuccess) return cuda_error(e, "attention (decode) launch");
     *splits_used = splits;
+    *direct = direct_out;
     return QK4V8_OK;
 }
 
@@ -353,9 +387,14 @@ int qk4v8_attention_decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scal
                                    int max_seqlen, int causal_in_block, float softmax_scale, int num_splits,
                                    void *workspace, size_t workspace_bytes, int32_t *dev_status, void *stream) {
     int splits = 0;
-    return decode_splitkv(q_codes, q_scales, B, Hq, nq, q_cap, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap,
-                          seqlens_k, max_seqlen, causal_in_block, softmax_scale, num_splits, workspace,
-                          workspace_bytes, dev_status, static_cast<cudaStream_t>(stream), &splits);
+    bool direct = false;
+    DecodeQuery q;
+    q.codes = q_codes;
+    q.scales = q_scales;
+    q.cap = q_cap;
+    return decode_splitkv(q, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
+                          causal_in_block, softmax_scale, num_splits, workspace, workspace_bytes, nullptr, nullptr,
+                          dev_status, static_cast<cudaStream_t>(stream), &splits, &direct);
 }
 
 int qk4v8_decode_merge(const void *workspace, size_t workspace_bytes, int B, int Hq, int nq, int num_splits,
@@ -385,11 +424,73 @@ int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int 
                            size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, void *stream) {
     if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
     int splits = 0;
-    int st = decode_splitkv(q_codes, q_scales, B, Hq, nq, q_cap, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap,
-                            seqlens_k, max_seqlen, causal_in_block, softmax_scale, num_splits, workspace,
-                            workspace_bytes, dev_status, static_cast<cudaStream_t>(stream), &splits);
-    if (st) return st;
+    bool direct = false;
+    DecodeQuery q;
+    q.codes = q_codes;
+    q.scales = q_scales;
+    q.cap = q_cap;
+    int st = decode_splitkv(q, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
+                            causal_in_block, softmax_scale, num_splits, workspace, workspace_bytes, out, lse,
+                            dev_status, static_cast<cudaStream_t>(stream), &splits, &direct);
+    if (st || direct) return st;
     return qk4v8_decode_merge(workspace, workspace_bytes, B, Hq, nq, splits, out, lse, stream);
+}
+
+size_t qk4v8_decode_bf16_workspace_bytes(int B, int Hq, int Hkv, int nq, int num_splits) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq <= 0 || num_splits <= 0) return 0;
+    if (swap_ab_rows(Hq, Hkv, nq)) return num_splits == 1 ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits);
+    // Larger groups: the queries are quantized into the front of the workspace
+    // (capacity 128 tokens), then the split partials follow.
+    const size_t packed = qk4v8_mxfp4_codes_bytes(B, Hq, 128) + qk4v8_scales_bytes(B, Hq, 128);
+    return packed + qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits);
+}
+
+int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_stride_b, int64_t q_stride_t,
+                                int64_t q_stride_h, const uint8_t *k_codes, const uint8_t *k_scales,
+                                const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap,
+                                const int32_t *seqlens_k, int max_seqlen, int causal_in_block, float softmax_scale,
+                                int num_splits, void *workspace, size_t workspace_bytes, void *out, float *lse,
+                                int32_t *dev_status, void *stream) {
+    if (!q) return set_error(QK4V8_ERR_INVALID_ARG, "q is null");
+    if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq < 1 || nq > 8 || (Hq / Hkv) * nq > 128)
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad sizes B=%d Hq=%d Hkv=%d nq=%d", B, Hq, Hkv, nq);
+    if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
+    const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen);
+    const size_t need = qk4v8_decode_bf16_workspace_bytes(B, Hq, Hkv, nq, splits);
+    if (need && (!workspace || !aligned16(workspace) || workspace_bytes < need))
+        return set_error(QK4V8_ERR_INVALID_ARG, "workspace must be 16-byte aligned and >= %zu bytes", need);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int used = 0;
+    bool direct = false;
+    DecodeQuery dq;
+    if (swap_ab_rows(Hq, Hkv, nq)) {
+        dq.bf16 = static_cast<const __nv_bfloat16 *>(q);
+        dq.sb = q_stride_b;
+        dq.st = q_stride_t;
+        dq.sh = q_stride_h;
+        int st = decode_splitkv(dq, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k,
+                                max_seqlen, causal_in_block, softmax_scale, splits, workspace, workspace_bytes, out,
+                                lse, dev_status, s, &used, &direct);
+        if (st || direct) return st;
+        return qk4v8_decode_merge(workspace, workspace_bytes, B, Hq, nq, used, out, lse, stream);
+    }
+    // More than 64 query rows per KV head: quantize Q into the front of the
+    // workspace for the 128-row kernel.
+    uint8_t *qc = static_cast<uint8_t *>(workspace);
+    uint8_t *qs = qc + qk4v8_mxfp4_codes_bytes(B, Hq, 128);
+    uint8_t *rest = qs + qk4v8_scales_bytes(B, Hq, 128);
+    const size_t rest_bytes = workspace_bytes - static_cast<size_t>(rest - qc);
+    int st = qk4v8_quantize_qk(q, B, nq, Hq, 128, q_stride_b, q_stride_t, q_stride_h, nullptr, 128, qc, qs, stream);
+    if (st) return st;
+    dq.codes = qc;
+    dq.scales = qs;
+    dq.cap = 128;
+    st = decode_splitkv(dq, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
+                        causal_in_block, softmax_scale, splits, rest, rest_bytes, nullptr, nullptr, dev_status, s,
+                        &used, &direct);
+    if (st) return st;
+    return qk4v8_decode_merge(rest, rest_bytes, B, Hq, nq, used, out, lse, stream);
 }
 
 // Test hook (declared in include/qk4v8_test.h): while enabled, attention

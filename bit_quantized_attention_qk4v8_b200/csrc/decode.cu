@@ -33,6 +33,7 @@
 
 #include <cstdint>
 
+#include "mx_encode.cuh"
 #include "pipeline.cuh"
 #include "ptx.cuh"
 #include "qk4v8_internal.h"
@@ -150,6 +151,17 @@ __device__ __forceinline__ bool wait_bar_peers(uint64_t *bar, uint32_t parity) {
     return mbar_try_wait(bar, parity) || wait_bar_peers_slow(bar, parity);
 }
 
+// One lane of the (fully active) warp, chosen by elect.sync.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // 2^-k as a float for an integer k >= 0 (0 once it would be subnormal).
 __device__ __forceinline__ float exp2_neg_int(int k) {
     return k < 126 ? __uint_as_float(static_cast<uint32_t>(127 - k) << 23) : 0.f;
@@ -192,9 +204,16 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
         if (warp >= 2) {
             for (int idx = threadIdx.x - 64; idx < R * 32; idx += kSoftmaxThreads) {
                 const int n = idx >> 5, c4 = idx & 31;
-                const int64_t row = partial_row(n);
-                reinterpret_cast<float4 *>(p.ws_o + row * 128)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (c4 == 0) p.ws_lse[row] = -INFINITY;
+                if (p.direct_out) {
+                    const int h = h_kv * p.G + n / nq, t = n % nq;
+                    const int64_t orow = (static_cast<int64_t>(b) * nq + t) * p.Hq + h;
+                    reinterpret_cast<uint2 *>(p.out + orow * 128)[c4] = make_uint2(0, 0);
+                    if (c4 == 0 && p.lse) p.lse[(static_cast<int64_t>(b) * p.Hq + h) * nq + t] = -INFINITY;
+                } else {
+                    const int64_t row = partial_row(n);
+                    reinterpret_cast<float4 *>(p.ws_o + row * 128)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (c4 == 0) p.ws_lse[row] = -INFINITY;
+                }
             }
         }
         return;
@@ -220,7 +239,7 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
         }
-        mbar_init(q_full, 1);
+        mbar_init(q_full, Lay::kSoftmaxWarps);
         mbar_init(patch, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
@@ -253,40 +272,6 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
         }
-        // Q^T operand: row n < R is query head h_kv*G + n/nq at token n%nq; rows
-        // R..NT-1 are zero.
-        for (int c = lane; c < NT * 4; c += 32) {
-            const int n = c >> 2, j = c & 3;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (n < R) {
-                const int h = h_kv * p.G + n / nq, t = n % nq;
-                val = *reinterpret_cast<const uint4 *>(
-                    p.q_codes + ((static_cast<int64_t>(b) * p.Hq + h) * p.q_cap + t) * 64 + j * 16);
-            }
-            *reinterpret_cast<uint4 *>(smem + Lay::kQ + n * 64 + ((j ^ ((n >> 1) & 3)) << 4)) = val;
-        }
-        for (int n = lane; n < 128; n += 32) {
-            uint32_t scw = 0;
-            if (n < R) {
-                const int h = h_kv * p.G + n / nq, t = n % nq;
-                scw = *reinterpret_cast<const uint32_t *>(
-                    p.q_scales + ((static_cast<int64_t>(b) * p.Hq + h) * (p.q_cap / 128) + t / 128) * 512 +
-                    (t & 31) * 16 + ((t & 127) >> 5) * 4);
-            }
-            *reinterpret_cast<uint32_t *>(smem + Lay::kSfQ + (n & 31) * 16 + (n >> 5) * 4) = scw;
-            // P scale atoms: rows [0, NT) are P_hi (2^0), rows [NT, 2NT) P_lo (2^-5);
-            // the softmax raises a row's bytes when its reference max moves.
-            const uint32_t pw = n < NT ? kPhiScaleWord : kPloScaleWord;
-            *reinterpret_cast<uint32_t *>(smem + Lay::kSfP + (n & 31) * 16 + (n >> 5) * 4) = pw;
-            *reinterpret_cast<uint32_t *>(smem + Lay::kSfP + 512 + (n & 31) * 16 + (n >> 5) * 4) = pw;
-        }
-        // P^T buffers start at zero; rows of absent queries are never written again.
-        for (int c = lane; c < 2 * Lay::kPBytes / 16; c += 32)
-            reinterpret_cast<uint4 *>(smem + Lay::kP)[c] = make_uint4(0, 0, 0, 0);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && !p.test_stall) mbar_arrive(q_full);
-
         const int kvh = b * p.Hkv + h_kv;
         const int nblk = p.kv_cap / 128;
         int issued = 0;
@@ -336,65 +321,73 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
         }
     } else if (warp == 1) {
         // -------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            bool ok = wait_bar(q_full, 0, abort_flag, p.status);
-            if (ok) {
+        // The whole warp runs the loop and waits, so the descriptors stay
+        // warp-uniform; one elected lane issues the tcgen05 instructions.
+        const bool leader = elect_one();
+        bool ok = __all_sync(0xffffffffu, wait_bar(q_full, 0, abort_flag, p.status));
+        if (ok) {
+            tc_fence_after();
+            const uint32_t sb = smem_u32(smem);
+            constexpr uint32_t kIdQK = idesc_d(1u, NT);      // E2M1 x E2M1, N = NT
+            constexpr uint32_t kIdPV = idesc_d(0u, 2 * NT);  // E4M3 x E4M3, N = 2 NT
+            // Descriptors for stage 0 / buffer 0; other stages are fixed
+            // offsets of the 14-bit start-address field (in 16-byte units).
+            const uint64_t dQ = smem_desc(sb + Lay::kQ, 16, 512, 4);
+            const uint64_t dK0 = smem_desc(sb + Lay::kK, 16, 512, 4);
+            const uint64_t dV0 = smem_desc(sb + Lay::kV, 16, 1024, 2);
+            const uint64_t dP0 = smem_desc(sb + Lay::kP, 16, 1024, 2);
+            const uint64_t dSfK0 = smem_desc(sb + Lay::kSfK, 0, 128, 0);
+            const uint64_t dSfV0 = smem_desc(sb + Lay::kSfV, 0, 128, 0);
+            const uint64_t dSfP0 = smem_desc(sb + Lay::kSfP, 0, 128, 0);
+            if (leader) tc_cp_32x128b_warpx4(tmem + Lay::kColSfQ, smem_desc(sb + Lay::kSfQ, 0, 128, 0));
+            const uint32_t tO = tmem + Lay::kColO;
+            const uint32_t tSfQ = tmem + Lay::kColSfQ;
+            auto issue_pv = [&](int j) -> bool {
+                if (!__all_sync(0xffffffffu, wait_bar(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.status)))
+                    return false;
                 tc_fence_after();
-                const uint32_t sb = smem_u32(smem);
-                constexpr uint32_t kIdQK = idesc_d(1u, NT);      // E2M1 x E2M1, N = NT
-                constexpr uint32_t kIdPV = idesc_d(0u, 2 * NT);  // E4M3 x E4M3, N = 2 NT
-                // Descriptors for stage 0 / buffer 0; other stages are fixed
-                // offsets of the 14-bit start-address field (in 16-byte units).
-                const uint64_t dQ = smem_desc(sb + Lay::kQ, 16, 512, 4);
-                const uint64_t dK0 = smem_desc(sb + Lay::kK, 16, 512, 4);
-                const uint64_t dV0 = smem_desc(sb + Lay::kV, 16, 1024, 2);
-                const uint64_t dP0 = smem_desc(sb + Lay::kP, 16, 1024, 2);
-                const uint64_t dSfK0 = smem_desc(sb + Lay::kSfK, 0, 128, 0);
-                const uint64_t dSfV0 = smem_desc(sb + Lay::kSfV, 0, 128, 0);
-                tc_cp_32x128b_warpx4(tmem + Lay::kColSfQ, smem_desc(sb + Lay::kSfQ, 0, 128, 0));
-                const uint64_t dSfP0 = smem_desc(sb + Lay::kSfP, 0, 128, 0);
-                const uint32_t tO = tmem + Lay::kColO;
-                const uint32_t tSfQ = tmem + Lay::kColSfQ;
-                auto issue_pv = [&](int j) -> bool {
-                    if (!wait_bar(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.status)) return false;
-                    tc_fence_after();
-                    const int st = j % kStagesD;
-                    const uint32_t tSfV = tmem + col_sf_v_d(NT, j & 1);
-                    const uint32_t tSfP = tmem + col_sf_p_d(NT, j & 1);
+                const int st = j % kStagesD;
+                const uint32_t tSfV = tmem + col_sf_v_d(NT, j & 1);
+                const uint32_t tSfP = tmem + col_sf_p_d(NT, j & 1);
+                const uint64_t dV = dV0 + static_cast<uint64_t>(st * (Lay::kVBytes >> 4));
+                const uint64_t dP = dP0 + static_cast<uint64_t>((j & 1) * (Lay::kPBytes >> 4));
+                if (leader) {
                     tc_cp_32x128b_warpx4(tSfV, dSfV0 + static_cast<uint64_t>(st * 32));
                     tc_cp_32x128b_warpx4(tSfP, dSfP0 + static_cast<uint64_t>((j & 1) * 32));
-                    const uint64_t dV = dV0 + static_cast<uint64_t>(st * (Lay::kVBytes >> 4));
-                    const uint64_t dP = dP0 + static_cast<uint64_t>((j & 1) * (Lay::kPBytes >> 4));
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         tc_mma_mxf8(tO, dV + 2 * k, dP + 2 * k, sf_id_d(kIdPV, k), tSfV | (k << 30), tSfP | (k << 30),
                                     (j > 0 || k > 0) ? 1u : 0u);
                     tc_commit(&pv_done[j & 1]);
                     tc_commit(&kv_empty[st]);
-                    return true;
-                };
-                for (int it = 0; it < T && ok; ++it) {
-                    const int st = it % kStagesD;
-                    const int sbuf = it & 1;
-                    ok = wait_bar(&kv_full[st], (it / kStagesD) & 1, abort_flag, p.status);
-                    if (ok && last_partial && it == T - 1) ok = wait_bar(patch, 0, abort_flag, p.status);
-                    if (ok) ok = wait_bar(&s_free[sbuf], ((it >> 1) & 1) ^ 1, abort_flag, p.status);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t tSfK = tmem + col_sf_k_d(NT, sbuf);
+                }
+                __syncwarp();
+                return true;
+            };
+            for (int it = 0; it < T && ok; ++it) {
+                const int st = it % kStagesD;
+                const int sbuf = it & 1;
+                ok = wait_bar(&kv_full[st], (it / kStagesD) & 1, abort_flag, p.status);
+                if (ok && last_partial && it == T - 1) ok = wait_bar(patch, 0, abort_flag, p.status);
+                if (ok) ok = wait_bar(&s_free[sbuf], ((it >> 1) & 1) ^ 1, abort_flag, p.status);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                tc_fence_after();
+                const uint32_t tSfK = tmem + col_sf_k_d(NT, sbuf);
+                const uint64_t dK = dK0 + static_cast<uint64_t>(st * (Lay::kKBytes >> 4));
+                const uint32_t tS = tmem + static_cast<uint32_t>(NT * sbuf);
+                if (leader) {
                     tc_cp_32x128b_warpx4(tSfK, dSfK0 + static_cast<uint64_t>(st * 32));
-                    const uint64_t dK = dK0 + static_cast<uint64_t>(st * (Lay::kKBytes >> 4));
-                    const uint32_t tS = tmem + static_cast<uint32_t>(NT * sbuf);
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk)
                         tc_mma_mxf4(tS, dK + 2 * kk, dQ + 2 * kk, sf_id_d(kIdQK, 2 * kk), tSfK | ((2u * kk) << 30),
                                     tSfQ | ((2u * kk) << 30), kk > 0 ? 1u : 0u);
                     tc_commit(&s_full[sbuf]);
-                    if (it >= 1) ok = issue_pv(it - 1);
                 }
-                if (ok) ok = issue_pv(T - 1);
-                if (ok) tc_commit(o_final);
+                __syncwarp();
+                if (it >= 1) ok = issue_pv(it - 1);
             }
+            if (ok) ok = issue_pv(T - 1);
+            if (ok && leader) tc_commit(o_final);
         }
         __syncwarp();
     } else {
@@ -407,6 +400,70 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
         const int jt = quarter * 32 + lane;  // token within the tile, and channel in the epilogue
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         const int gbar = kBarGroup0 + cg;
+        {
+            // ------------------------------------------------------------ staging
+            // Q^T operand: row n < R is query head h_kv*G + n/nq at token n%nq;
+            // rows R..NT-1, and scale rows past NT, are zero.
+            const int stid = threadIdx.x - 64;
+            if (p.q_bf16) {
+                // MXFP4-encode the bf16 query rows here, 16 lanes per row, with
+                // the encoder of the quantization kernel (identical bytes).
+                const int sub = lane & 15;
+                for (int n0 = 2 * sw; n0 < NT; n0 += 2 * Lay::kSoftmaxWarps) {
+                    const int n = n0 + (lane >> 4);
+                    const bool valid = n < R;
+                    uint4 raw = make_uint4(0, 0, 0, 0);
+                    if (valid) {
+                        const int h = h_kv * p.G + n / nq, t = n % nq;
+                        raw = *reinterpret_cast<const uint4 *>(p.q_bf16 + b * p.q_sb + t * p.q_st + h * p.q_sh +
+                                                               sub * 8);
+                    }
+                    int X;
+                    const uint32_t packed = mxfp4_encode8(raw, valid, X);
+                    const int j = sub >> 2;  // 16-byte chunk (block of 32 channels) of the 64-byte row
+                    *reinterpret_cast<uint32_t *>(smem + Lay::kQ + n * 64 + ((j ^ ((n >> 1) & 3)) << 4) +
+                                                  (sub & 3) * 4) = packed;
+                    if ((sub & 3) == 0)
+                        smem[Lay::kSfQ + (n & 31) * 16 + (n >> 5) * 4 + j] = valid ? static_cast<uint8_t>(X + 127) : 0;
+                }
+                for (int n = NT + stid; n < 128; n += kSoftmaxThreads)
+                    *reinterpret_cast<uint32_t *>(smem + Lay::kSfQ + (n & 31) * 16 + (n >> 5) * 4) = 0;
+            } else {
+                for (int c = stid; c < NT * 4; c += kSoftmaxThreads) {
+                    const int n = c >> 2, j = c & 3;
+                    uint4 val = make_uint4(0, 0, 0, 0);
+                    if (n < R) {
+                        const int h = h_kv * p.G + n / nq, t = n % nq;
+                        val = *reinterpret_cast<const uint4 *>(
+                            p.q_codes + ((static_cast<int64_t>(b) * p.Hq + h) * p.q_cap + t) * 64 + j * 16);
+                    }
+                    *reinterpret_cast<uint4 *>(smem + Lay::kQ + n * 64 + ((j ^ ((n >> 1) & 3)) << 4)) = val;
+                }
+                for (int n = stid; n < 128; n += kSoftmaxThreads) {
+                    uint32_t scw = 0;
+                    if (n < R) {
+                        const int h = h_kv * p.G + n / nq, t = n % nq;
+                        scw = *reinterpret_cast<const uint32_t *>(
+                            p.q_scales + ((static_cast<int64_t>(b) * p.Hq + h) * (p.q_cap / 128) + t / 128) * 512 +
+                            (t & 31) * 16 + ((t & 127) >> 5) * 4);
+                    }
+                    *reinterpret_cast<uint32_t *>(smem + Lay::kSfQ + (n & 31) * 16 + (n >> 5) * 4) = scw;
+                }
+            }
+            // P scale atoms start at 2^0 for P_hi rows [0, NT) and 2^-5 for P_lo rows
+            // [NT, 2NT); the P^T buffers start at zero, and rows of absent queries
+            // are never written again.
+            for (int n = stid; n < 128; n += kSoftmaxThreads) {
+                const uint32_t pw = n < NT ? kPhiScaleWord : kPloScaleWord;
+                *reinterpret_cast<uint32_t *>(smem + Lay::kSfP + (n & 31) * 16 + (n >> 5) * 4) = pw;
+                *reinterpret_cast<uint32_t *>(smem + Lay::kSfP + 512 + (n & 31) * 16 + (n >> 5) * 4) = pw;
+            }
+            for (int c = stid; c < 2 * Lay::kPBytes / 16; c += kSoftmaxThreads)
+                reinterpret_cast<uint4 *>(smem + Lay::kP)[c] = make_uint4(0, 0, 0, 0);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && !p.test_stall) mbar_arrive(q_full);
+        }
         // Exchange slots of this column group, [quarter][NC].
         float *xmax = reinterpret_cast<float *>(smem + Lay::kXmax) + cg * 4 * NC;
         int *xe = reinterpret_cast<int *>(smem + Lay::kXe) + cg * 4 * NC;
@@ -655,12 +712,21 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) l += ldexpf(lsum[q * NC + i], esum[q * NC + i]);
                     const bool any = l > 0.f;
-                    const int64_t row = partial_row(c0 + i);
                     // O and l are both relative to m_O = m - e.
-                    p.ws_o[row * 128 + jt] = any ? (__uint_as_float(ohi[e]) + __uint_as_float(olo[e])) / l : 0.f;
-                    if (jt == 0)
-                        p.ws_lse[row] = any ? log2f(l) - m_neg[i] - static_cast<float>(esum[quarter * NC + i])
-                                            : -INFINITY;
+                    const float o = any ? (__uint_as_float(ohi[e]) + __uint_as_float(olo[e])) / l : 0.f;
+                    const float lse2 =
+                        any ? log2f(l) - m_neg[i] - static_cast<float>(esum[quarter * NC + i]) : -INFINITY;
+                    if (p.direct_out) {
+                        const int n = c0 + i, h = h_kv * p.G + n / nq, t = n % nq;
+                        p.out[((static_cast<int64_t>(b) * nq + t) * p.Hq + h) * 128 + jt] = __float2bfloat16_rn(o);
+                        if (jt == 0 && p.lse)
+                            p.lse[(static_cast<int64_t>(b) * p.Hq + h) * nq + t] =
+                                any ? lse2 * 0.6931471805599453f : -INFINITY;
+                    } else {
+                        const int64_t row = partial_row(c0 + i);
+                        p.ws_o[row * 128 + jt] = o;
+                        if (jt == 0) p.ws_lse[row] = lse2;
+                    }
                 }
             }
         }

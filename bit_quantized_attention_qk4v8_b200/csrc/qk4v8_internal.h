@@ -15,6 +15,11 @@ constexpr uint64_t kWaitTimeoutNs = 1000000000ull;
 
 struct AttnParams {
     const uint8_t *q_codes;   // [B][Hq][q_cap][64]
+    // Swap-AB decode only: when q_bf16 is set, the kernel quantizes the query
+    // rows itself from bf16 [b][t][h][128] (element strides q_sb, q_st, q_sh)
+    // and q_codes / q_scales are unused.
+    const __nv_bfloat16 *q_bf16;
+    int64_t q_sb, q_st, q_sh;
     const uint8_t *q_scales;  // [B][Hq][q_cap/128][512]
     const uint8_t *k_scales;  // [B][Hkv][kv_cap/128][512]
     const uint8_t *v_scales;  // [B][Hkv][kv_cap/128][512]
@@ -32,6 +37,7 @@ struct AttnParams {
     float *lse;               // prefill [B][Hq][Sq] (natural log), nullable
     float *ws_o;              // decode partial outputs [B][Hq][nq][splits][128]
     float *ws_lse;            // decode partial log2-sum-exp [B][Hq][nq][splits]
+    int direct_out;           // swap-AB decode with one split: write out [B][nq][Hq][128] and lse directly
     int32_t *status;          // nullable
     int test_stall;           // test hook: the producer withholds the Q-ready signal
     float *test_dump_s;       // test hook: CTA 0 writes its first raw score tile [128 lanes][128 keys]

@@ -12,25 +12,11 @@
 
 #include <cstdint>
 
+#include "mx_encode.cuh"
 #include "ptx.cuh"
 #include "qk4v8_internal.h"
 
 namespace qk4v8 {
-
-// Shared exponent from the float bits of a non-negative amax.
-// floor(log2 amax) is the unbiased exponent field; bf16 inputs that are
-// subnormal (or zero) land at the -127 clamp for both element formats.
-__device__ __forceinline__ int shared_exponent(float amax, int emax) {
-    int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF);
-    int X = e - 127 - emax;
-    X = X < -127 ? -127 : X;
-    X = X > 127 ? 127 : X;
-    return X;
-}
-
-__device__ __forceinline__ float pow2_neg(int X) {  // 2^-X for X in [-127, 126]
-    return __uint_as_float(static_cast<uint32_t>(127 - X) << 23);
-}
 
 // ------------------------------------------------------------------ MXFP4
 
@@ -62,26 +48,8 @@ __global__ void __launch_bounds__(256) quantize_qk_kernel(const __nv_bfloat16 *_
         const bool valid = in_range && t < valid_len;
         uint4 raw = make_uint4(0, 0, 0, 0);
         if (valid) raw = *reinterpret_cast<const uint4 *>(x + b * sb + t * ss + h * sh + sub * 8);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-        float v[8];
-        float amax = 0.f;
-        uint32_t sign = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[2 * i] = __uint_as_float(w[i] << 16);
-            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-            sign |= ((w[i] >> 15) & 1u) << (8 * i + 3);
-            sign |= ((w[i] >> 31) & 1u) << (8 * i + 7);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        const int X = shared_exponent(amax, 2);
-        const float f = pow2_neg(X);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = fabsf(v[i]) * f;  // exact: power-of-two scaling
-        uint32_t packed = valid ? (cvt_e2m1x8(v) | sign) : 0u;
+        int X;
+        const uint32_t packed = mxfp4_encode8(raw, valid, X);
         if (!in_range) continue;
         const int64_t head = static_cast<int64_t>(b) * H + h;
         reinterpret_cast<uint32_t *>(codes + (head * cap + t) * 64)[sub] = packed;

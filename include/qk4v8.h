@@ -194,7 +194,9 @@ QK4V8_API int qk4v8_decode_merge(const void *workspace, size_t workspace_bytes, 
  *   max_seqlen host upper bound on seqlens_k, used to plan the splits
  *   causal_in_block  query t of nq attends keys j <= L - nq + t
  *   num_splits  0 = qk4v8_decode_default_splits
- *   workspace  device scratch of qk4v8_decode_workspace_bytes(B, Hq, nq, splits)
+ *   workspace  device scratch of qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
+ *            unused (and may be null) when the call runs one split with
+ *            (Hq / Hkv) * nq <= 64, as the split kernel then writes out itself
  *   out      bf16 [B][nq][Hq][128]; lse float [B][Hq][nq] (nullable)
  * Requires (Hq / Hkv) * nq <= 128.
  */
@@ -204,6 +206,33 @@ QK4V8_API int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_sc
                            const int32_t *seqlens_k, int max_seqlen, int causal_in_block,
                            float softmax_scale, int num_splits, void *workspace, size_t workspace_bytes,
                            void *out, float *lse, int32_t *dev_status, void *stream);
+
+/*
+ * Decode step from bf16 queries (MpFA QK4V8 article, section 3.2: the query's
+ * MXFP4 scales are computed as it is loaded, inside the attention call).
+ * Same result, bit for bit, as qk4v8_quantize_qk (capacity 128) followed by
+ * qk4v8_attention_decode, in one call and usually one launch:
+ *   - (Hq / Hkv) * nq <= 64: the split kernel reads the bf16 query rows and
+ *     encodes them to MXFP4 itself; with one split it also writes out and lse
+ *     directly, so there is no merge launch and no workspace.
+ *   - larger groups: the queries are quantized into the front of the
+ *     workspace, then the 128-row split kernel and the merge run.
+ *   q        bf16 [B][nq][Hq][128] (device), element strides q_stride_b,
+ *            q_stride_t, q_stride_h, each a multiple of 8; channel stride 1;
+ *            16-byte aligned
+ *   workspace  device scratch of qk4v8_decode_bf16_workspace_bytes(B, Hq, Hkv,
+ *            nq, splits) bytes (0: may be null), 16-byte aligned
+ *   other arguments, out, lse and errors as for qk4v8_attention_decode.
+ */
+QK4V8_API size_t qk4v8_decode_bf16_workspace_bytes(int B, int Hq, int Hkv, int nq, int num_splits);
+
+QK4V8_API int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_stride_b,
+                                          int64_t q_stride_t, int64_t q_stride_h, const uint8_t *k_codes,
+                                          const uint8_t *k_scales, const uint8_t *v_codes, const uint8_t *v_scales,
+                                          int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
+                                          int causal_in_block, float softmax_scale, int num_splits, void *workspace,
+                                          size_t workspace_bytes, void *out, float *lse, int32_t *dev_status,
+                                          void *stream);
 
 /*
  * Decode for callers that cannot allocate device memory: qk4v8_attention_decode

@@ -115,6 +115,31 @@ def test_decode_rejects_bad_args(lib):
     assert b"workspace" in lib.qk4v8_last_error() or True
 
 
+def test_bf16_decode_workspace_bytes(lib):
+    f = lib.qk4v8_decode_bf16_workspace_bytes
+    part = lib.qk4v8_decode_workspace_bytes
+    assert f(32, 32, 8, 1, 1) == 0                      # 4 rows, one split: written directly, no scratch
+    assert f(32, 32, 8, 1, 3) == part(32, 32, 1, 3)      # partials for the merge
+    assert f(2, 64, 8, 8, 1) == 0                        # 64 rows still on the split kernel
+    packed_q = 2 * 128 * 128 * 64 + 2 * 128 * 512         # 128 rows: MXFP4 Q, capacity 128, in front
+    assert f(2, 128, 8, 8, 2) == packed_q + part(2, 128, 8, 2)
+    assert f(0, 8, 8, 1, 1) == 0 and f(1, 30, 8, 1, 1) == 0
+
+
+def test_bf16_decode_rejects_bad_args(lib):
+    def call(q=FAKE, nq=1, Hq=32, Hkv=8, sb=32 * 128, st=32 * 128, sh=128, splits=1, ws=None, wsb=0, out=FAKE):
+        return lib.qk4v8_attention_decode_bf16(q, 2, Hq, nq, sb, st, sh, FAKE, FAKE, FAKE, FAKE, Hkv, 8192, FAKE,
+                                               8192, 1, 0.0, splits, ws, wsb, out, None, None, None)
+
+    assert call(q=None) == 1
+    assert call(nq=9) == 1
+    assert call(Hq=64, Hkv=1, nq=4) == 1      # 256 rows
+    assert call(out=FAKE + 2) == 1
+    assert call(splits=3) == 1                # partials need a workspace
+    assert call(q=FAKE + 2) == 1              # bf16 rows must be 16-byte aligned
+    assert call(sh=100) == 1                  # strides in whole 16-byte units
+
+
 def test_prefill_rejects_bad_args(lib):
     def call(Sq=256, q_cap=256, Sk=256, kv_cap=256, Hq=4, Hkv=2, out=FAKE):
         return lib.qk4v8_attention_prefill(FAKE, FAKE, 1, Hq, Sq, q_cap, FAKE, FAKE, FAKE, FAKE, Hkv, Sk, kv_cap,
