@@ -167,12 +167,16 @@ def to_dev(bits):
 
 def decode_kernel_name(rows: int) -> str:
     """The split-KV kernel the library launches for `rows` = (Hq / Hkv) * nq query rows per KV head."""
+    if rows <= 4:
+        return "qk4v8_decode_kernel<16,4,4,3,2> (swap-AB split-KV decode)"
+    if rows <= 8:
+        return "qk4v8_decode_kernel<16,8,8,3,2> (swap-AB split-KV decode)"
     if rows <= 16:
-        return "qk4v8_decode_kernel<16,16,3,2> (swap-AB split-KV decode)"
+        return "qk4v8_decode_kernel<16,16,16,3,2> (swap-AB split-KV decode)"
     if rows <= 32:
-        return "qk4v8_decode_kernel<32,16,6,1> (swap-AB split-KV decode)"
+        return "qk4v8_decode_kernel<32,32,16,6,1> (swap-AB split-KV decode)"
     if rows <= 64:
-        return "qk4v8_decode_kernel<64,32,6,1> (swap-AB split-KV decode)"
+        return "qk4v8_decode_kernel<64,64,16,6,1> (swap-AB split-KV decode)"
     return "qk4v8_attention_kernel<true> (128-row split-KV decode)"
 
 

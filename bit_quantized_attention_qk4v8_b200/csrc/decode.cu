@@ -56,15 +56,19 @@ constexpr int kBarGroup0 = 1, kBarAllSoftmax = 5;
 // be sitting in).
 constexpr uint64_t kVoteTimeoutNs = 4 * kWaitTimeoutNs;
 
-template <int NT, int NC, int ST>
+// NT: query rows of the MMA (its N, at least 16); RW: rows the softmax warps
+// cover (RW <= NT, the launch's G*nq at most); NC: rows per softmax warp.
+template <int NT, int RW, int NC, int ST>
 struct DecodeLayout {
+    static_assert(RW <= NT && RW % NC == 0 && NC % 4 == 0, "row split");
+    static_assert(RW == NC || NC % 8 == 0, "column groups start at multiples of 8 rows (P^T swizzle)");
     static constexpr int kStages = ST;             // K/V pipeline stages
-    static constexpr int kCG = NT / NC;            // column groups
+    static constexpr int kCG = RW / NC;            // column groups
     static constexpr int kSoftmaxWarps = 4 * kCG;
     static constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
     static constexpr int kThreads = 64 + kSoftmaxThreads;
-    static constexpr int kQ = 0;  // NT rows x 64 B, 64-byte swizzle (8 KB reserved)
-    static constexpr int kK = 8192;
+    static constexpr int kQ = 0;  // NT rows x 64 B, 64-byte swizzle
+    static constexpr int kK = NT * 64 < 1024 ? 1024 : NT * 64;
     static constexpr int kKBytes = 128 * 64;
     static constexpr int kV = kK + ST * kKBytes;
     static constexpr int kVBytes = 128 * 128;
@@ -83,9 +87,9 @@ struct DecodeLayout {
     static constexpr int kVote = kLim + 256;    // [column group][tile parity][quarter] u32 vote words
     static constexpr int kMneg = kVote + 128;   // [softmax warp][NC] float: -m of each row
     static constexpr int kBar = kMneg + 1024;
-    // kv_full/empty per stage, q_full, patch, s_full/free x2, p_full x2,
-    // pv_done x2, o_final, vote x2 and e exchange per column group.
-    static constexpr int kNumBars = 2 * ST + 11 + 3 * kCG;
+    // kv_full/empty per stage, q_full, patch, s_full x2, p_full x2, pv_done x2,
+    // o_final, vote x2 and e exchange per column group.
+    static constexpr int kNumBars = 2 * ST + 9 + 3 * kCG;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16 + 1024;
     // TMEM columns: S^T x2 [0, 2NT), O^T [2NT, 4NT), then scale factors:
@@ -167,13 +171,34 @@ __device__ __forceinline__ float exp2_neg_int(int k) {
     return k < 126 ? __uint_as_float(static_cast<uint32_t>(127 - k) << 23) : 0.f;
 }
 
+// O *= 2^-E_c for the nc columns at taddr (P_hi part) and taddr + nt (P_lo
+// part), E_c held by lane c of the warp. Kept out of line: it runs only when a
+// row's reference moves past kEMaxD.
+__device__ __noinline__ void rescale_o_cols(uint32_t taddr, int nt, int nc, int E) {
+    for (int c8 = 0; c8 < nc; c8 += 8) {
+        uint32_t ohi[8], olo[8];
+        tmem_load_cols<8>(taddr + c8, ohi);
+        tmem_load_cols<8>(taddr + nt + c8, olo);
+        tc_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float a = exp2_neg_int(__shfl_sync(0xffffffffu, E, c8 + c));
+            ohi[c] = __float_as_uint(__uint_as_float(ohi[c]) * a);
+            olo[c] = __float_as_uint(__uint_as_float(olo[c]) * a);
+        }
+        tmem_store_cols<8>(taddr + c8, ohi);
+        tmem_store_cols<8>(taddr + nt + c8, olo);
+    }
+    tc_wait_st();
+}
+
 }  // namespace
 
-template <int NT, int NC, int ST, int MINB>
-__global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
+template <int NT, int RW, int NC, int ST, int MINB>
+__global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
     qk4v8_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                         const AttnParams p) {
-    using Lay = DecodeLayout<NT, NC, ST>;
+    using Lay = DecodeLayout<NT, RW, NC, ST>;
     constexpr int kStagesD = Lay::kStages;
     constexpr int kSoftmaxThreads = Lay::kSoftmaxThreads;
     extern __shared__ uint8_t smem_raw[];
@@ -224,12 +249,14 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
     uint64_t *kv_empty = bars + kStagesD;
     uint64_t *q_full = bars + 2 * kStagesD;
     uint64_t *patch = q_full + 1;
+    // S buffer (it & 1) needs no release barrier: the MMA warp issues S(it+2)
+    // only after waiting for p_full of tile it, and every softmax warp arrives
+    // there after its reads of S(it) have completed.
     uint64_t *s_full = q_full + 2;   // [2]
-    uint64_t *s_free = q_full + 4;   // [2]
-    uint64_t *p_full = q_full + 6;   // [2]
-    uint64_t *pv_done = q_full + 8;  // [2]
-    uint64_t *o_final = q_full + 10;
-    uint64_t *vote_bar = q_full + 11;            // [column group][tile parity]: one arrival per warp
+    uint64_t *p_full = q_full + 4;   // [2]
+    uint64_t *pv_done = q_full + 6;  // [2]
+    uint64_t *o_final = q_full + 8;
+    uint64_t *vote_bar = q_full + 9;             // [column group][tile parity]: one arrival per warp
     uint64_t *xe_bar = vote_bar + 2 * Lay::kCG;  // [column group]: offsets posted for an O rescale
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::kMisc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + Lay::kMisc + 4);
@@ -243,7 +270,6 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
         mbar_init(patch, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
-            mbar_init(&s_free[s], Lay::kSoftmaxWarps);
             mbar_init(&p_full[s], Lay::kSoftmaxWarps);
             mbar_init(&pv_done[s], 1);
         }
@@ -369,7 +395,6 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
                 const int sbuf = it & 1;
                 ok = wait_bar(&kv_full[st], (it / kStagesD) & 1, abort_flag, p.status);
                 if (ok && last_partial && it == T - 1) ok = wait_bar(patch, 0, abort_flag, p.status);
-                if (ok) ok = wait_bar(&s_free[sbuf], ((it >> 1) & 1) ^ 1, abort_flag, p.status);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
                 const uint32_t tSfK = tmem + col_sf_k_d(NT, sbuf);
@@ -504,10 +529,6 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
                 tmem_load_cols<NC>(tmem + lane_base + static_cast<uint32_t>(NT * sbuf + c0), sraw);
                 tc_wait_ld();
             }
-            // S buffer `sbuf` is next written by S(it+2), issued after this tile's P.
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[sbuf]);
 
             // u = s * scale - m (log2 units); -inf where the key is masked. Every row
             // may see this key unless it lies past L, or in the last nq-1 positions
@@ -646,22 +667,7 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
                     bool okw = wait_bar(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag, p.status);
                     if (__all_sync(0xffffffffu, okw)) {
                         tc_fence_after();
-#pragma unroll 1
-                        for (int c8 = 0; c8 < NC; c8 += 8) {
-                            uint32_t ohi[8], olo[8];
-                            tmem_load_cols<8>(tmem + lane_base + Lay::kColO + c0 + c8, ohi);
-                            tmem_load_cols<8>(tmem + lane_base + Lay::kColO + NT + c0 + c8, olo);
-                            tc_wait_ld();
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const float a = exp2_neg_int(__shfl_sync(0xffffffffu, E, c8 + c));
-                                ohi[c] = __float_as_uint(__uint_as_float(ohi[c]) * a);
-                                olo[c] = __float_as_uint(__uint_as_float(olo[c]) * a);
-                            }
-                            tmem_store_cols<8>(tmem + lane_base + Lay::kColO + c0 + c8, ohi);
-                            tmem_store_cols<8>(tmem + lane_base + Lay::kColO + NT + c0 + c8, olo);
-                        }
-                        tc_wait_st();
+                        rescale_o_cols(tmem + lane_base + Lay::kColO + c0, NT, NC, E);
                     }
                 }
             }
@@ -739,31 +745,33 @@ __global__ void __launch_bounds__(DecodeLayout<NT, NC, ST>::kThreads, MINB)
     }
 }
 
-template <int NT, int NC, int ST, int MINB>
+template <int NT, int RW, int NC, int ST, int MINB>
 static cudaError_t launch_nt(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, int grid,
                              cudaStream_t stream) {
-    using Lay = DecodeLayout<NT, NC, ST>;
+    using Lay = DecodeLayout<NT, RW, NC, ST>;
     constexpr int kMaxDevices = 64;
     static bool configured[kMaxDevices] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= kMaxDevices || !configured[dev]) {
-        e = cudaFuncSetAttribute(qk4v8_decode_kernel<NT, NC, ST, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(qk4v8_decode_kernel<NT, RW, NC, ST, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Lay::kBytes);
         if (e != cudaSuccess) return e;
         if (dev < kMaxDevices) configured[dev] = true;
     }
-    qk4v8_decode_kernel<NT, NC, ST, MINB><<<grid, Lay::kThreads, Lay::kBytes, stream>>>(tk, tv, p);
+    qk4v8_decode_kernel<NT, RW, NC, ST, MINB><<<grid, Lay::kThreads, Lay::kBytes, stream>>>(tk, tv, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, int grid,
                           cudaStream_t stream) {
     const int R = p.G * p.Sq;
-    if (R <= 16) return launch_nt<16, 16, kDecodeSmallStages, 2>(tk, tv, p, grid, stream);
-    if (R <= 32) return launch_nt<32, 16, 6, 1>(tk, tv, p, grid, stream);
-    return launch_nt<64, 32, 6, 1>(tk, tv, p, grid, stream);
+    if (R <= 4) return launch_nt<16, 4, 4, kDecodeSmallStages, 2>(tk, tv, p, grid, stream);
+    if (R <= 8) return launch_nt<16, 8, 8, kDecodeSmallStages, 2>(tk, tv, p, grid, stream);
+    if (R <= 16) return launch_nt<16, 16, 16, kDecodeSmallStages, 2>(tk, tv, p, grid, stream);
+    if (R <= 32) return launch_nt<32, 32, 16, 6, 1>(tk, tv, p, grid, stream);
+    return launch_nt<64, 64, 16, 6, 1>(tk, tv, p, grid, stream);
 }
 
 }  // namespace qk4v8
