@@ -543,18 +543,21 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
                 mrow[i + 2] = m4.z;
                 mrow[i + 3] = m4.w;
             }
+            // Rows past R (absent queries, zero Q) run through the same code with
+            // s = 0; their results are never written.
             float u[NC];
-            if (it > 0 && ok && tok < L - (p.causal ? nq - 1 : 0)) {
 #pragma unroll
-                for (int i = 0; i < NC; ++i)
-                    u[i] = i < nv ? fmaf(__uint_as_float(sraw[i]), sc, mrow[i]) : -INFINITY;
-            } else {
+            for (int i = 0; i < NC; i += 2) {
+                const float2 v = ffma2(make_float2(__uint_as_float(sraw[i]), __uint_as_float(sraw[i + 1])),
+                                       make_float2(sc, sc), make_float2(mrow[i], mrow[i + 1]));
+                u[i] = v.x;
+                u[i + 1] = v.y;
+            }
+            if (!(it > 0 && ok && tok < L - (p.causal ? nq - 1 : 0))) {
                 const bool any_key = ok && tok < L;
 #pragma unroll
-                for (int i = 0; i < NC; ++i) {
-                    const bool valid = any_key && i < nv && tok < lim_s[c0 + i];
-                    u[i] = valid ? fmaf(__uint_as_float(sraw[i]), sc, mrow[i]) : -INFINITY;
-                }
+                for (int i = 0; i < NC; ++i)
+                    if (!(any_key && tok < lim_s[c0 + i])) u[i] = -INFINITY;
             }
             if (it == 0) {
                 // The group's first tile fixes m_O = m of each row: the row's largest
@@ -586,7 +589,6 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
                 if (__any_sync(0xffffffffu, umax > kTauD)) {
 #pragma unroll
                     for (int i = 0; i < NC; ++i) {
-                        if (i >= nv) break;
                         const float mx = warp_max_f32(u[i]);
                         if (mx > kTauD) {
                             const float de = ceilf(fminf(mx, kMaxMoveD));
@@ -614,32 +616,31 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
                 bool okw = wait_bar(&pv_done[sbuf], ((it >> 1) & 1) ^ 1, abort_flag, p.status);
                 (void)__all_sync(0xffffffffu, okw);
             }
-            // Encode P^T bytes. P_hi = E4M3(p). Its value comes back exactly from the
-            // code's 7 magnitude bits placed at bit 20 of a float, times 2^120: f32
-            // and E4M3 treat their lowest exponent alike, so subnormal codes decode
-            // the same way. P_lo = E4M3(32 (p - P_hi)) carries the next bits.
+            // Encode P^T bytes from p as f16 pairs (rounding error 2^-11 of p, far
+            // below what P_lo resolves): P_hi = E4M3(p); its value comes back
+            // exactly as f16; P_lo = E4M3(32 (p - P_hi)), where the difference is
+            // exact since P_hi is within 2^-4 of p. The row sums take p itself.
             uint8_t *pb = smem + Lay::kP + sbuf * Lay::kPBytes;
+            const __half2 k32 = __float2half2_rn(32.f), km32 = __float2half2_rn(-32.f);
 #pragma unroll
             for (int i = 0; i < NC; i += 2) {
-                if (i >= nv) break;
                 const float p0 = exp2_approx(u[i]);
                 const float p1 = exp2_approx(u[i + 1]);
-                lacc[i] += p0;
-                lacc[i + 1] += p1;
-                const uint32_t h2 = cvt_e4m3x2(p0, p1);
-                const float hv0 = __uint_as_float((h2 << 20) & 0x0FF00000u);
-                const float hv1 = __uint_as_float((h2 << 12) & 0x0FF00000u);
-                const float d0 = fmaf(hv0, -0x1p125f, p0 * 32.f);
-                const float d1 = fmaf(hv1, -0x1p125f, p1 * 32.f);
-                const uint32_t l2 = cvt_e4m3x2(d0, d1);
+                const float2 la = fadd2(make_float2(lacc[i], lacc[i + 1]), make_float2(p0, p1));
+                lacc[i] = la.x;
+                lacc[i + 1] = la.y;
+                const __half2 ph = __floats2half2_rn(p0, p1);
+                const uint32_t phw = *reinterpret_cast<const uint32_t *>(&ph);
+                const uint16_t h2 = cvt_e4m3x2_from_f16x2(phw);
+                const uint32_t hvw = cvt_e4m3x2_to_f16x2(h2);
+                const __half2 d = __hfma2(*reinterpret_cast<const __half2 *>(&hvw), km32, __hmul2(ph, k32));
+                const uint16_t l2 = cvt_e4m3x2_from_f16x2(*reinterpret_cast<const uint32_t *>(&d));
                 const int o0 = (pofs ^ ((i & 7) << 4)) + i * 128;
                 const int o1 = (pofs ^ (((i + 1) & 7) << 4)) + (i + 1) * 128;
                 st_u8(pb, o0, h2);
                 st_u8(pb, o0 + NT * 128, l2);
-                if (i + 1 < nv) {
-                    st_u8(pb, o1, h2 >> 8);
-                    st_u8(pb, o1 + NT * 128, l2 >> 8);
-                }
+                st_u8(pb, o1, h2 >> 8);
+                st_u8(pb, o1 + NT * 128, l2 >> 8);
             }
             // Collect the vote. Every warp of the group reads the same four words.
             const bool okv = wait_bar_peers(&vote_bar[2 * cg + sbuf], (it >> 1) & 1);

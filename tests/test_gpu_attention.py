@@ -144,6 +144,10 @@ def test_prefill_softmax_scale_and_peaked_scores():
     (2, 4, 300, 4, 1, 7, [300, 7]),
     (1, 8, 600, 16, 1, 2, None),       # G*nq = 128 rows: the 128-row kernel's decode path
     (2, 3, 900, 12, 4, 3, [900, 400]), # odd row count (G*nq = 9)
+    (2, 2, 1500, 16, 4, 2, None),      # G*nq = 8: the 8-row instance
+    (2, 1, 3000, 64, 8, 1, [3000, 2999]),  # GQA 8, one token: 8 rows, one split (direct output)
+    (2, 5, 700, 5, 5, 2, [700, 64]),   # G*nq = 5
+    (2, 4, 800, 32, 4, 2, [800, 511]),  # G*nq = 32: the 32-row instance
 ])
 def test_decode_parity(B, nq, L, Hq, Hkv, splits, lens):
     gen = make_gen(B, nq, L, Hq, Hkv, seed=L + nq, lens=lens, k_out=4)
