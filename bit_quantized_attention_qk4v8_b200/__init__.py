@@ -253,3 +253,39 @@ def decode_merge(workspace: torch.Tensor, B: int, Hq: int, nq: int, num_splits: 
 
 def default_scale() -> float:
     return 1.0 / math.sqrt(D)
+
+
+# ----------------------------------------------------------------------------------------------------------
+# Measurement hooks (include/qk4v8_test.h): not part of the attention API.
+
+def prefill_stage_qk(q: MXFP4, k: MXFP4, seqlens_k=None, causal: bool = True,
+                     softmax_scale: Optional[float] = None, row_max: Optional[torch.Tensor] = None,
+                     dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The QK^T stage of the prefill kernel alone (same tile schedule, no exp / P / PV).
+
+    Returns row_max float32 [B, Hq, Sq]: each query row's largest allowed score
+    times softmax_scale * log2(e) (-inf for a row with no allowed key).
+    """
+    dev = q.codes.device
+    B, Hq, Sq = q.B, q.H, q.length
+    sl = _seqlens(seqlens_k, B, dev)
+    if row_max is None:
+        row_max = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+    check(lib().qk4v8_test_prefill_stage_qk(q.codes.data_ptr(), q.scales.data_ptr(), B, Hq, Sq, q.cap,
+                                            k.codes.data_ptr(), k.scales.data_ptr(), k.H, k.length, k.cap, _ptr(sl),
+                                            int(bool(causal)), float(softmax_scale or 0.0), row_max.data_ptr(),
+                                            _ptr(dev_status), _stream(dev)), "qk4v8_test_prefill_stage_qk")
+    return row_max
+
+
+MMA_PEAK_SHAPES = {0: ("mxf4", 128, 128, 64), 1: ("mxf8f6f4", 128, 144, 32),
+                   2: ("mxf8f6f4", 128, 256, 32), 3: ("mxf4", 128, 256, 64)}
+
+
+def mma_peak_run(kind: int, ctas: int, iters: int, device=None, dev_status: Optional[torch.Tensor] = None) -> int:
+    """Enqueue one tensor-pipe peak run; returns its FLOP count (2*M*N*K per instruction)."""
+    dev = torch.device(device or "cuda")
+    check(lib().qk4v8_test_mma_peak(int(kind), int(ctas), int(iters), _ptr(dev_status), _stream(dev)),
+          "qk4v8_test_mma_peak")
+    _, m, n, kk = MMA_PEAK_SHAPES[int(kind)]
+    return 2 * m * n * kk * int(ctas) * int(iters)

@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqk4v8.so")
-SOURCES = ["quantize.cu", "attention.cu", "decode.cu", "api.cu"]
+SOURCES = ["quantize.cu", "attention.cu", "prefill.cu", "decode.cu", "mma_peak.cu", "api.cu"]
 HEADERS = ["ptx.cuh", "pipeline.cuh", "mx_encode.cuh", "qk4v8_internal.h"]
 
 NVCC_FLAGS = [

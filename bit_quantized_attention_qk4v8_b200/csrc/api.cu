@@ -186,23 +186,31 @@ int qk4v8_quantize(const void *q, const void *k, const void *v, int B, int Sq, i
     return qk4v8_quantize_v(v, B, Sk, Hkv, d, ks * Sk, ks, 128, seqlens_k, kv_cap, v_codes, v_scales, stream);
 }
 
-int qk4v8_attention_prefill(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int Sq, int q_cap,
-                            const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
-                            const uint8_t *v_scales, int Hkv, int Sk, int kv_cap, const int32_t *seqlens_k,
-                            int causal, float softmax_scale, void *out, float *lse, int32_t *dev_status,
-                            void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by the prefill entry point and its QK^T-stage test build.
+int prefill_common(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int Sq, int q_cap,
+                   const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes, const uint8_t *v_scales,
+                   int Hkv, int Sk, int kv_cap, const int32_t *seqlens_k, int causal, float softmax_scale, void *out,
+                   float *lse, int32_t *dev_status, void *stream, bool stage_qk) {
     int st;
-    if ((st = validate_packed(q_codes, q_scales, "Q")) || (st = validate_packed(k_codes, k_scales, "K")) ||
-        (st = validate_packed(v_codes, v_scales, "V")))
+    if ((st = validate_packed(q_codes, q_scales, "Q")) || (st = validate_packed(k_codes, k_scales, "K")))
         return st;
-    if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
+    if (!stage_qk && (st = validate_packed(v_codes, v_scales, "V"))) return st;
+    if (!stage_qk && (!out || !aligned16(out)))
+        return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv)
         return set_error(QK4V8_ERR_INVALID_ARG, "bad heads B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
     if (Sq <= 0 || q_cap % 128 || q_cap < Sq || kv_cap <= 0 || kv_cap % 128 || Sk < 0 || Sk > kv_cap)
         return set_error(QK4V8_ERR_INVALID_ARG, "bad lengths Sq=%d q_cap=%d Sk=%d kv_cap=%d", Sq, q_cap, Sk, kv_cap);
     if ((st = check_device())) return st;
     CUtensorMap tk, tv;
-    if ((st = make_k_map(&tk, k_codes, B * Hkv, kv_cap)) || (st = make_v_map(&tv, v_codes, B * Hkv, kv_cap)))
+    if ((st = make_k_map(&tk, k_codes, B * Hkv, kv_cap))) return st;
+    if (stage_qk)
+        tv = tk;  // unused by the QK^T stage
+    else if ((st = make_v_map(&tv, v_codes, B * Hkv, kv_cap)))
         return st;
     qk4v8::AttnParams p{};
     p.q_codes = q_codes;
@@ -230,8 +238,31 @@ int qk4v8_attention_prefill(const uint8_t *q_codes, const uint8_t *q_scales, int
     p.test_stall = g_test_stall;
     p.test_dump_s = g_test_dump_s;
     const int grid = B * Hq * p.n_qtiles;
-    cudaError_t e = qk4v8::launch_attention(tk, tv, p, grid, static_cast<cudaStream_t>(stream));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = stage_qk ? qk4v8::launch_prefill_stage_qk(tk, tv, p, grid, s)
+                             : qk4v8::launch_prefill(tk, tv, p, grid, s);
     return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "attention (prefill) launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int qk4v8_attention_prefill(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int Sq, int q_cap,
+                            const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
+                            const uint8_t *v_scales, int Hkv, int Sk, int kv_cap, const int32_t *seqlens_k,
+                            int causal, float softmax_scale, void *out, float *lse, int32_t *dev_status,
+                            void *stream) {
+    return prefill_common(q_codes, q_scales, B, Hq, Sq, q_cap, k_codes, k_scales, v_codes, v_scales, Hkv, Sk, kv_cap,
+                          seqlens_k, causal, softmax_scale, out, lse, dev_status, stream, false);
+}
+
+int qk4v8_test_prefill_stage_qk(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int Sq, int q_cap,
+                                const uint8_t *k_codes, const uint8_t *k_scales, int Hkv, int Sk, int kv_cap,
+                                const int32_t *seqlens_k, int causal, float softmax_scale, float *row_max,
+                                int32_t *dev_status, void *stream) {
+    return prefill_common(q_codes, q_scales, B, Hq, Sq, q_cap, k_codes, k_scales, nullptr, nullptr, Hkv, Sk, kv_cap,
+                          seqlens_k, causal, softmax_scale, nullptr, row_max, dev_status, stream, true);
 }
 
 size_t qk4v8_decode_workspace_bytes(int B, int Hq, int nq, int num_splits) {
@@ -501,6 +532,15 @@ void qk4v8_test_set_stall(int enable) { g_test_stall = enable ? 1 : 0; }
 // Test hook (declared in include/qk4v8_test.h): while set, CTA 0 of each
 // attention launch writes its first raw score tile to `dev_ptr`.
 void qk4v8_test_set_dump_scores(float *dev_ptr) { g_test_dump_s = dev_ptr; }
+
+int qk4v8_test_mma_peak(int kind, int ctas, int iters, int32_t *dev_status, void *stream) {
+    if (kind < 0 || kind > 3 || ctas <= 0 || ctas > 65535 || iters <= 0 || iters > (1 << 24))
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad MMA peak run kind=%d ctas=%d iters=%d", kind, ctas, iters);
+    int st;
+    if ((st = check_device())) return st;
+    cudaError_t e = qk4v8::launch_mma_peak(kind, ctas, iters, dev_status, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "MMA peak launch");
+}
 
 }  // extern "C"
 

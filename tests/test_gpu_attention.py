@@ -225,3 +225,61 @@ def test_quantize_entry_point_matches_separate_calls():
     torch.cuda.synchronize()
     for a, b in ((qp, qp2), (kp, kp2), (vp, vp2)):
         assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales)
+
+
+def dequantized_scores(qp, kp, Sq, Lk):
+    """fp64 S = Q K^T (no softmax scale) of the dequantized packed tensors, [B, Hq, Sq, Lk] per KV group."""
+    qc = unpack_e2m1(qp.codes.cpu().numpy()[:, :, :Sq])
+    qs = qk_scales_logical(qp.scales.cpu().numpy(), Sq)
+    kc = unpack_e2m1(kp.codes.cpu().numpy()[:, :, :Lk])
+    ks = qk_scales_logical(kp.scales.cpu().numpy(), Lk)
+
+    def deq(c, s):
+        v = E2M1[c & 7] * np.where(c & 8, -1.0, 1.0)
+        return v * np.exp2(np.repeat(s.astype(np.float64) - 127, 32, axis=-1))
+
+    qd, kd = deq(qc, qs), deq(kc, ks)
+    G = qd.shape[1] // kd.shape[1]
+    kd = np.repeat(kd, G, axis=1)
+    return np.einsum("bhid,bhjd->bhij", qd, kd)
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv,causal,lens", [
+    (1, 384, 4, 2, True, None),
+    (2, 200, 2, 1, False, [200, 77]),
+    (2, 130, 2, 2, True, [130, 0]),
+])
+def test_prefill_stage_qk_row_max(B, S, Hq, Hkv, causal, lens):
+    """The QK^T-stage build: each row's largest allowed scaled score, exactly as the scores' max."""
+    gen = make_gen(B, S, S, Hq, Hkv, seed=S + 3, lens=lens, k_out=2, mult=20.0)
+    qp, kp, vp, sl = quantize_on_gpu(gen)
+    rm = qk.prefill_stage_qk(qp, kp, seqlens_k=sl, causal=causal)
+    torch.cuda.synchronize()
+    s = dequantized_scores(qp, kp, S, S)
+    c = (1.0 / math.sqrt(128)) * math.log2(math.e)
+    L = gen["seqlens"]
+    ref = np.full((B, Hq, S), -np.inf)
+    for b in range(B):
+        for i in range(S):
+            lim = L[b] if not causal else min(L[b], i + L[b] - S + 1)
+            if lim > 0:
+                ref[b, :, i] = s[b, :, i, :lim].max(axis=-1) * c
+    got = rm.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(got), fin)
+    # fp32 accumulation of exact FP4 products: relative error ~1e-6
+    assert np.abs(got[fin] - ref[fin]).max() <= 1e-5 * max(1.0, np.abs(ref[fin]).max())
+
+
+def test_prefill_o_rescale_path():
+    """Later keys score far (>64 binades) above the first tile's row max, so O is rescaled mid-row."""
+    gen = make_gen(1, 128, 512, 2, 1, seed=41)
+    k = (gen["k"].astype(np.uint32) << 16).view(np.float32).copy()
+    k[:, :128] *= np.float32(1e-3)      # the first key tile: near-zero scores
+    gen["k"] = f32_to_bf16_bits(k)
+    scale = 6.0                          # scores of the later tiles reach ~100 binades
+    out, lse, _ = run_prefill(gen, False, scale=scale)
+    (ref, rlse), _ = oracle_attention_from(gen, False, scale=scale)
+    assert_close(out, ref, "prefill O rescale")
+    l = lse.cpu().numpy().transpose(0, 2, 1)
+    assert np.abs(l - rlse).max() < 1e-2 + 1e-5 * np.abs(rlse).max()
