@@ -58,6 +58,8 @@ def parse_args():
     ap.add_argument("--splits", type=int, default=0, help="decode KV splits (0 = library default)")
     ap.add_argument("--prefill-steps", type=int, default=10)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="prefill only (a profiling aid): prints the prefill object alone")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -290,6 +292,7 @@ def run_prefill(args):
     stream = torch.cuda.current_stream()
     qp, kp, vp = qk.quantize(q, k, v)
     out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
+    row_max = torch.empty((wl.B, wl.Hq, wl.Sq), dtype=torch.float32, device="cuda")
     n = max(1, args.prefill_steps)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
 
@@ -306,18 +309,59 @@ def run_prefill(args):
         step()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(n):
-        step(i)
-    t1.record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0.record(stream)
+        for i in range(n):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / n
     attn_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+
+    # The QK^T stage alone: the same kernel built without exp, P and P.V, same tile schedule.
+    for _ in range(3):
+        qk.prefill_stage_qk(qp, kp, causal=True, row_max=row_max)
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(n):
+        qk.prefill_stage_qk(qp, kp, causal=True, row_max=row_max)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    stage_ms = s0.elapsed_time(s1) / n
+
     # FlashAttention-style FLOP count of causal attention: 4 * B * Hq * d * (S(S+1)/2)
     pairs = wl.Sq * (wl.Sq + 1) / 2
     flops = 4.0 * wl.B * wl.Hq * 128 * pairs
     qk_flops = flops / 2
-    return dict(wl=wl, ms=ms, attn_ms=attn_ms, flops=flops, qk_flops=qk_flops)
+    # Executed work: every 128 x 128 tile on or below the causal diagonal is computed in full.
+    nt = (wl.Sq + 127) // 128
+    tiles = wl.B * wl.Hq * nt * (nt + 1) // 2
+    return dict(wl=wl, ms=ms, attn_ms=attn_ms, stage_ms=stage_ms, flops=flops, qk_flops=qk_flops, tiles=tiles,
+                clocks=clk.summary())
+
+
+def run_mma_peaks(kinds=(0, 1), iters=200000):
+    """Tensor-pipe peak (TFLOP/s) of the attention's own MMA shapes, one CTA per SM, CUDA-event timed."""
+    import torch
+    import bit_quantized_attention_qk4v8_b200 as qk
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    stream = torch.cuda.current_stream()
+    res = {}
+    for kind in kinds:
+        qk.mma_peak_run(kind, sms, 1000)
+        torch.cuda.synchronize()
+        best = 0.0
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fl = qk.mma_peak_run(kind, sms, iters)
+            b.record(stream)
+            torch.cuda.synchronize()
+            best = max(best, fl / (a.elapsed_time(b) * 1e-3) / 1e12)
+        name, m, nn, kk = qk.MMA_PEAK_SHAPES[kind]
+        res[f"{name}_m{m}n{nn}k{kk}"] = best
+    return res
 
 
 # ------------------------------------------------------------------------ CPU oracle
@@ -407,6 +451,41 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------------------- main
 
+def prefill_object(args, peak_src, bf16_tf):
+    p = run_prefill(args)
+    peaks = run_mma_peaks()
+    fp4_peak = peaks["mxf4_m128n128k64"]      # the QK^T instruction's own measured peak
+    fp8_peak = peaks["mxf8f6f4_m128n144k32"]  # the P.V instruction's own measured peak
+    # Roofline time of the executed MMAs: QK^T in FP4; P.V twice (P_hi and P_lo terms) in FP8 at
+    # N = 144 (128 channels, the ones row that sums P, padding to a multiple of 16).
+    t_roof = p["qk_flops"] / (fp4_peak * 1e12) + 2 * p["qk_flops"] * (144 / 128) / (fp8_peak * 1e12)
+    attn_s = p["attn_ms"] * 1e-3
+    clocks = p["clocks"]
+    sm_hz = (clocks.get("sm_mhz") or 1965.0) * 1e6
+    # MUFU bound: one ex2 per executed score element, 16 per clock per SM.
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    mufu_s = p["tiles"] * 128 * 128 / (16.0 * sms * sm_hz)
+    return {
+        "workload": PREFILL_WORKLOAD, "value": p["flops"] / (p["ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
+        "ms_per_step": p["ms"], "steps": args.prefill_steps, "step": "quantize Q,K,V + causal prefill attention",
+        "attention_ms": p["attn_ms"], "attention_tflops": p["flops"] / attn_s / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "qk4v8_prefill_kernel<false>",
+                     "achieved": p["flops"] / attn_s / 1e12,
+                     "peak": p["flops"] / t_roof / 1e12, "unit": "TFLOPS",
+                     "frac": t_roof / attn_s,
+                     "peak_source": "measured tcgen05 peaks of the kernel's own MMA shapes (mma_peaks)"},
+        "qk_stage": {"kernel": "qk4v8_prefill_kernel<true> (QK^T stage build)", "ms": p["stage_ms"],
+                     "tflops": p["qk_flops"] / (p["stage_ms"] * 1e-3) / 1e12,
+                     "frac_of_measured_fp4": p["qk_flops"] / (p["stage_ms"] * 1e-3) / 1e12 / fp4_peak,
+                     "frac_of_spec_fp4_9pf": p["qk_flops"] / (p["stage_ms"] * 1e-3) / 1e12 / 9000.0},
+        "mma_peaks_tflops": peaks,
+        "mufu_bound_ms": mufu_s * 1e3, "mufu_frac": mufu_s / attn_s,
+        "bf16_x4_fp4_nominal_tflops": bf16_tf * 4.0,
+        "clocks": clocks,
+    }
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -418,6 +497,11 @@ def main():
         raise SystemExit("bench.py needs a CUDA device (B200); the library has no CPU path")
     world, rank, local = dist_setup(args.gpus)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = load_peaks()
+
+    if args.no_decode:
+        if rank == 0:
+            print(json.dumps({"prefill": prefill_object(args, peak_src, bf16_tf)}), flush=True)
+        return 0
 
     d = run_decode(args, world, rank)
     wl = d["wl"]
@@ -461,22 +545,7 @@ def main():
     }
 
     if not args.no_prefill:
-        p = run_prefill(args)
-        fp4_peak = bf16_tf * 4.0   # nominal dense ratio fp4 : bf16 = 9 : 2.25
-        fp8_peak = bf16_tf * 2.0   # nominal dense ratio fp8 : bf16 = 4.5 : 2.25
-        # Roofline time of the executed MMAs: QK^T in FP4, P.V twice (hi and lo terms) in FP8,
-        # plus the row-sum columns of V.
-        t_roof = p["qk_flops"] / (fp4_peak * 1e12) + 2 * p["qk_flops"] * (144 / 128) / (fp8_peak * 1e12)
-        line["prefill"] = {
-            "workload": PREFILL_WORKLOAD, "value": p["flops"] / (p["ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
-            "ms_per_step": p["ms"], "steps": args.prefill_steps, "step": "quantize Q,K,V + causal prefill attention",
-            "attention_ms": p["attn_ms"], "attention_tflops": p["flops"] / (p["attn_ms"] * 1e-3) / 1e12,
-            "roofline": {"bound": "tensor", "kernel": "qk4v8_attention_kernel<false>",
-                         "achieved": p["flops"] / (p["attn_ms"] * 1e-3) / 1e12,
-                         "peak": p["flops"] / t_roof / 1e12, "unit": "TFLOPS",
-                         "frac": t_roof / (p["attn_ms"] * 1e-3),
-                         "peak_source": f"{peak_src} bf16_tflops x4 (fp4) and x2 (fp8), nominal ratios"},
-        }
+        line["prefill"] = prefill_object(args, peak_src, bf16_tf)
         line["gpu_launches"] += 4 * args.prefill_steps
 
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
