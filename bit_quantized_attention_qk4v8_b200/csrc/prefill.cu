@@ -82,10 +82,9 @@ struct PfSmem {
     static constexpr int kSfV = kSfK + kPfKStages * 512;
     static constexpr int kSfP = kSfV + kPfVStages * 512;           // one atom per P buffer (P_hi and P_lo share it)
     static constexpr int kSfOne = kSfP + 2 * 512;
-    // Handshake slots [quarter][tile parity]: a flags word, then per row (lane)
-    // the shift E of O and the reference m_O.
-    static constexpr int kHsFlags = kSfOne + 512;                  // u32 [4][2]
-    static constexpr int kHsE = kHsFlags + 4 * 2 * 4;              // int [4][2][32]
+    // Handshake slots [quarter][tile parity][row (lane)]: the shift E of O, and
+    // (tile parity 0 only) the reference m_O.
+    static constexpr int kHsE = kSfOne + 512;                      // int [4][2][32]
     static constexpr int kHsM = kHsE + 4 * 2 * 32 * 4;             // float [4][2][32]
     static constexpr int kXmax = kHsM + 4 * 2 * 32 * 4;            // float [2 parities][128 rows] (QK stage)
     static constexpr int kBar = kXmax + 2 * 128 * 4;
@@ -168,11 +167,6 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ uint32_t lds32_volatile(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.volatile.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
 
 // Wait on an mbarrier phase that every peer reaches within its own bounded
 // waits. It does not give up on the abort flag, so all waiters see the same
@@ -545,12 +539,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int limit = u.L;
         if (p.causal) limit = imin(limit, qi + u.L - p.Sq + 1);
         limit = imax(limit, 0);
-        // Handshake slots of this quarter (shared-space addresses): flags [tile
-        // parity], E and m [tile parity][lane].
-        const uint32_t a_flags = smem_u32(smem + S::kHsFlags) + quarter * 8;
+        // Handshake slots of this thread's row (shared-space addresses), E and m
+        // by tile parity.
         const uint32_t a_e = smem_u32(smem + S::kHsE) + quarter * 256 + lane * 4;
         const uint32_t a_m = smem_u32(smem + S::kHsM) + quarter * 256 + lane * 4;
-        const uint32_t a_abort = smem_u32(smem + S::kMisc + 4);
         uint64_t *hs = hs_bar + quarter * 2;
         uint8_t *pbuf = smem + S::kP + pp * S::kPBuf;
         const int swz = row & 7;
@@ -572,9 +564,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         };
         auto receive = [&](int j) -> bool {
             if (!__all_sync(0xffffffffu, wait_bar(&hs[j & 1], (j >> 1) & 1, abort_flag, p.status))) return false;
-            const uint32_t f = lds32_volatile(a_flags + (j & 1) * 4);
-            if (f & 2u) return false;  // the owner is unwinding
-            if (f & 1u) e -= static_cast<int>(lds32(a_e + (j & 1) * 128));
+            e -= static_cast<int>(lds32(a_e + (j & 1) * 128));
             return true;
         };
 
@@ -584,13 +574,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const int jv = imax(0, imin(limit - i * 128, 128));  // keys j < jv are allowed
-            uint32_t pw[64];  // P bytes: P_hi words [0, 32), P_lo words [32, 64); 4 words per 16-key chunk
-            int eb[4];        // e + x of each block when it was encoded
+            int eb[4];  // e + x of each block when it was encoded
             // The tile in two halves of 64 keys, to bound the registers held at once.
             // S is released to the tensor core once the second half has been read.
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t sh[64];
+                uint32_t pw[32];  // this half's P bytes: P_hi words [0, 16), P_lo words [16, 32)
                 tc_ld_32x32b_x32(tmem + lane_base + pf_col_s(pp) + 64 * hh,
                                  *reinterpret_cast<uint32_t (*)[32]>(&sh[0]));
                 tc_ld_32x32b_x32(tmem + lane_base + pf_col_s(pp) + 64 * hh + 32,
@@ -672,9 +662,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             hh2[half] = h2;
                             ll2[half] = cvt_e4m3x2_from_f16x2(*reinterpret_cast<const uint32_t *>(&d));
                         }
-                        pw[8 * b + q] = __byte_perm(hh2[0], hh2[1], 0x5410);
-                        pw[32 + 8 * b + q] = __byte_perm(ll2[0], ll2[1], 0x5410);
+                        pw[8 * b2 + q] = __byte_perm(hh2[0], hh2[1], 0x5410);
+                        pw[16 + 8 * b2 + q] = __byte_perm(ll2[0], ll2[1], 0x5410);
                     }
+                }
+                // P buffer pp was last read by P V(i-2), issued at the end of this
+                // warp's previous tile.
+                if (hh == 0 && i >= 2 &&
+                    !__all_sync(0xffffffffu, wait_bar(&pv_done[pp], (k - 1) & 1, abort_flag, p.status))) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t prow = smem_u32(pbuf) + row * 128;
+#pragma unroll
+                for (int c2 = 0; c2 < 4; ++c2) {
+                    const uint32_t cofs = static_cast<uint32_t>(((4 * hh + c2) ^ swz) << 4);
+                    sts128(prow + cofs, pw[4 * c2], pw[4 * c2 + 1], pw[4 * c2 + 2], pw[4 * c2 + 3]);
+                    sts128(prow + 128 * 128 + cofs, pw[16 + 4 * c2], pw[17 + 4 * c2], pw[18 + 4 * c2], pw[19 + 4 * c2]);
                 }
             }
             if (!ok) break;
@@ -703,29 +707,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 tc_fence_after();
                 pf_rescale_o(tmem + lane_base + kPfColO, 144, E);
             }
-            {
-                if (any) sts32(a_e + (i & 1) * 128, static_cast<uint32_t>(E));
-                __syncwarp();
-                if (lane == 0) {
-                    sts32(a_flags + (i & 1) * 4, (any ? 1u : 0u) | (lds32_volatile(a_abort) ? 2u : 0u));
-                    mbar_arrive(&hs[i & 1]);
-                }
-            }
-            // P buffer pp was last read by P V(i-2), which has had this whole tile to
-            // finish.
-            if (i >= 2 && !__all_sync(0xffffffffu, wait_bar(&pv_done[pp], (k - 1) & 1, abort_flag, p.status))) {
-                ok = false;
-                break;
-            }
-            {
-                const uint32_t prow = smem_u32(pbuf) + row * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t cofs = static_cast<uint32_t>((c ^ swz) << 4);
-                    sts128(prow + cofs, pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-                    sts128(prow + 128 * 128 + cofs, pw[32 + 4 * c], pw[33 + 4 * c], pw[34 + 4 * c], pw[35 + 4 * c]);
-                }
-            }
+            // A warp that unwinds posts nothing; its peer's bounded wait then sees
+            // the abort flag.
+            sts32(a_e + (i & 1) * 128, static_cast<uint32_t>(E));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&hs[i & 1]);
             // Scale bytes of (row, block b): 2^(e + x) relative to m_O, with the
             // block's own e and the shifts of m_O since it was encoded. A block far
             // below m_O clamps at the smallest E8M0 value; it is negligible there.
