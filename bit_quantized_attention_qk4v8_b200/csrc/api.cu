@@ -56,7 +56,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
-// K codes [B*Hkv][cap][64] as a 3-D uint8 tensor, 128-token x 64-byte boxes,
+// MXFP4 codes [B*H][cap][64] (K, or Q for prefill) as a 3-D uint8 tensor, 128-token x 64-byte boxes,
 // 64-byte swizzle (one token row is exactly one swizzle span).
 int make_k_map(CUtensorMap *map, const uint8_t *codes, int BH, int cap) {
     auto enc = get_encode_fn();
@@ -206,8 +206,8 @@ int prefill_common(const uint8_t *q_codes, const uint8_t *q_scales, int B, int H
     if (Sq <= 0 || q_cap % 128 || q_cap < Sq || kv_cap <= 0 || kv_cap % 128 || Sk < 0 || Sk > kv_cap)
         return set_error(QK4V8_ERR_INVALID_ARG, "bad lengths Sq=%d q_cap=%d Sk=%d kv_cap=%d", Sq, q_cap, Sk, kv_cap);
     if ((st = check_device())) return st;
-    CUtensorMap tk, tv;
-    if ((st = make_k_map(&tk, k_codes, B * Hkv, kv_cap))) return st;
+    CUtensorMap tq, tk, tv;
+    if ((st = make_k_map(&tq, q_codes, B * Hq, q_cap)) || (st = make_k_map(&tk, k_codes, B * Hkv, kv_cap))) return st;
     if (stage_qk)
         tv = tk;  // unused by the QK^T stage
     else if ((st = make_v_map(&tv, v_codes, B * Hkv, kv_cap)))
@@ -237,10 +237,8 @@ int prefill_common(const uint8_t *q_codes, const uint8_t *q_scales, int B, int H
     p.status = dev_status;
     p.test_stall = g_test_stall;
     p.test_dump_s = g_test_dump_s;
-    const int grid = B * Hq * p.n_qtiles;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = stage_qk ? qk4v8::launch_prefill_stage_qk(tk, tv, p, grid, s)
-                             : qk4v8::launch_prefill(tk, tv, p, grid, s);
+    cudaError_t e = stage_qk ? qk4v8::launch_prefill_stage_qk(tq, tk, tv, p, s) : qk4v8::launch_prefill(tq, tk, tv, p, s);
     return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "attention (prefill) launch");
 }
 

@@ -51,12 +51,13 @@ cudaError_t launch_quantize_v(const void *v, int B, int S, int H, int64_t sb, in
                               cudaStream_t stream);
 cudaError_t launch_attention(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p,
                              int grid, cudaStream_t stream);
-// Prefill kernel (one CTA per (sequence, query head, 128-token query tile)),
-// and its QK^T-stage-only build over the same tile schedule.
-cudaError_t launch_prefill(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p, int grid,
-                           cudaStream_t stream);
-cudaError_t launch_prefill_stage_qk(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p,
-                                    int grid, cudaStream_t stream);
+// Prefill kernel (persistent: one CTA per SM over the (sequence, query head,
+// 128-token query tile) units), and its QK^T-stage-only build over the same
+// schedule. tmap_q maps the packed Q codes like tmap_k the K codes.
+cudaError_t launch_prefill(const CUtensorMap &tmap_q, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v,
+                           const AttnParams &p, cudaStream_t stream);
+cudaError_t launch_prefill_stage_qk(const CUtensorMap &tmap_q, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v,
+                                    const AttnParams &p, cudaStream_t stream);
 // Tensor-pipe peak run of one block-scaled MMA shape (measurement aid).
 cudaError_t launch_mma_peak(int kind, int ctas, int iters, int32_t *status, cudaStream_t stream);
 // Swap-AB split-KV decode kernel; handles G*nq <= kDecodeMaxRows query rows.
