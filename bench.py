@@ -58,6 +58,9 @@ def parse_args():
     ap.add_argument("--splits", type=int, default=0, help="decode KV splits (0 = library default)")
     ap.add_argument("--prefill-steps", type=int, default=10)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-extra-decode", action="store_true",
+                    help="skip the long-context and speculative-verify decode workloads")
+    ap.add_argument("--extra-steps", type=int, default=50, help="timed steps of each extra decode workload")
     ap.add_argument("--no-decode", action="store_true",
                     help="prefill only (a profiling aid): prints the prefill object alone")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -277,6 +280,67 @@ def run_decode(args, world, rank):
                 launches_per_step=launches, attn_timing=attn_timing,
                 clocks=clk.summary(), e2e_ms=e2e_ms, e2e_steps=e2e_steps,
                 h2d=q_host.numel() * 2, d2h=out_host.numel() * 2)
+
+
+def run_decode_workload(name, steps, warmup, hbm_gbs):
+    """One of the other decode workloads (long context, speculative verify): one
+    qk4v8_attention_decode_bf16 call per step over its pre-quantized cache."""
+    import torch
+    import bit_quantized_attention_qk4v8_b200 as qk
+    import synth
+    wl = synth.WORKLOADS[name]
+    gen = wl.generate()
+    lens = gen["seqlens"].astype(np.int64)
+    q = to_dev(gen["q"])
+    sl = torch.from_numpy(gen["seqlens"]).cuda()
+    cap = qk.round_cap(wl.Lk)
+    k = to_dev(gen["k"])
+    kp = qk.quantize_qk(k, cap=cap, seqlens=sl)
+    del k
+    v = to_dev(gen["v"])
+    vp = qk.quantize_v(v, cap=cap, seqlens=sl)
+    del v, gen
+    max_len = int(lens.max())
+    splits = qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, max_len)
+    ws_bytes = qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device="cuda") if ws_bytes else None
+    out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=max_len, num_splits=splits, workspace=ws, out=out)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(steps):
+            step()
+    graph.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    del graph
+    ms = t0.elapsed_time(t1) / steps
+    kv_bytes = int(lens.sum()) * wl.Hkv * KV_BYTES_PER_TOKEN_HEAD   # the packed cache each step streams
+    gbs = kv_bytes / (ms * 1e-3) / 1e9
+    rows = wl.G * wl.Sq
+    one_launch = rows <= 64 and splits == 1
+    return {
+        "workload": name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "nq": wl.Sq, "kv_len_mean": float(lens.mean()),
+        "kv_len_max": max_len, "kv_splits": splits, "ms_per_step": ms, "value": gbs, "unit": "GB/s",
+        "tokens_per_s": wl.B * wl.Sq / (ms * 1e-3),
+        "launches_per_step": 1 if one_launch else (2 if rows <= 64 else 3),
+        "roofline": {"bound": "hbm", "kernel": decode_kernel_name(rows), "achieved": gbs, "peak": hbm_gbs,
+                     "unit": "GB/s", "frac": gbs / hbm_gbs, "algorithmic_bytes_per_step": kv_bytes,
+                     "note": "step time (all launches of the call); the split kernel dominates it"},
+        "clocks": clk.summary(),
+    }
 
 
 # ---------------------------------------------------------------------------- prefill
@@ -544,6 +608,12 @@ def main():
         "clocks": d["clocks"],
     }
 
+    if not args.no_extra_decode and world == 1:
+        line["decode_workloads"] = {}
+        for name in ("decode_long_b8_hq64_hkv8_l64k_128k", "verify_b64_nq8_hq64_hkv8_l16384"):
+            w = run_decode_workload(name, args.extra_steps, min(args.warmup, 5), hbm_gbs)
+            line["decode_workloads"][name] = w
+            line["gpu_launches"] += w["launches_per_step"] * args.extra_steps
     if not args.no_prefill:
         line["prefill"] = prefill_object(args, peak_src, bf16_tf)
         line["gpu_launches"] += 4 * args.prefill_steps

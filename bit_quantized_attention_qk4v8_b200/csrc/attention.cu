@@ -15,10 +15,13 @@
 //  - V is extended with a row of ones, so column 128 of the O accumulator is
 //    the softmax denominator sum_j P_hi + P_lo, accumulated by the same MMA.
 //
-// One CTA computes one work unit: 128 query rows against one KV head.
-//  - Prefill unit: one query head and 128 consecutive query tokens.
+// One CTA computes one work unit: 128 query rows against one KV head. The
+// library launches it for split-KV decode with 65..128 query rows per KV head
+// (the swap-AB decode kernel covers up to 64, the prefill kernel prefill):
 //  - Decode unit: the G*nq query rows of a GQA group against one contiguous
 //    split of the KV cache. Rows go round-robin over the four TMEM lane quarters.
+//  - The kDecode = false form (one query head, 128 consecutive query tokens) is
+//    kept in the template but not instantiated.
 // Warp roles (192 threads):
 //  - warp 0: TMA producer (Q gather, K/V tiles, scale atoms; ragged-tile cleanup)
 //  - warp 1: TMEM allocator and single-thread MMA issuer
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const Unit u = decode_unit<kDecode>(p);
     const int T = u.tile_end - u.tile_begin;
-    if (T <= 0 || (p.status && *reinterpret_cast<const volatile int32_t *>(p.status) != 0)) {
+    if (T <= 0) {
         if (warp >= 2) write_empty_row<kDecode>(p, u, row_info<kDecode>(p, u, ((warp & 3) << 5) | lane));
         return;
     }
@@ -224,7 +227,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bars.p_full, 4);
         mbar_init(bars.pv_done, 1);
         mbar_init(bars.o_final, 1);
-        *abort_flag = 0;
+        // A status already set by another launch or CTA: unwind at once (every
+        // wait returns false), decided once for the whole CTA.
+        *abort_flag = (p.status && *reinterpret_cast<const volatile int32_t *>(p.status) != 0) ? 1u : 0u;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -615,27 +620,23 @@ __global__ void __launch_bounds__(256) qk4v8_decode_merge_kernel(const float *__
             wsum > 0.f ? (mx + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
 }
 
+// The 128-row kernel serves split-KV decode with more than 64 query rows per
+// KV head (prefill has its own kernel).
 cudaError_t launch_attention(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p, int grid,
                              cudaStream_t stream) {
+    if (!p.decode) return cudaErrorInvalidValue;
     // The dynamic shared-memory limit is a per-device function attribute.
     constexpr int kMaxDevices = 64;
-    static bool configured[2][kMaxDevices] = {};
+    static bool configured[kMaxDevices] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const int which = p.decode ? 1 : 0;
-    if (dev >= kMaxDevices || !configured[which][dev]) {
-        e = p.decode ? cudaFuncSetAttribute(qk4v8_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            kSmemBytes)
-                     : cudaFuncSetAttribute(qk4v8_attention_kernel<false>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (dev >= kMaxDevices || !configured[dev]) {
+        e = cudaFuncSetAttribute(qk4v8_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
-        if (dev < kMaxDevices) configured[which][dev] = true;
+        if (dev < kMaxDevices) configured[dev] = true;
     }
-    if (p.decode)
-        qk4v8_attention_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tmap_k, tmap_v, p);
-    else
-        qk4v8_attention_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tmap_k, tmap_v, p);
+    qk4v8_attention_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tmap_k, tmap_v, p);
     return cudaGetLastError();
 }
 

@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
         return ((static_cast<int64_t>(b) * p.Hq + h) * nq + t) * p.num_splits + split;
     };
 
-    if (T <= 0 || (p.status && *reinterpret_cast<const volatile int32_t *>(p.status) != 0)) {
+    if (T <= 0) {
         // A split with no key: O = 0 and lse2 = -inf for every query row.
         if (warp >= 2) {
             for (int idx = threadIdx.x - 64; idx < R * 32; idx += kSoftmaxThreads) {
@@ -279,7 +279,9 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
             mbar_init(&vote_bar[2 * g + 1], 4);
             mbar_init(&xe_bar[g], 4);
         }
-        *abort_flag = 0;
+        // A status already set by another launch or CTA: unwind at once (every
+        // wait returns false), decided once for the whole CTA.
+        *abort_flag = (p.status && *reinterpret_cast<const volatile int32_t *>(p.status) != 0) ? 1u : 0u;
         fence_barrier_init();
     }
     if (warp == 1) {
