@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--no-extra-decode", action="store_true",
                     help="skip the long-context and speculative-verify decode workloads")
     ap.add_argument("--extra-steps", type=int, default=50, help="timed steps of each extra decode workload")
+    ap.add_argument("--decode-workload", default=DECODE_WORKLOAD,
+                    help="decode workload of the main measurement (a profiling aid; the headline is the default)")
     ap.add_argument("--no-decode", action="store_true",
                     help="prefill only (a profiling aid): prints the prefill object alone")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -189,22 +191,23 @@ def run_decode(args, world, rank):
     import torch
     import bit_quantized_attention_qk4v8_b200 as qk
     import synth
-    wl = synth.WORKLOADS[DECODE_WORKLOAD]
+    wl = synth.WORKLOADS[args.decode_workload]
     gen = wl.generate()
     q_host = torch.from_numpy(gen["q"].view(np.int16)).view(torch.bfloat16).pin_memory()
     q = q_host.cuda()
     sl = torch.from_numpy(gen["seqlens"]).cuda()
     kp = qk.quantize_qk(to_dev(gen["k"]), seqlens=sl)      # the cache: quantized once, outside the timing
     vp = qk.quantize_v(to_dev(gen["v"]), seqlens=sl)
-    splits = args.splits if args.splits > 0 else qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, wl.Lk)
+    max_len = int(gen["seqlens"].max())
+    splits = args.splits if args.splits > 0 else qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, max_len)
     ws_bytes = qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)
     ws = torch.empty((ws_bytes,), dtype=torch.uint8, device="cuda") if ws_bytes else None
     out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
-    kv_bytes = wl.B * wl.Hkv * wl.Lk * KV_BYTES_PER_TOKEN_HEAD
+    kv_bytes = int(gen["seqlens"].astype(np.int64).sum()) * wl.Hkv * KV_BYTES_PER_TOKEN_HEAD
 
     def step():
-        qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=wl.Lk, num_splits=splits, workspace=ws, out=out)
+        qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=max_len, num_splits=splits, workspace=ws, out=out)
 
     for _ in range(args.warmup):
         step()
@@ -260,7 +263,7 @@ def run_decode(args, world, rank):
 
     def e2e_step():
         q.copy_(q_host, non_blocking=True)
-        qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=wl.Lk, num_splits=splits, workspace=ws, out=out)
+        qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=max_len, num_splits=splits, workspace=ws, out=out)
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(min(args.warmup, 5)):
@@ -590,9 +593,9 @@ def main():
         "dtype": "e2m1/e4m3 MMA, f32 softmax and accumulate",
         "data": "synthetic",
         "config": {
-            "workload": DECODE_WORKLOAD, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "nq": wl.Sq, "L": wl.Lk, "d": 128,
+            "workload": args.decode_workload, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "nq": wl.Sq, "L": wl.Lk, "d": 128,
             "kv_splits": d["splits"], "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": "no flush: the packed KV cache (419 MB) is larger than L2 (126 MB)",
+            "l2": f"no flush: the packed KV cache ({d['kv_bytes'] / 1e6:.0f} MB) is larger than L2 (126 MB)",
             "tokens_per_s": wl.B * wl.Sq * steps * world / (d["elapsed_ms"] * 1e-3),
         },
         "roofline": {

@@ -137,9 +137,44 @@ __device__ __forceinline__ void tmem_store_cols(uint32_t taddr, const uint32_t (
     }
 }
 
-__device__ __forceinline__ void st_u8(uint8_t *base, int off, uint32_t v) {
-    base[off] = static_cast<uint8_t>(v);
+// Low byte of v to shared address addr + kOff (the offset folds into the store).
+template <int kOff>
+__device__ __forceinline__ void sts_u8(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.b8 [%0+%2], %1;" ::"r"(addr), "r"(v), "n"(kOff) : "memory");
 }
+
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// Stores the P^T bytes of query rows i and i+1 (P_hi rows at 0, P_lo rows at
+// NT*128) for this thread's token. pa is the token's byte in row 0; the
+// 128-byte swizzle moves row r's byte to 16-byte chunk (chunk ^ (r % 8)), so row
+// r sits at (pa ^ ((r & 7) << 4)) + r * 128 (the buffer base is 1024-aligned).
+template <int NT, int I>
+__device__ __forceinline__ void store_p_pair(uint32_t pa, uint32_t h2, uint32_t l2) {
+    const uint32_t a0 = pa ^ static_cast<uint32_t>((I & 7) << 4);
+    const uint32_t a1 = pa ^ static_cast<uint32_t>(((I + 1) & 7) << 4);
+    sts_u8<I * 128>(a0, h2);
+    sts_u8<I * 128 + NT * 128>(a0, l2);
+    sts_u8<(I + 1) * 128>(a1, h2 >> 8);
+    sts_u8<(I + 1) * 128 + NT * 128>(a1, l2 >> 8);
+}
+
+template <int NT, int I, int NC>
+struct StorePairs {
+    __device__ __forceinline__ static void run(uint32_t pa, const uint32_t (&h)[NC / 2], const uint32_t (&l)[NC / 2]) {
+        store_p_pair<NT, I>(pa, h[I / 2], l[I / 2]);
+        StorePairs<NT, I + 2, NC>::run(pa, h, l);
+    }
+};
+template <int NT, int NC>
+struct StorePairs<NT, NC, NC> {
+    __device__ __forceinline__ static void run(uint32_t, const uint32_t (&)[NC / 2], const uint32_t (&)[NC / 2]) {}
+};
 
 // Wait on an mbarrier phase that every peer reaches within its own bounded
 // waits. Unlike wait_bar it does not give up on the abort flag, so all waiters
@@ -501,6 +536,7 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
         // pofs ^ ((i & 7) << 4) plus i * 128: the 128-byte swizzle puts token jt
         // of row n in 16-byte chunk (jt / 16) ^ (n % 8), and c0 is a multiple of 8.
         const int pofs = c0 * 128 + ((jt >> 4) << 4) + (jt & 15);
+        const uint32_t pa_base = smem_u32(smem + Lay::kP) + static_cast<uint32_t>(pofs);
         // Per query row: -m, this warp's reference max (log2 units, so p =
         // 2^(s * scale - m)), kept in shared memory as it is the same for all
         // lanes; lacc, this thread's share of the row sum relative to m. Lane
@@ -539,7 +575,7 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
             float mrow[NC];
 #pragma unroll
             for (int i = 0; i < NC; i += 4) {
-                const float4 m4 = *reinterpret_cast<const float4 *>(m_neg + i);
+                const float4 m4 = lds_f4(smem_u32(m_neg + i));
                 mrow[i] = m4.x;
                 mrow[i + 1] = m4.y;
                 mrow[i + 2] = m4.z;
@@ -622,7 +658,8 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
             // below what P_lo resolves): P_hi = E4M3(p); its value comes back
             // exactly as f16; P_lo = E4M3(32 (p - P_hi)), where the difference is
             // exact since P_hi is within 2^-4 of p. The row sums take p itself.
-            uint8_t *pb = smem + Lay::kP + sbuf * Lay::kPBytes;
+            const uint32_t pa = pa_base + static_cast<uint32_t>(sbuf * Lay::kPBytes);
+            uint32_t hb[NC / 2], lb[NC / 2];
             const __half2 k32 = __float2half2_rn(32.f), km32 = __float2half2_rn(-32.f);
 #pragma unroll
             for (int i = 0; i < NC; i += 2) {
@@ -637,13 +674,10 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
                 const uint32_t hvw = cvt_e4m3x2_to_f16x2(h2);
                 const __half2 d = __hfma2(*reinterpret_cast<const __half2 *>(&hvw), km32, __hmul2(ph, k32));
                 const uint16_t l2 = cvt_e4m3x2_from_f16x2(*reinterpret_cast<const uint32_t *>(&d));
-                const int o0 = (pofs ^ ((i & 7) << 4)) + i * 128;
-                const int o1 = (pofs ^ (((i + 1) & 7) << 4)) + (i + 1) * 128;
-                st_u8(pb, o0, h2);
-                st_u8(pb, o0 + NT * 128, l2);
-                st_u8(pb, o1, h2 >> 8);
-                st_u8(pb, o1 + NT * 128, l2 >> 8);
+                hb[i / 2] = h2;
+                lb[i / 2] = l2;
             }
+            StorePairs<NT, 0, NC>::run(pa, hb, lb);
             // Collect the vote. Every warp of the group reads the same four words.
             const bool okv = wait_bar_peers(&vote_bar[2 * cg + sbuf], (it >> 1) & 1);
             const uint32_t flags = okv ? (votes[sbuf * 4] | votes[sbuf * 4 + 1] | votes[sbuf * 4 + 2] |
