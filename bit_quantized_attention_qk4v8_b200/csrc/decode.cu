@@ -88,8 +88,9 @@ struct DecodeLayout {
     static constexpr int kMneg = kVote + 128;   // [softmax warp][NC] float: -m of each row
     static constexpr int kBar = kMneg + 1024;
     // kv_full/empty per stage, q_full, patch, s_full x2, p_full x2, pv_done x2,
+    // s_free x2,
     // o_final, vote x2 and e exchange per column group.
-    static constexpr int kNumBars = 2 * ST + 9 + 3 * kCG;
+    static constexpr int kNumBars = 2 * ST + 9 + 3 * kCG + 2;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16 + 1024;
     // TMEM columns: S^T x2 [0, 2NT), O^T [2NT, 4NT), then scale factors:
@@ -284,15 +285,15 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
     uint64_t *kv_empty = bars + kStagesD;
     uint64_t *q_full = bars + 2 * kStagesD;
     uint64_t *patch = q_full + 1;
-    // S buffer (it & 1) needs no release barrier: the MMA warp issues S(it+2)
-    // only after waiting for p_full of tile it, and every softmax warp arrives
-    // there after its reads of S(it) have completed.
+    // S buffer (it & 1) is released by s_free: every softmax warp arrives there
+    // once its read of S(it) has completed, early in the tile.
     uint64_t *s_full = q_full + 2;   // [2]
     uint64_t *p_full = q_full + 4;   // [2]
     uint64_t *pv_done = q_full + 6;  // [2]
     uint64_t *o_final = q_full + 8;
     uint64_t *vote_bar = q_full + 9;             // [column group][tile parity]: one arrival per warp
     uint64_t *xe_bar = vote_bar + 2 * Lay::kCG;  // [column group]: offsets posted for an O rescale
+    uint64_t *s_free = xe_bar + Lay::kCG;        // [2]: S buffer read by every softmax warp
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::kMisc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + Lay::kMisc + 4);
 
@@ -305,6 +306,7 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
         mbar_init(patch, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
+            mbar_init(&s_free[s], Lay::kSoftmaxWarps);
             mbar_init(&p_full[s], Lay::kSoftmaxWarps);
             mbar_init(&pv_done[s], 1);
         }
@@ -427,12 +429,15 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
                 __syncwarp();
                 return true;
             };
-            for (int it = 0; it < T && ok; ++it) {
+            // S(it) = K(it) Q^T into S buffer it & 1, once K/V(it) have landed and
+            // (from it = 2 on) every softmax warp has read S(it-2).
+            auto issue_qk = [&](int it) -> bool {
                 const int st = it % kStagesD;
                 const int sbuf = it & 1;
-                ok = wait_bar(&kv_full[st], (it / kStagesD) & 1, abort_flag, p.status);
-                if (ok && last_partial && it == T - 1) ok = wait_bar(patch, 0, abort_flag, p.status);
-                if (!__all_sync(0xffffffffu, ok)) break;
+                bool w = wait_bar(&kv_full[st], (it / kStagesD) & 1, abort_flag, p.status);
+                if (w && last_partial && it == T - 1) w = wait_bar(patch, 0, abort_flag, p.status);
+                if (w && it >= 2) w = wait_bar(&s_free[sbuf], ((it - 2) >> 1) & 1, abort_flag, p.status);
+                if (!__all_sync(0xffffffffu, w)) return false;
                 tc_fence_after();
                 const uint32_t tSfK = tmem + col_sf_k_d(NT, sbuf);
                 const uint64_t dK = dK0 + static_cast<uint64_t>(st * (Lay::kKBytes >> 4));
@@ -446,9 +451,27 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
                     tc_commit(&s_full[sbuf]);
                 }
                 __syncwarp();
-                if (it >= 1) ok = issue_pv(it - 1);
+                return true;
+            };
+            if (ST >= 5) {
+                // Deep K/V pipeline: S(it+2) goes out as soon as S(it) has been read
+                // (early in tile it), ahead of P V(it) (end of tile it), so the next
+                // scores are ready when the softmax warps finish a tile.
+                ok = issue_qk(0);
+                if (ok && T > 1) ok = issue_qk(1);
+                for (int it = 0; it < T && ok; ++it) {
+                    if (it + 2 < T) ok = issue_qk(it + 2);
+                    if (ok) ok = issue_pv(it);
+                }
+            } else {
+                // Shallow pipeline: S(it) waits for K/V(it), which needs the stage that
+                // P V(it - ST) frees, so P V goes first.
+                for (int it = 0; it < T && ok; ++it) {
+                    ok = issue_qk(it);
+                    if (ok && it >= 1) ok = issue_pv(it - 1);
+                }
+                if (ok) ok = issue_pv(T - 1);
             }
-            if (ok) ok = issue_pv(T - 1);
             if (ok && leader) tc_commit(o_final);
         }
         __syncwarp();
@@ -567,6 +590,9 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
                 tmem_load_cols<NC>(tmem + lane_base + static_cast<uint32_t>(NT * sbuf + c0), sraw);
                 tc_wait_ld();
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[sbuf]);  // the tensor core may now compute S(it+2)
 
             // u = s * scale - m (log2 units); -inf where the key is masked. Every row
             // may see this key unless it lies past L, or in the last nq-1 positions
