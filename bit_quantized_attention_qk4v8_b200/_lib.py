@@ -42,6 +42,7 @@ SIGNATURES = {
                                      _i32, _i32, _f32, _i32, _vp, _sz, _vp, _vp, _vp, _vp], _i32),
     "qk4v8_test_set_stall": ([_i32], None),
     "qk4v8_test_set_dump_scores": ([_vp], None),
+    "qk4v8_test_set_force_swap_ab": ([_i32], None),
     "qk4v8_test_prefill_stage_qk": ([_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _f32,
                                      _vp, _vp, _vp], _i32),
     "qk4v8_test_mma_peak": ([_i32, _i32, _i32, _vp, _vp], _i32),

@@ -4,13 +4,14 @@ from __future__ import annotations
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqk4v8.so")
-SOURCES = ["quantize.cu", "attention.cu", "prefill.cu", "decode.cu", "mma_peak.cu", "api.cu"]
-HEADERS = ["ptx.cuh", "pipeline.cuh", "mx_encode.cuh", "qk4v8_internal.h"]
+SOURCES = ["quantize.cu", "attention.cu", "prefill.cu", "decode.cu", "gqa_decode.cu", "mma_peak.cu", "api.cu"]
+HEADERS = ["ptx.cuh", "pipeline.cuh", "mx_encode.cuh", "tile_ops.cuh", "qk4v8_internal.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -41,14 +42,18 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
     flags = NVCC_FLAGS + list(extra_flags or [])
-    objs = []
+    objs, cmds = [], []
     for src in SOURCES:
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
         cmd = [_nvcc(), *flags, "-I", os.path.join(ROOT, "include"), "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
         objs.append(obj)
+    # The translation units are independent: compile them side by side.
+    with ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 1)) as pool:
+        for _ in pool.map(lambda c: subprocess.run(c, check=True), cmds):
+            pass
     tmp = LIB + ".tmp"
     cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC", *objs,
            "-o", tmp]

@@ -20,6 +20,7 @@ namespace {
 thread_local char g_last_error[512] = "";
 int g_test_stall = 0;
 float *g_test_dump_s = nullptr;
+int g_test_force_swap_ab = 0;
 
 int set_error(int status, const char *fmt, ...) {
     va_list ap;
@@ -315,7 +316,17 @@ struct DecodeQuery {
     int64_t sb = 0, st = 0, sh = 0;
 };
 
-bool swap_ab_rows(int Hq, int Hkv, int nq) { return (Hq / Hkv) * nq <= qk4v8::kDecodeMaxRows; }
+// Which split kernel serves a GQA group of G*nq query rows: the swap-AB kernel
+// up to 32 rows (or up to 64 under the test hook), the GQA decode kernel for
+// 33..64, the 128-row attention kernel above. The first two write the output
+// directly when there is one split.
+bool swap_ab_rows(int Hq, int Hkv, int nq) {
+    const int rows = (Hq / Hkv) * nq;
+    return rows < qk4v8::kGqaMinRows || (g_test_force_swap_ab && rows <= qk4v8::kDecodeMaxRows);
+}
+bool gqa_rows(int Hq, int Hkv, int nq) {
+    return !swap_ab_rows(Hq, Hkv, nq) && (Hq / Hkv) * nq <= qk4v8::kDecodeMaxRows;
+}
 
 // Validates decode arguments, builds the tensor maps and launches the split-KV
 // kernel. With `out` given and a single split on the swap-AB kernel, the kernel
@@ -346,11 +357,11 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
         return set_error(QK4V8_ERR_INVALID_ARG, "bad lengths q_cap=%d kv_cap=%d max_seqlen=%d", q.cap, kv_cap,
                          max_seqlen);
     if (q.bf16 && !swap_ab_rows(Hq, Hkv, nq))
-        return set_error(QK4V8_ERR_INVALID_ARG, "bf16 Q in the split kernel needs (Hq/Hkv)*nq <= %d",
-                         qk4v8::kDecodeMaxRows);
+        return set_error(QK4V8_ERR_INVALID_ARG, "bf16 Q in the split kernel needs (Hq/Hkv)*nq < %d",
+                         qk4v8::kGqaMinRows);
     if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
     const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen);
-    const bool direct_out = out && splits == 1 && swap_ab_rows(Hq, Hkv, nq);
+    const bool direct_out = out && splits == 1 && (swap_ab_rows(Hq, Hkv, nq) || gqa_rows(Hq, Hkv, nq));
     if (out && !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
     const size_t need = direct_out ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
     if (need && (!workspace || !aligned16(workspace) || workspace_bytes < need))
@@ -396,9 +407,11 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
     p.status = dev_status;
     p.test_stall = g_test_stall;
     p.test_dump_s = g_test_dump_s;
-    // G*nq <= 64 query rows: the swap-AB decode kernel; larger groups use the
-    // 128-row attention kernel in its decode instantiation.
+    // G*nq <= 32 query rows: the swap-AB decode kernel; 33..64: the GQA decode
+    // kernel; larger groups use the 128-row attention kernel in its decode
+    // instantiation.
     cudaError_t e = swap_ab_rows(Hq, Hkv, nq) ? qk4v8::launch_decode(tk, tv, p, B * Hkv * splits, stream)
+                    : gqa_rows(Hq, Hkv, nq)   ? qk4v8::launch_gqa_decode(tk, tv, p, stream)
                                               : qk4v8::launch_attention(tk, tv, p, B * Hkv * splits, stream);
     if (e != cudaSuccess) return cuda_error(e, "attention (decode) launch");
     *splits_used = splits;
@@ -467,10 +480,15 @@ int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int 
 
 size_t qk4v8_decode_bf16_workspace_bytes(int B, int Hq, int Hkv, int nq, int num_splits) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq <= 0 || num_splits <= 0) return 0;
-    if (swap_ab_rows(Hq, Hkv, nq)) return num_splits == 1 ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits);
+    // Sized by the row count alone (not by the test hook that moves groups of
+    // 33..64 rows to the swap-AB kernel, which needs less).
+    const int rows = (Hq / Hkv) * nq;
+    if (rows < qk4v8::kGqaMinRows) return num_splits == 1 ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits);
     // Larger groups: the queries are quantized into the front of the workspace
-    // (capacity 128 tokens), then the split partials follow.
+    // (capacity 128 tokens), then the split partials follow (none when the GQA
+    // decode kernel writes the output directly from one split).
     const size_t packed = qk4v8_mxfp4_codes_bytes(B, Hq, 128) + qk4v8_scales_bytes(B, Hq, 128);
+    if (rows <= qk4v8::kDecodeMaxRows && num_splits == 1) return packed;
     return packed + qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits);
 }
 
@@ -504,8 +522,8 @@ int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_
         if (st || direct) return st;
         return qk4v8_decode_merge(workspace, workspace_bytes, B, Hq, nq, used, out, lse, stream);
     }
-    // More than 64 query rows per KV head: quantize Q into the front of the
-    // workspace for the 128-row kernel.
+    // More than 32 query rows per KV head: quantize Q into the front of the
+    // workspace for the GQA decode kernel or the 128-row kernel.
     uint8_t *qc = static_cast<uint8_t *>(workspace);
     uint8_t *qs = qc + qk4v8_mxfp4_codes_bytes(B, Hq, 128);
     uint8_t *rest = qs + qk4v8_scales_bytes(B, Hq, 128);
@@ -516,9 +534,9 @@ int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_
     dq.scales = qs;
     dq.cap = 128;
     st = decode_splitkv(dq, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
-                        causal_in_block, softmax_scale, splits, rest, rest_bytes, nullptr, nullptr, dev_status, s,
-                        &used, &direct);
-    if (st) return st;
+                        causal_in_block, softmax_scale, splits, rest, rest_bytes, out, lse, dev_status, s, &used,
+                        &direct);
+    if (st || direct) return st;
     return qk4v8_decode_merge(rest, rest_bytes, B, Hq, nq, used, out, lse, stream);
 }
 
@@ -530,6 +548,10 @@ void qk4v8_test_set_stall(int enable) { g_test_stall = enable ? 1 : 0; }
 // Test hook (declared in include/qk4v8_test.h): while set, CTA 0 of each
 // attention launch writes its first raw score tile to `dev_ptr`.
 void qk4v8_test_set_dump_scores(float *dev_ptr) { g_test_dump_s = dev_ptr; }
+
+// Test hook (declared in include/qk4v8_test.h): while enabled, decode groups of
+// 33..64 query rows run on the swap-AB kernel instead of the GQA decode kernel.
+void qk4v8_test_set_force_swap_ab(int enable) { g_test_force_swap_ab = enable ? 1 : 0; }
 
 int qk4v8_test_mma_peak(int kind, int ctas, int iters, int32_t *dev_status, void *stream) {
     if (kind < 0 || kind > 3 || ctas <= 0 || ctas > 65535 || iters <= 0 || iters > (1 << 24))

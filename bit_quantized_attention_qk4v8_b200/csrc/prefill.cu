@@ -50,6 +50,7 @@
 #include "pipeline.cuh"
 #include "ptx.cuh"
 #include "qk4v8_internal.h"
+#include "tile_ops.cuh"
 
 namespace qk4v8 {
 
@@ -119,98 +120,6 @@ constexpr uint32_t pf_idesc(uint32_t fmt, uint32_t n) {
 constexpr uint32_t kPfIdQK = pf_idesc(1u, 128);             // E2M1 x E2M1, N = 128 keys
 constexpr uint32_t kPfIdPV = pf_idesc(0u, PfSmem::kVRows);  // E4M3 x E4M3, N = 144
 __device__ __forceinline__ uint32_t pf_sf_id(uint32_t idesc, uint32_t id) { return idesc | (id << 29) | (id << 4); }
-
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-
-// Largest of 32 floats (as raw bits), a tree of three-input maxima.
-__device__ __forceinline__ float max32(const uint32_t (&s)[32]) {
-    float t[11];
-#pragma unroll
-    for (int g = 0; g < 10; ++g)
-        t[g] = fmax3(__uint_as_float(s[3 * g]), __uint_as_float(s[3 * g + 1]), __uint_as_float(s[3 * g + 2]));
-    t[10] = fmaxf(__uint_as_float(s[30]), __uint_as_float(s[31]));
-    const float a = fmax3(t[0], t[1], t[2]), b = fmax3(t[3], t[4], t[5]), c = fmax3(t[6], t[7], t[8]);
-    return fmaxf(fmax3(a, b, c), fmaxf(t[9], t[10]));
-}
-
-__device__ __forceinline__ uint32_t tc_ld_32x32b_x1(uint32_t taddr) {
-    uint32_t r;
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
-    return r;
-}
-
-__device__ __forceinline__ void tc_ld_32x32b_x4(uint32_t taddr, uint32_t (&r)[4]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(taddr));
-}
-
-__device__ __forceinline__ void tc_st_32x32b_x4(uint32_t taddr, const uint32_t (&r)[4]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]),
-                 "r"(r[1]), "r"(r[2]), "r"(r[3])
-                 : "memory");
-}
-
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
-__device__ __forceinline__ void sts32(uint32_t addr, uint32_t a) {
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
-}
-
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-
-
-// Wait on an mbarrier phase that every peer reaches within its own bounded
-// waits. It does not give up on the abort flag, so all waiters see the same
-// phase and take the same branch afterwards.
-constexpr uint64_t kPfVoteTimeoutNs = 4 * kWaitTimeoutNs;
-
-__device__ __noinline__ bool pf_wait_peers_slow(uint64_t *bar, uint32_t parity) {
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait_sleep(bar, parity, 20000))
-        if (globaltimer_ns() - t0 > kPfVoteTimeoutNs) return false;
-    return true;
-}
-
-__device__ __forceinline__ bool pf_wait_peers(uint64_t *bar, uint32_t parity) {
-    return mbar_try_wait(bar, parity) || pf_wait_peers_slow(bar, parity);
-}
-
-// O *= 2^-E for the four columns at taddr of this thread's row, E >= 0.
-__device__ __noinline__ void pf_rescale_o(uint32_t taddr, int ncols, int E) {
-    const float a = E < 126 ? __uint_as_float(static_cast<uint32_t>(127 - E) << 23) : 0.f;
-    for (int c = 0; c < ncols; c += 4) {
-        uint32_t o[4];
-        tc_ld_32x32b_x4(taddr + c, o);
-        tc_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 4; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
-        tc_st_32x32b_x4(taddr + c, o);
-    }
-    tc_wait_st();
-}
-
-// End of the CTA: every warp arrives here from its own role branch (the
-// warpgroups hold different register counts, so they never share this code);
-// the MMA warp then frees the tensor memory.
-__device__ __forceinline__ void pf_teardown(bool mma_warp, uint32_t tmem, uint32_t ncols) {
-    tc_fence_before();
-    __syncthreads();
-    if (mma_warp) {
-        tc_fence_after();
-        tmem_dealloc(tmem, ncols);
-    }
-}
 
 struct PfUnit {
     int b, h_q, h_kv, q0, L, T;
@@ -560,7 +469,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // when the loop unwound early, so TMEM is freed with nothing in flight.
         if (leader) tc_commit(drain);
         __syncwarp();
-        (void)pf_wait_peers(drain, 0);
+        (void)wait_peers(drain, 0);
     } else if (warp < kPfSoftmaxWarps) {
         // ------------------------------------------------------------------ softmax
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -759,7 +668,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    pf_rescale_o(tmem + lane_base + kPfColO, 144, E);
+                    rescale_o_lane(tmem + lane_base + kPfColO, 144, E);
                 }
                 // A warp that unwinds posts nothing; its peer's bounded wait then sees
                 // the abort flag.
@@ -842,7 +751,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             ++c;
         }
     }
-    pf_teardown(warp == kPfMmaWarp, tmem, kPfTmemCols);
+    teardown_tmem(warp == kPfMmaWarp, tmem, kPfTmemCols);
 }
 
 template <bool kStageQK>

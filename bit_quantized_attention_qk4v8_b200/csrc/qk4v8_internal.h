@@ -64,6 +64,11 @@ cudaError_t launch_mma_peak(int kind, int ctas, int iters, int32_t *status, cuda
 constexpr int kDecodeMaxRows = 64;
 cudaError_t launch_decode(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p, int grid,
                           cudaStream_t stream);
+// GQA decode kernel for kGqaMinRows..kDecodeMaxRows query rows per KV head
+// (persistent over the (sequence, KV head, split) units; packed MXFP4 queries).
+constexpr int kGqaMinRows = 33;
+cudaError_t launch_gqa_decode(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p,
+                              cudaStream_t stream);
 cudaError_t launch_decode_merge(const float *ws_o, const float *ws_lse, int B, int Hq, int nq, int splits,
                                 __nv_bfloat16 *out, float *lse, cudaStream_t stream);
 

@@ -33,6 +33,15 @@ QK4V8_API void qk4v8_test_set_stall(int enable);
 QK4V8_API void qk4v8_test_set_dump_scores(float *dev_ptr);
 
 /*
+ * While `enable` is non-zero, decode calls whose GQA group has 33..64 query
+ * rows per KV head run on the swap-AB split kernel (the one that serves up to
+ * 32 rows) instead of the GQA decode kernel, so that tests and measurements
+ * can compare the two. Both compute the same attention. Host-side state, not
+ * thread safe; workspace sizes do not depend on it.
+ */
+QK4V8_API void qk4v8_test_set_force_swap_ab(int enable);
+
+/*
  * The QK^T stage of qk4v8_attention_prefill alone, for measurement: the same
  * prefill kernel built without exp, P and P V, over the same causal tile
  * schedule (Q and K loads with their scale atoms, the block-scaled FP4 MMAs,

@@ -120,7 +120,10 @@ def test_bf16_decode_workspace_bytes(lib):
     part = lib.qk4v8_decode_workspace_bytes
     assert f(32, 32, 8, 1, 1) == 0                      # 4 rows, one split: written directly, no scratch
     assert f(32, 32, 8, 1, 3) == part(32, 32, 1, 3)      # partials for the merge
-    assert f(2, 64, 8, 8, 1) == 0                        # 64 rows still on the split kernel
+    assert f(2, 32, 8, 8, 1) == 0                        # 32 rows: quantized inside the swap-AB kernel
+    packed_64 = 2 * 64 * 128 * 64 + 2 * 64 * 512          # 33..64 rows: MXFP4 Q, capacity 128, in front
+    assert f(2, 64, 8, 8, 1) == packed_64                # one split: the GQA decode kernel writes out directly
+    assert f(2, 64, 8, 8, 2) == packed_64 + part(2, 64, 8, 2)
     packed_q = 2 * 128 * 128 * 64 + 2 * 128 * 512         # 128 rows: MXFP4 Q, capacity 128, in front
     assert f(2, 128, 8, 8, 2) == packed_q + part(2, 128, 8, 2)
     assert f(0, 8, 8, 1, 1) == 0 and f(1, 30, 8, 1, 1) == 0

@@ -148,6 +148,10 @@ def test_prefill_softmax_scale_and_peaked_scores():
     (2, 1, 3000, 64, 8, 1, [3000, 2999]),  # GQA 8, one token: 8 rows, one split (direct output)
     (2, 5, 700, 5, 5, 2, [700, 64]),   # G*nq = 5
     (2, 4, 800, 32, 4, 2, [800, 511]),  # G*nq = 32: the 32-row instance
+    (2, 8, 1100, 24, 4, 0, [1100, 513]),  # G*nq = 48: the GQA decode kernel, odd tile counts
+    (1, 3, 900, 11, 1, 2, None),          # G*nq = 33: the GQA decode kernel's smallest group
+    (3, 8, 1000, 64, 8, 3, [1000, 129, 1]),  # 64 rows, splits of 3 tiles, a one-tile and a one-key sequence
+    (2, 4, 2300, 16, 1, 1, [2300, 2001]),  # 64 rows from 16 heads x 4 tokens, direct output
 ])
 def test_decode_parity(B, nq, L, Hq, Hkv, splits, lens):
     gen = make_gen(B, nq, L, Hq, Hkv, seed=L + nq, lens=lens, k_out=4)
@@ -283,3 +287,44 @@ def test_prefill_o_rescale_path():
     assert_close(out, ref, "prefill O rescale")
     l = lse.cpu().numpy().transpose(0, 2, 1)
     assert np.abs(l - rlse).max() < 1e-2 + 1e-5 * np.abs(rlse).max()
+
+
+@pytest.mark.parametrize("B,nq,L,Hq,Hkv,splits", [
+    (2, 8, 1500, 64, 8, 1),
+    (2, 8, 1500, 40, 8, 2),
+])
+def test_gqa_decode_kernel_agrees_with_swap_ab_kernel(B, nq, L, Hq, Hkv, splits):
+    """33..64 query rows per KV head: the GQA decode kernel and the swap-AB kernel
+    (selected by a test hook) compute the same attention, each within the
+    oracle's tolerance."""
+    gen = make_gen(B, nq, L, Hq, Hkv, seed=L + Hq, k_out=4)
+    (ref, rlse), _ = oracle_attention_from(gen, True)
+    out_gqa, lse_gqa, _ = run_decode(gen, True, splits)
+    _lib.lib().qk4v8_test_set_force_swap_ab(1)
+    try:
+        out_swap, lse_swap, _ = run_decode(gen, True, splits)
+    finally:
+        _lib.lib().qk4v8_test_set_force_swap_ab(0)
+    assert_close(out_gqa, ref, "GQA decode kernel")
+    assert_close(out_swap, ref, "swap-AB kernel")
+    fin = np.isfinite(rlse)
+    for lse in (lse_gqa, lse_swap):
+        l = lse.cpu().numpy().transpose(0, 2, 1)
+        assert np.abs(l[fin] - rlse[fin]).max() < 1e-2
+
+
+def test_gqa_decode_o_rescale_path():
+    """64 rows per KV head; later keys score far (>64 binades) above the first
+    tile's row max, so the GQA decode kernel rescales O mid-row (both lanes of
+    each row, agreed between the two threads that own them)."""
+    gen = make_gen(1, 8, 1024, 16, 2, seed=43)
+    k = (gen["k"].astype(np.uint32) << 16).view(np.float32).copy()
+    k[:, :128] *= np.float32(1e-3)      # the first key tile: near-zero scores
+    gen["k"] = f32_to_bf16_bits(k)
+    scale = 6.0
+    for splits in (1, 2):
+        out, lse, _ = run_decode(gen, False, splits, scale=scale)
+        (ref, rlse), _ = oracle_attention_from(gen, False, scale=scale)
+        assert_close(out, ref, f"GQA decode O rescale, splits={splits}")
+        l = lse.cpu().numpy().transpose(0, 2, 1)
+        assert np.abs(l - rlse).max() < 1e-2 + 1e-5 * np.abs(rlse).max()
