@@ -480,8 +480,10 @@ int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int 
 
 size_t qk4v8_decode_bf16_workspace_bytes(int B, int Hq, int Hkv, int nq, int num_splits) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq <= 0 || num_splits <= 0) return 0;
-    // Sized by the row count alone (not by the test hook that moves groups of
-    // 33..64 rows to the swap-AB kernel, which needs less).
+    // Sized by the row count alone (the test hook that moves groups of 33..64
+    // rows to the swap-AB kernel only lowers the need). Up to 32 rows the
+    // swap-AB kernel quantizes the queries itself and writes the output directly
+    // from one split.
     const int rows = (Hq / Hkv) * nq;
     if (rows < qk4v8::kGqaMinRows) return num_splits == 1 ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits);
     // Larger groups: the queries are quantized into the front of the workspace
@@ -523,19 +525,34 @@ int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_
         return qk4v8_decode_merge(workspace, workspace_bytes, B, Hq, nq, used, out, lse, stream);
     }
     // More than 32 query rows per KV head: quantize Q into the front of the
-    // workspace for the GQA decode kernel or the 128-row kernel.
+    // workspace (capacity 128 tokens). The GQA decode kernel (up to 64 rows)
+    // reads only the nq rows of each head, so only those are written; the
+    // 128-row kernel gets the whole capacity.
     uint8_t *qc = static_cast<uint8_t *>(workspace);
     uint8_t *qs = qc + qk4v8_mxfp4_codes_bytes(B, Hq, 128);
     uint8_t *rest = qs + qk4v8_scales_bytes(B, Hq, 128);
     const size_t rest_bytes = workspace_bytes - static_cast<size_t>(rest - qc);
-    int st = qk4v8_quantize_qk(q, B, nq, Hq, 128, q_stride_b, q_stride_t, q_stride_h, nullptr, 128, qc, qs, stream);
-    if (st) return st;
+    const bool gqa = gqa_rows(Hq, Hkv, nq);
+    int st;
+    if (gqa) {
+        if (!aligned16(q) || q_stride_b % 8 || q_stride_t % 8 || q_stride_h % 8 || q_stride_b < 0 || q_stride_t < 0 ||
+            q_stride_h < 0)
+            return set_error(QK4V8_ERR_INVALID_ARG, "bf16 Q must be 16-byte aligned with strides of whole 8-element "
+                                                    "(16-byte) units");
+        if ((st = check_device())) return st;
+        cudaError_t e = qk4v8::launch_quantize_qk(q, B, nq, Hq, q_stride_b, q_stride_t, q_stride_h, nullptr, 128, qc,
+                                                  qs, s, /*pad_to_cap=*/false);
+        if (e != cudaSuccess) return cuda_error(e, "quantize (decode queries) launch");
+    } else if ((st = qk4v8_quantize_qk(q, B, nq, Hq, 128, q_stride_b, q_stride_t, q_stride_h, nullptr, 128, qc, qs,
+                                       stream))) {
+        return st;
+    }
     dq.codes = qc;
     dq.scales = qs;
     dq.cap = 128;
     st = decode_splitkv(dq, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
-                        causal_in_block, softmax_scale, splits, rest, rest_bytes, out, lse, dev_status, s, &used,
-                        &direct);
+                        causal_in_block, softmax_scale, splits, rest, rest_bytes, gqa ? out : nullptr,
+                        gqa ? lse : nullptr, dev_status, s, &used, &direct);
     if (st || direct) return st;
     return qk4v8_decode_merge(rest, rest_bytes, B, Hq, nq, used, out, lse, stream);
 }

@@ -32,9 +32,9 @@
 // scale their lanes by the same 2^-E, agreed through a two-way exchange, and
 // pass E on to the other set.
 //
-// Warp roles (352 threads): warps 0..7 softmax and epilogue, warp 8 TMA
-// producer of K (it also stages the packed Q rows of each unit), warp 9 TMEM
-// allocator and single-thread tcgen05 issuer, warp 10 TMA producer of V. Splits write fp32 partials
+// Warp roles (384 threads): warps 0..7 softmax and epilogue, warp 8 TMA
+// producer of K, warp 9 TMEM allocator and single-thread tcgen05 issuer,
+// warp 10 TMA producer of V, warp 11 stages each unit's packed query rows. Splits write fp32 partials
 // (O / l, log2-sum-exp) for the merge kernel; one split writes bf16 directly.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -54,10 +54,11 @@ namespace {
 constexpr int kGdKStages = 6;             // K tiles in flight (freed when the pair's QK^T completes)
 constexpr int kGdVStages = 4;             // V tiles in flight (freed when the pair's P V completes)
 constexpr int kGdSoftmaxWarps = 8;
-constexpr int kGdThreads = 32 * kGdSoftmaxWarps + 96;
-constexpr int kGdProducerWarp = 8;   // Q and K
+constexpr int kGdThreads = 32 * kGdSoftmaxWarps + 128;
+constexpr int kGdProducerWarp = 8;   // K
 constexpr int kGdMmaWarp = 9;
 constexpr int kGdVProducerWarp = 10;
+constexpr int kGdQWarp = 11;
 constexpr float kGdTau = 8.0f;             // m_w moves once a score passes it by 2^8
 constexpr int kGdEMax = 64;                // largest offset e before O is rescaled
 constexpr float kGdMaxMove = 16777216.0f;  // cap on one move of m_w, keeps it an exact integer
@@ -232,10 +233,10 @@ __global__ void __launch_bounds__(kGdThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kGdProducerWarp) {
-        // ---------------------------------------------------------- Q and K producer
+        // ------------------------------------------------------------- K producer
         if (lane == 0) prefetch_tensormap(&tmap_k);
         const int nblk = p.kv_cap / 128;
-        int g = 0, c = 0;  // tiles and units so far (units with at least one tile)
+        int g = 0;  // tiles so far
         int gk_issued = 0;
         bool ok = true;
         for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
@@ -243,58 +244,6 @@ __global__ void __launch_bounds__(kGdThreads, 1)
             const int T = u.T;
             if (T <= 0) continue;
             const int kvh = u.b * p.Hkv + u.h_kv;
-            // Q rows of the unit (packed MXFP4) into buffer c & 1: codes to rows n and
-            // 128 + n (64-byte swizzle: chunk j of row n at j ^ ((n / 2) % 4)), the
-            // row's scale word to atom rows n and 64 + n. The MMA warp frees the
-            // buffer after the unit's last QK^T.
-            const int qb = c & 1;
-            ok = __all_sync(0xffffffffu, wait_bar(&q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status));
-            if (!ok) break;
-            uint4 qv[8];
-            uint32_t sv[2];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int idx = lane + 32 * i, n = idx >> 2, j = idx & 3;
-                qv[i] = make_uint4(0, 0, 0, 0);
-                if (n < R) {
-                    const int h = u.h_kv * p.G + n / nq, t = n % nq;
-                    qv[i] = *reinterpret_cast<const uint4 *>(
-                        p.q_codes + ((static_cast<int64_t>(u.b) * p.Hq + h) * p.q_cap + t) * 64 + j * 16);
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int n = lane + 32 * i;
-                sv[i] = 0;
-                if (n < R) {
-                    const int h = u.h_kv * p.G + n / nq, t = n % nq;
-                    sv[i] = *reinterpret_cast<const uint32_t *>(
-                        p.q_scales + ((static_cast<int64_t>(u.b) * p.Hq + h) * (p.q_cap / 128) + t / 128) * 512 +
-                        (t & 31) * 16 + ((t & 127) >> 5) * 4);
-                }
-            }
-            uint8_t *qbuf = smem + S::kQ + qb * S::kQBytes;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int idx = lane + 32 * i, n = idx >> 2, j = idx & 3;
-                if (n < R) {
-                    const int cofs = (j ^ ((n >> 1) & 3)) << 4;
-                    *reinterpret_cast<uint4 *>(qbuf + n * 64 + cofs) = qv[i];
-                    *reinterpret_cast<uint4 *>(qbuf + (128 + n) * 64 + cofs) = qv[i];
-                }
-            }
-            uint8_t *sfq = smem + S::kSfQ + qb * 512;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int n = lane + 32 * i;
-                if (n < R) {
-                    *reinterpret_cast<uint32_t *>(sfq + (n & 31) * 16 + (n >> 5) * 4) = sv[i];
-                    *reinterpret_cast<uint32_t *>(sfq + (n & 31) * 16 + ((n >> 5) + 2) * 4) = sv[i];
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && !(p.test_stall && c == 0)) mbar_arrive(&q_full[qb]);
             // K tiles of the unit: the K ring frees as soon as the pair's QK^T
             // completes, so K runs up to kGdKStages tiles ahead of the tensor core.
             for (int it = 0; it < T && ok; ++it) {
@@ -312,7 +261,6 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                 gk_issued = gk + 1;
             }
             g += T;
-            ++c;
         }
         // Let every issued copy land before the CTA can retire.
         if (lane == 0) {
@@ -321,6 +269,69 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                 while (!mbar_try_wait(&k_full[gk % kGdKStages], (gk / kGdKStages) & 1))
                     if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
             }
+        }
+    } else if (warp == kGdQWarp) {
+        // ------------------------------------------------------------ Q staging
+        // The packed query rows of each unit into Q buffer c & 1, while earlier
+        // units run: codes to rows n and 128 + n (64-byte swizzle: chunk j of
+        // row n at j ^ ((n / 2) % 4)), the row's scale word to atom rows n and
+        // 64 + n. The MMA warp frees the buffer after the unit's last QK^T.
+        int c = 0;  // units so far (units with at least one tile)
+        bool ok = true;
+        for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
+            const GdUnit u = gd_unit(p, un);
+            if (u.T <= 0) continue;
+            const int qb = c & 1;
+            ok = __all_sync(0xffffffffu, wait_bar(&q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status));
+            if (!ok) break;
+            uint8_t *qbuf = smem + S::kQ + qb * S::kQBytes;
+            uint8_t *sfq = smem + S::kSfQ + qb * 512;
+            {
+                uint4 qv[8];
+                uint32_t sv[2];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int idx = lane + 32 * i, n = idx >> 2, jj = idx & 3;
+                    qv[i] = make_uint4(0, 0, 0, 0);
+                    if (n < R) {
+                        const int h = u.h_kv * p.G + n / nq, t = n % nq;
+                        qv[i] = *reinterpret_cast<const uint4 *>(
+                            p.q_codes + ((static_cast<int64_t>(u.b) * p.Hq + h) * p.q_cap + t) * 64 + jj * 16);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int n = lane + 32 * i;
+                    sv[i] = 0;
+                    if (n < R) {
+                        const int h = u.h_kv * p.G + n / nq, t = n % nq;
+                        sv[i] = *reinterpret_cast<const uint32_t *>(
+                            p.q_scales + ((static_cast<int64_t>(u.b) * p.Hq + h) * (p.q_cap / 128) + t / 128) * 512 +
+                            (t & 31) * 16 + ((t & 127) >> 5) * 4);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int idx = lane + 32 * i, n = idx >> 2, jj = idx & 3;
+                    if (n < R) {
+                        const int cofs = (jj ^ ((n >> 1) & 3)) << 4;
+                        *reinterpret_cast<uint4 *>(qbuf + n * 64 + cofs) = qv[i];
+                        *reinterpret_cast<uint4 *>(qbuf + (128 + n) * 64 + cofs) = qv[i];
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int n = lane + 32 * i;
+                    if (n < R) {
+                        *reinterpret_cast<uint32_t *>(sfq + (n & 31) * 16 + (n >> 5) * 4) = sv[i];
+                        *reinterpret_cast<uint32_t *>(sfq + (n & 31) * 16 + ((n >> 5) + 2) * 4) = sv[i];
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && !(p.test_stall && c == 0)) mbar_arrive(&q_full[qb]);
+            ++c;
         }
     } else if (warp == kGdVProducerWarp) {
         // -------------------------------------------------------------- V producer

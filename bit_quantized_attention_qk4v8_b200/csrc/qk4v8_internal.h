@@ -43,9 +43,11 @@ struct AttnParams {
     float *test_dump_s;       // test hook: CTA 0 writes its first raw score tile [128 lanes][128 keys]
 };
 
+// pad_to_cap: write all `cap` token rows of each sequence (rows past the valid
+// length get zero codes and scales); otherwise only the S input rows.
 cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                                const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
-                               cudaStream_t stream);
+                               cudaStream_t stream, bool pad_to_cap = true);
 cudaError_t launch_quantize_v(const void *v, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                               const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
                               cudaStream_t stream);

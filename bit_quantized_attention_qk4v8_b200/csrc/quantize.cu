@@ -22,13 +22,16 @@ namespace qk4v8 {
 
 // 16 lanes per token row (128 channels), 8 channels per lane, 4 lanes per group
 // of 32. Rows are visited in input order (b, t, h) so loads are contiguous.
+// Tokens 0 .. row_len-1 of each sequence are visited: row_len = cap writes the
+// whole capacity (zero codes and scales past the valid length), row_len = S
+// only the rows of the input.
 __global__ void __launch_bounds__(256) quantize_qk_kernel(const __nv_bfloat16 *__restrict__ x, int B, int S, int H,
                                                           int64_t sb, int64_t ss, int64_t sh,
                                                           const int32_t *__restrict__ seqlens, int cap,
-                                                          uint8_t *__restrict__ codes,
+                                                          int row_len, uint8_t *__restrict__ codes,
                                                           uint8_t *__restrict__ scales) {
     const int sub = threadIdx.x & 15;  // lane within the row
-    const int64_t n_rows = static_cast<int64_t>(B) * cap * H;
+    const int64_t n_rows = static_cast<int64_t>(B) * row_len * H;
     const int64_t row_step = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 4);
     // The loop bound is taken per warp (two rows) so every lane reaches the shuffles.
     for (int64_t base = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 4) + ((threadIdx.x >> 5) << 1);
@@ -38,8 +41,8 @@ __global__ void __launch_bounds__(256) quantize_qk_kernel(const __nv_bfloat16 *_
         const int64_t row = in_range ? row_raw : base;
         const int h = static_cast<int>(row % H);
         const int64_t bt = row / H;
-        const int t = static_cast<int>(bt % cap);
-        const int b = static_cast<int>(bt / cap);
+        const int t = static_cast<int>(bt % row_len);
+        const int b = static_cast<int>(bt / row_len);
         int valid_len = S;
         if (seqlens) {
             int L = seqlens[b];
@@ -151,15 +154,16 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__
 
 cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                                const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
-                               cudaStream_t stream) {
-    const int64_t rows = static_cast<int64_t>(B) * cap * H;
+                               cudaStream_t stream, bool pad_to_cap) {
+    const int row_len = pad_to_cap ? cap : S;
+    const int64_t rows = static_cast<int64_t>(B) * row_len * H;
     const int rows_per_cta = 256 / 16;
     int64_t grid = (rows + rows_per_cta - 1) / rows_per_cta;
     const int64_t max_grid = 148 * 16;
     if (grid > max_grid) grid = max_grid;
     if (grid < 1) grid = 1;
     quantize_qk_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(x), B, S, H, sb, ss, sh, seqlens, cap, codes, scales);
+        static_cast<const __nv_bfloat16 *>(x), B, S, H, sb, ss, sh, seqlens, cap, row_len, codes, scales);
     return cudaGetLastError();
 }
 
