@@ -267,7 +267,9 @@ int qk4v8_test_prefill_stage_qk(const uint8_t *q_codes, const uint8_t *q_scales,
 size_t qk4v8_decode_workspace_bytes(int B, int Hq, int nq, int num_splits) {
     if (B <= 0 || Hq <= 0 || nq <= 0 || num_splits <= 0) return 0;
     const size_t rows = static_cast<size_t>(B) * Hq * nq * num_splits;
-    return rows * 128 * sizeof(float) + rows * sizeof(float);
+    // Split partials O [rows][128] and log2-sum-exp [rows], then the piece count
+    // of each (sequence, head), which the GQA decode kernel records for its merge.
+    return rows * 128 * sizeof(float) + rows * sizeof(float) + static_cast<size_t>(B) * Hq * sizeof(int32_t);
 }
 
 int qk4v8_decode_default_splits(int B, int Hq, int Hkv, int nq, int max_seqlen) {
@@ -361,9 +363,12 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
                          qk4v8::kGqaMinRows);
     if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
     const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen);
-    const bool direct_out = out && splits == 1 && (swap_ab_rows(Hq, Hkv, nq) || gqa_rows(Hq, Hkv, nq));
+    // Direct output: the swap-AB kernel with one split, and the GQA decode kernel
+    // always (with splits, its own merge launch finishes the cut sequences).
+    const bool gqa = gqa_rows(Hq, Hkv, nq);
+    const bool direct_out = out && ((splits == 1 && swap_ab_rows(Hq, Hkv, nq)) || gqa);
     if (out && !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
-    const size_t need = direct_out ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
+    const size_t need = (direct_out && splits == 1) ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
     if (need && (!workspace || !aligned16(workspace) || workspace_bytes < need))
         return set_error(QK4V8_ERR_INVALID_ARG, "workspace must be 16-byte aligned and >= %zu bytes", need);
     if ((st = check_device())) return st;
@@ -399,10 +404,12 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
         p.direct_out = 1;
         p.out = static_cast<__nv_bfloat16 *>(out);
         p.lse = lse;
-    } else {
+    }
+    if (need) {
         const size_t rows = static_cast<size_t>(B) * Hq * nq * splits;
         p.ws_o = static_cast<float *>(workspace);
         p.ws_lse = p.ws_o + rows * 128;
+        p.piece_counts = reinterpret_cast<int32_t *>(p.ws_lse + rows);
     }
     p.status = dev_status;
     p.test_stall = g_test_stall;

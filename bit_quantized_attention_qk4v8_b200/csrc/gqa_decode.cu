@@ -90,8 +90,9 @@ struct GdSmem {
     // hs [pair parity][row group]; mo [row group]; ue [row group];
     // xb [set][row group][tile half][parity].
     static constexpr int kNumBars = 2 * kGdKStages + 2 * kGdVStages + 4 + 1 + 8 + 3 + 4 + 2 + 2 + 16;
-    static constexpr int kMisc = kBar + kNumBars * 8;
-    static constexpr int kUsed = kMisc + 16;
+    static constexpr int kMisc = kBar + kNumBars * 8;    // TMEM address, abort flag
+    static constexpr int kSched = kMisc + 16;            // GdSched
+    static constexpr int kUsed = kSched + 64;
     static constexpr int kBytes = kUsed + 1024;  // slack for aligning the base
 };
 static_assert(GdSmem::kQBytes % 1024 == 0 && GdSmem::kK % 1024 == 0 && GdSmem::kV % 1024 == 0 &&
@@ -117,22 +118,211 @@ constexpr uint32_t kGdIdQK = gd_idesc(1u, 128);             // E2M1 x E2M1, N = 
 constexpr uint32_t kGdIdPV = gd_idesc(0u, GdSmem::kVRows);  // E4M3 x E4M3, N = 144
 __device__ __forceinline__ uint32_t gd_sf_id(uint32_t idesc, uint32_t id) { return idesc | (id << 29) | (id << 4); }
 
+// One piece of work: key tiles [tile_begin, tile_begin + T) of the sequence
+// (b, h_kv). `whole` when the piece is the whole sequence; otherwise it is
+// piece `slot` of `n_pieces`, written as a partial (O / l, log2-sum-exp).
 struct GdUnit {
-    int b, h_kv, split, L, tile_begin, T;
+    int b, h_kv, L, tile_begin, T, slot, n_pieces;
+    bool whole;
 };
 
-// Work unit `idx`: one (sequence, KV head, key split), splits innermost.
-__device__ __forceinline__ GdUnit gd_unit(const AttnParams &p, int idx) {
-    GdUnit u;
-    u.split = idx % p.num_splits;
-    const int rem = idx / p.num_splits;
-    u.h_kv = rem % p.Hkv;
-    u.b = rem / p.Hkv;
-    u.L = imax(0, imin(p.seqlens[u.b], p.kv_cap));
-    const int n_tiles = (u.L + 127) / 128;
-    u.tile_begin = u.split * p.split_tiles;
-    u.T = imax(0, imin(u.tile_begin + p.split_tiles, n_tiles) - u.tile_begin);
-    return u;
+__device__ __forceinline__ int gd_tiles(const AttnParams &p, int b) {
+    return (imax(0, imin(p.seqlens[b], p.kv_cap)) + 127) / 128;
+}
+
+// Schedule of one CTA, computed once at the start.
+//   Fixed splits: units (sequence, split) blockIdx.x, +grid, ... with
+//   split_tiles key tiles each.
+//   Balanced ("stream-K"): the key tiles of all sequences in (b, h_kv) order
+//   form one list of W tiles; CTA i takes tiles [i W / G, (i+1) W / G), so every
+//   CTA gets the same work up to one tile. A sequence cut by a range boundary
+//   becomes pieces in consecutive CTAs. Used for the direct-output call when
+//   every range is at least one tile and no sequence can be cut into more
+//   pieces than there are partial slots (num_splits). A CTA runs the first and
+//   the last sequence of its range (the ones that may be cut) before the ones
+//   in between, so that cut sequences are complete, and merged, early.
+struct GdSched {
+    int streamk;
+    int b0, h0, bL, hL;   // first and last sequence of this CTA's range
+    long long W, x0, x1;  // tile list length and this CTA's range [x0, x1)
+    long long P0, PL;     // first tiles of those sequences in the list
+};
+
+// CTA holding tile x of the balanced list: the largest i with floor(i W / G) <= x.
+__device__ __forceinline__ int gd_cta_of(long long x, long long W, int G) {
+    return static_cast<int>(((x + 1) * G - 1) / W);
+}
+
+// Finds the first sequence (in (b, h) order) that is non-empty and ends past
+// tile x, or (allow_empty) is empty and starts at or past x. One full warp.
+// Returns false if there is none.
+__device__ __noinline__ bool gd_find(const AttnParams &p, long long x, bool allow_empty, int &b_out, int &h_out,
+                                     long long &P_out) {
+    const int lane = threadIdx.x & 31;
+    long long P = 0;  // first tile of batch entry `base`
+    for (int base = 0; base < p.B; base += 32) {
+        const int b = base + lane;
+        const int t = b < p.B ? gd_tiles(p, b) : 0;
+        long long incl = static_cast<long long>(t) * p.Hkv;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const long long Pb = P + incl - static_cast<long long>(t) * p.Hkv;
+        const bool hit =
+            b < p.B && ((t > 0 && Pb + static_cast<long long>(t) * p.Hkv > x) || (allow_empty && t == 0 && Pb >= x));
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (m) {
+            const int src = __ffs(m) - 1;
+            const int tb = __shfl_sync(0xffffffffu, t, src);
+            const long long pb = __shfl_sync(0xffffffffu, Pb, src);
+            b_out = base + src;
+            h_out = (tb > 0 && x > pb) ? static_cast<int>((x - pb) / tb) : 0;
+            P_out = pb + static_cast<long long>(h_out) * tb;
+            return true;
+        }
+        P += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    return false;
+}
+
+// Whether the balanced schedule applies: at least one tile per CTA, and no
+// sequence cut into more pieces than the num_splits partial slots (a sequence
+// of t tiles meets at most ceil(t / range) + 1 of the ranges).
+__device__ __forceinline__ bool gd_balanced(const AttnParams &p, long long W, int tmax, int G) {
+    const long long range = W / G;
+    return p.num_splits >= 2 && range >= 1 && (tmax + range - 1) / range + 1 <= p.num_splits;
+}
+
+// Computed by one full warp: per-batch tile counts scanned 32 at a time.
+__device__ __noinline__ void gd_schedule(const AttnParams &p, GdSched &sc) {
+    const int lane = threadIdx.x & 31;
+    const int G = gridDim.x, i = blockIdx.x;
+    long long W = 0;
+    int tmax = 0;
+    for (int base = 0; base < p.B; base += 32) {
+        const int b = base + lane;
+        const int t = b < p.B ? gd_tiles(p, b) : 0;
+        tmax = max(tmax, __reduce_max_sync(0xffffffffu, t));
+        W += static_cast<long long>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(t))) * p.Hkv;
+    }
+    sc.W = W;
+    sc.streamk = 0;
+    sc.b0 = sc.h0 = sc.bL = sc.hL = 0;
+    sc.P0 = sc.PL = 0;
+    sc.x0 = sc.x1 = 0;
+    if (!p.direct_out || !gd_balanced(p, W, tmax, G)) return;
+    sc.streamk = 1;
+    sc.x0 = static_cast<long long>(i) * W / G;
+    const long long x1 = static_cast<long long>(i + 1) * W / G;
+    // The last CTA also takes the empty sequences that sit at the end of the list.
+    sc.x1 = i == G - 1 ? W + 1 : x1;
+    // The first sequence of the range (it may be empty, sitting at x0) and the
+    // sequence of its last tile.
+    if (!gd_find(p, sc.x0, true, sc.b0, sc.h0, sc.P0)) sc.b0 = p.B;
+    if (!gd_find(p, x1 - 1, false, sc.bL, sc.hL, sc.PL)) {
+        sc.bL = sc.b0;
+        sc.hL = sc.h0;
+        sc.PL = sc.P0;
+    }
+}
+
+// Walks this CTA's units in order; every role warp runs its own copy.
+struct GdIter {
+    int un;         // fixed splits: next unit index
+    int phase;      // balanced: 0 first sequence, 1 last, 2 those in between, 3 those after the last
+    int b, h, tb;   // balanced: next sequence of phases 2 and 3, and its tile count
+    long long P;    // balanced: its first tile in the list
+};
+
+__device__ __forceinline__ void gd_begin(const AttnParams &p, const GdSched &sc, GdIter &it) {
+    it.un = blockIdx.x;
+    it.phase = 0;
+    it.b = it.h = it.tb = 0;
+    it.P = 0;
+}
+
+// Steps (b, h, P) to the next sequence in (b, h) order.
+__device__ __forceinline__ void gd_step(const AttnParams &p, int &b, int &h, long long &P, int &tb) {
+    P += tb;
+    if (++h >= p.Hkv) {
+        h = 0;
+        ++b;
+        tb = b < p.B ? gd_tiles(p, b) : 0;
+    }
+}
+
+// The piece of sequence (b, h), first tile Ps, that lies in this CTA's range.
+__device__ __forceinline__ void gd_piece(const AttnParams &p, const GdSched &sc, int b, int h, long long Ps,
+                                         GdUnit &u) {
+    const int Ts = gd_tiles(p, b);
+    const long long t0 = Ps < sc.x0 ? sc.x0 - Ps : 0;
+    const long long t1 = Ps + Ts > sc.x1 ? sc.x1 - Ps : Ts;
+    u.b = b;
+    u.h_kv = h;
+    u.L = imax(0, imin(p.seqlens[b], p.kv_cap));
+    u.tile_begin = static_cast<int>(t0);
+    u.T = Ts > 0 ? static_cast<int>(t1 - t0) : 0;
+    u.whole = t0 == 0 && t1 == Ts;
+    if (Ts > 0) {
+        const int first = gd_cta_of(Ps, sc.W, gridDim.x);
+        u.slot = static_cast<int>(blockIdx.x) - first;
+        u.n_pieces = gd_cta_of(Ps + Ts - 1, sc.W, gridDim.x) - first + 1;
+    } else {
+        u.slot = 0;
+        u.n_pieces = 1;
+    }
+}
+
+__device__ __forceinline__ bool gd_next(const AttnParams &p, const GdSched &sc, GdIter &it, GdUnit &u) {
+    if (!sc.streamk) {
+        if (it.un >= p.B * p.Hkv * p.num_splits) return false;
+        const int idx = it.un;
+        it.un += gridDim.x;
+        const int split = idx % p.num_splits;
+        const int rem = idx / p.num_splits;
+        u.h_kv = rem % p.Hkv;
+        u.b = rem / p.Hkv;
+        u.L = imax(0, imin(p.seqlens[u.b], p.kv_cap));
+        const int n_tiles = (u.L + 127) / 128;
+        u.tile_begin = split * p.split_tiles;
+        u.T = imax(0, imin(u.tile_begin + p.split_tiles, n_tiles) - u.tile_begin);
+        u.slot = split;
+        u.n_pieces = p.num_splits;
+        u.whole = p.num_splits == 1;
+        return true;
+    }
+    if (sc.b0 >= p.B) return false;
+    const bool last_differs = sc.bL != sc.b0 || sc.hL != sc.h0;
+    if (it.phase == 0) {
+        gd_piece(p, sc, sc.b0, sc.h0, sc.P0, u);
+        it.phase = last_differs ? 1 : 3;
+        it.b = sc.b0;
+        it.h = sc.h0;
+        it.P = sc.P0;
+        it.tb = gd_tiles(p, sc.b0);
+        gd_step(p, it.b, it.h, it.P, it.tb);
+        return true;
+    }
+    if (it.phase == 1) {
+        gd_piece(p, sc, sc.bL, sc.hL, sc.PL, u);
+        it.phase = 2;
+        return true;
+    }
+    if (it.phase == 2) {
+        if (it.b != sc.bL || it.h != sc.hL) {
+            gd_piece(p, sc, it.b, it.h, it.P, u);
+            gd_step(p, it.b, it.h, it.P, it.tb);
+            return true;
+        }
+        it.phase = 3;
+        gd_step(p, it.b, it.h, it.P, it.tb);  // past the last sequence
+    }
+    if (it.b >= p.B || it.P >= sc.x1) return false;
+    gd_piece(p, sc, it.b, it.h, it.P, u);
+    gd_step(p, it.b, it.h, it.P, it.tb);
+    return true;
 }
 
 }  // namespace
@@ -145,7 +335,6 @@ __global__ void __launch_bounds__(kGdThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_units = p.B * p.Hkv * p.num_splits;
     const int nq = p.Sq;
     const int R = p.G * nq;  // query rows of a unit, 33..64
 
@@ -170,6 +359,7 @@ __global__ void __launch_bounds__(kGdThreads, 1)
     uint64_t *xb_bar = ue_bar + 2;  // [set][row group][tile half][parity]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kMisc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + S::kMisc + 4);
+    GdSched *sched = reinterpret_cast<GdSched *>(smem + S::kSched);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGdKStages; ++s) {
@@ -207,6 +397,7 @@ __global__ void __launch_bounds__(kGdThreads, 1)
         tmem_alloc(tmem_slot, kGdTmemCols);
         tmem_relinquish();
     }
+    if (warp == 0) gd_schedule(p, *sched);
     // Both Q buffers and their scale atoms start at zero: rows R..63 and 64..127
     // (and 128+R..191) are never written again, and zero codes with zero
     // scales contribute nothing.
@@ -231,6 +422,7 @@ __global__ void __launch_bounds__(kGdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const GdSched gs = *sched;
 
     if (warp == kGdProducerWarp) {
         // ------------------------------------------------------------- K producer
@@ -239,8 +431,10 @@ __global__ void __launch_bounds__(kGdThreads, 1)
         int g = 0;  // tiles so far
         int gk_issued = 0;
         bool ok = true;
-        for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
-            const GdUnit u = gd_unit(p, un);
+        GdIter it;
+        gd_begin(p, gs, it);
+        GdUnit u;
+        while (ok && gd_next(p, gs, it, u)) {
             const int T = u.T;
             if (T <= 0) continue;
             const int kvh = u.b * p.Hkv + u.h_kv;
@@ -276,63 +470,65 @@ __global__ void __launch_bounds__(kGdThreads, 1)
         // units run: codes to rows n and 128 + n (64-byte swizzle: chunk j of
         // row n at j ^ ((n / 2) % 4)), the row's scale word to atom rows n and
         // 64 + n. The MMA warp frees the buffer after the unit's last QK^T.
-        int c = 0;  // units so far (units with at least one tile)
+        int c = 0;  // units staged
         bool ok = true;
-        for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
-            const GdUnit u = gd_unit(p, un);
-            if (u.T <= 0) continue;
+        auto stage_q = [&](const GdUnit &v) -> bool {
             const int qb = c & 1;
-            ok = __all_sync(0xffffffffu, wait_bar(&q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status));
-            if (!ok) break;
+            if (!__all_sync(0xffffffffu, wait_bar(&q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status)))
+                return false;
             uint8_t *qbuf = smem + S::kQ + qb * S::kQBytes;
             uint8_t *sfq = smem + S::kSfQ + qb * 512;
-            {
-                uint4 qv[8];
-                uint32_t sv[2];
+            uint4 qv[8];
+            uint32_t sv[2];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int idx = lane + 32 * i, n = idx >> 2, jj = idx & 3;
-                    qv[i] = make_uint4(0, 0, 0, 0);
-                    if (n < R) {
-                        const int h = u.h_kv * p.G + n / nq, t = n % nq;
-                        qv[i] = *reinterpret_cast<const uint4 *>(
-                            p.q_codes + ((static_cast<int64_t>(u.b) * p.Hq + h) * p.q_cap + t) * 64 + jj * 16);
-                    }
+            for (int i = 0; i < 8; ++i) {
+                const int idx = lane + 32 * i, n = idx >> 2, jj = idx & 3;
+                qv[i] = make_uint4(0, 0, 0, 0);
+                if (n < R) {
+                    const int h = v.h_kv * p.G + n / nq, t = n % nq;
+                    qv[i] = *reinterpret_cast<const uint4 *>(
+                        p.q_codes + ((static_cast<int64_t>(v.b) * p.Hq + h) * p.q_cap + t) * 64 + jj * 16);
                 }
+            }
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int n = lane + 32 * i;
-                    sv[i] = 0;
-                    if (n < R) {
-                        const int h = u.h_kv * p.G + n / nq, t = n % nq;
-                        sv[i] = *reinterpret_cast<const uint32_t *>(
-                            p.q_scales + ((static_cast<int64_t>(u.b) * p.Hq + h) * (p.q_cap / 128) + t / 128) * 512 +
-                            (t & 31) * 16 + ((t & 127) >> 5) * 4);
-                    }
+            for (int i = 0; i < 2; ++i) {
+                const int n = lane + 32 * i;
+                sv[i] = 0;
+                if (n < R) {
+                    const int h = v.h_kv * p.G + n / nq, t = n % nq;
+                    sv[i] = *reinterpret_cast<const uint32_t *>(
+                        p.q_scales + ((static_cast<int64_t>(v.b) * p.Hq + h) * (p.q_cap / 128) + t / 128) * 512 +
+                        (t & 31) * 16 + ((t & 127) >> 5) * 4);
                 }
+            }
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int idx = lane + 32 * i, n = idx >> 2, jj = idx & 3;
-                    if (n < R) {
-                        const int cofs = (jj ^ ((n >> 1) & 3)) << 4;
-                        *reinterpret_cast<uint4 *>(qbuf + n * 64 + cofs) = qv[i];
-                        *reinterpret_cast<uint4 *>(qbuf + (128 + n) * 64 + cofs) = qv[i];
-                    }
+            for (int i = 0; i < 8; ++i) {
+                const int idx = lane + 32 * i, n = idx >> 2, jj = idx & 3;
+                if (n < R) {
+                    const int cofs = (jj ^ ((n >> 1) & 3)) << 4;
+                    *reinterpret_cast<uint4 *>(qbuf + n * 64 + cofs) = qv[i];
+                    *reinterpret_cast<uint4 *>(qbuf + (128 + n) * 64 + cofs) = qv[i];
                 }
+            }
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int n = lane + 32 * i;
-                    if (n < R) {
-                        *reinterpret_cast<uint32_t *>(sfq + (n & 31) * 16 + (n >> 5) * 4) = sv[i];
-                        *reinterpret_cast<uint32_t *>(sfq + (n & 31) * 16 + ((n >> 5) + 2) * 4) = sv[i];
-                    }
+            for (int i = 0; i < 2; ++i) {
+                const int n = lane + 32 * i;
+                if (n < R) {
+                    *reinterpret_cast<uint32_t *>(sfq + (n & 31) * 16 + (n >> 5) * 4) = sv[i];
+                    *reinterpret_cast<uint32_t *>(sfq + (n & 31) * 16 + ((n >> 5) + 2) * 4) = sv[i];
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0 && !(p.test_stall && c == 0)) mbar_arrive(&q_full[qb]);
             ++c;
-        }
+            return true;
+        };
+        GdIter it;
+        gd_begin(p, gs, it);
+        GdUnit u;
+        while (ok && gd_next(p, gs, it, u))
+            if (u.T > 0) ok = stage_q(u);
     } else if (warp == kGdVProducerWarp) {
         // -------------------------------------------------------------- V producer
         // V tiles on their own warp, so that a V stage waiting for its P V never
@@ -341,8 +537,10 @@ __global__ void __launch_bounds__(kGdThreads, 1)
         const int nblk = p.kv_cap / 128;
         int g = 0, gv_issued = 0;
         bool ok = true;
-        for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
-            const GdUnit u = gd_unit(p, un);
+        GdIter it;
+        gd_begin(p, gs, it);
+        GdUnit u;
+        while (ok && gd_next(p, gs, it, u)) {
             const int T = u.T;
             if (T <= 0) continue;
             const int kvh = u.b * p.Hkv + u.h_kv;
@@ -423,8 +621,10 @@ __global__ void __launch_bounds__(kGdThreads, 1)
         __syncwarp();
         bool ok = true;
         int g = 0, gp0 = 0, c = 0, n_patch = 0;  // tiles, pairs and units so far
-        for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
-            const GdUnit u = gd_unit(p, un);
+        GdIter it;
+        gd_begin(p, gs, it);
+        GdUnit u;
+        while (ok && gd_next(p, gs, it, u)) {
             const int T = u.T;
             if (T <= 0) continue;
             const int NP = (T + 1) / 2;
@@ -574,28 +774,58 @@ __global__ void __launch_bounds__(kGdThreads, 1)
             ++nx;
             return w;
         };
-        for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
-            const GdUnit u = gd_unit(p, un);
-            const int T = u.T;
-            const int h_q = u.h_kv * p.G + r / nq, tq = r % nq;
-            const int64_t orow = (static_cast<int64_t>(u.b) * p.Hq + h_q) * nq + tq;  // [b][h][t]
-            if (T <= 0) {
-                // A split with no key: O = 0 and lse = -inf for every query row.
-                if (row_valid) {
-                    if (p.direct_out) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(
-                            p.out + ((static_cast<int64_t>(u.b) * nq + tq) * p.Hq + h_q) * 128 + c_lo);
+        // Final bf16 columns c_lo .. c_lo+31 of row r (and, for one thread of the
+        // row, its natural-log lse) from O / l and the log2-sum-exp.
+        auto write_out = [&](const GdUnit &v, const float (&o)[32], float lse2) {
+            const int h_q = v.h_kv * p.G + r / nq, tq = r % nq;
+            uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((static_cast<int64_t>(v.b) * nq + tq) * p.Hq + h_q) * 128 +
+                                                   c_lo);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(0, 0, 0, 0);
-                        if (c_lo == 0 && p.lse) p.lse[orow] = -INFINITY;
-                    } else {
-                        const int64_t prow = orow * p.num_splits + u.split;
-                        float4 *dst = reinterpret_cast<float4 *>(p.ws_o + prow * 128 + c_lo);
+            for (int q = 0; q < 4; ++q) {
+                uint32_t w[4];
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (c_lo == 0) p.ws_lse[prow] = -INFINITY;
-                    }
+                for (int kk = 0; kk < 4; ++kk) {
+                    const __nv_bfloat162 v2 = __floats2bfloat162_rn(o[8 * q + 2 * kk], o[8 * q + 2 * kk + 1]);
+                    w[kk] = *reinterpret_cast<const uint32_t *>(&v2);
                 }
+                dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            if (c_lo == 0 && p.lse)
+                p.lse[(static_cast<int64_t>(v.b) * p.Hq + h_q) * nq + tq] =
+                    lse2 > -INFINITY ? lse2 * 0.6931471805599453f : -INFINITY;
+        };
+        // Finishes unit v for this thread's columns: in the direct-output call a
+        // whole sequence goes straight to the output; otherwise the piece is
+        // written as the fp32 partial of its slot, for the merge kernel.
+        auto finish = [&](const GdUnit &v, const float (&o)[32], float lse2) {
+            // The merge launch reads, per sequence, how many pieces to merge: 0 when
+            // the sequence was written whole. The piece in slot 0 records it.
+            if (p.direct_out && p.piece_counts && v.slot == 0 && warp == 0 && lane == 0)
+                p.piece_counts[v.b * p.Hkv + v.h_kv] = v.whole ? 0 : v.n_pieces;
+            if (!row_valid) return;
+            if (v.whole && p.direct_out) {
+                write_out(v, o, lse2);
+                return;
+            }
+            const int h_q = v.h_kv * p.G + r / nq, tq = r % nq;
+            const int64_t prow = ((static_cast<int64_t>(v.b) * p.Hq + h_q) * nq + tq) * p.num_splits + v.slot;
+            float4 *dst = reinterpret_cast<float4 *>(p.ws_o + prow * 128 + c_lo);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            if (c_lo == 0) p.ws_lse[prow] = lse2;
+        };
+        GdIter it;
+        gd_begin(p, gs, it);
+        GdUnit u;
+        while (ok && gd_next(p, gs, it, u)) {
+            const int T = u.T;
+            const int tq = r % nq;
+            if (T <= 0) {
+                // A piece with no key: O = 0 and lse = -inf for every query row.
+                float zero[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) zero[k] = 0.f;
+                finish(u, zero, -INFINITY);
                 continue;
             }
             // Exclusive key bound of this row (bottom-right causal alignment of the
@@ -835,30 +1065,7 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                 }
                 // O and l are both relative to m_O = m_w - e (log2 units).
                 const float lse2 = anyk ? log2f(l) - mneg - static_cast<float>(e) : -INFINITY;
-                if (row_valid) {
-                    if (p.direct_out) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(
-                            p.out + ((static_cast<int64_t>(u.b) * nq + tq) * p.Hq + h_q) * 128 + c_lo);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) {
-                                const __nv_bfloat162 v2 = __floats2bfloat162_rn(ov[8 * q + 2 * kk], ov[8 * q + 2 * kk + 1]);
-                                w[kk] = *reinterpret_cast<const uint32_t *>(&v2);
-                            }
-                            dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
-                        }
-                        if (c_lo == 0 && p.lse) p.lse[orow] = anyk ? lse2 * 0.6931471805599453f : -INFINITY;
-                    } else {
-                        const int64_t prow = orow * p.num_splits + u.split;
-                        float4 *dst = reinterpret_cast<float4 *>(p.ws_o + prow * 128 + c_lo);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            dst[q] = make_float4(ov[4 * q], ov[4 * q + 1], ov[4 * q + 2], ov[4 * q + 3]);
-                        if (c_lo == 0) p.ws_lse[prow] = lse2;
-                    }
-                }
+                finish(u, ov, lse2);
             }
             // All four owners of these rows are done with the unit (its m_O slot).
             __syncwarp();
@@ -870,6 +1077,66 @@ __global__ void __launch_bounds__(kGdThreads, 1)
         }
     }
     teardown_tmem(warp == kGdMmaWarp, tmem, kGdTmemCols);
+}
+
+// Merge of the cut sequences of a direct-output call with num_splits >= 2. One
+// CTA per sequence (b, h_kv) reads the piece count the decode kernel recorded
+// for it (0: written whole) and merges the pieces of a cut sequence. Thread
+// (row r, quarter q) merges channels 32q .. 32q+31 of row r:
+//     O = sum_s 2^(lse2_s - m) O_s / sum_s 2^(lse2_s - m),  m = max_s lse2_s.
+__global__ void __launch_bounds__(256) qk4v8_gqa_merge_kernel(const AttnParams p) {
+    const int b = static_cast<int>(blockIdx.x) / p.Hkv, h = static_cast<int>(blockIdx.x) % p.Hkv;
+    const int np = p.piece_counts[blockIdx.x];
+    const int R = p.G * p.Sq, nq = p.Sq;
+    const int r = threadIdx.x >> 2, c0 = (threadIdx.x & 3) * 32;
+    if (np < 2 || r >= R) return;
+    const int h_q = h * p.G + r / nq, tq = r % nq;
+    const int64_t orow = (static_cast<int64_t>(b) * p.Hq + h_q) * nq + tq;
+    const int64_t base = orow * p.num_splits;
+    // Two pieces at a time, their lse and O loads issued together, with a
+    // running max and sum over the pieces.
+    float m = -INFINITY, wsum = 0.f;
+    float acc[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+    for (int q0 = 0; q0 < np; q0 += 2) {
+        const bool two = q0 + 1 < np;
+        const float l0 = p.ws_lse[base + q0];
+        const float l1 = two ? p.ws_lse[base + q0 + 1] : -INFINITY;
+        const float4 *s0 = reinterpret_cast<const float4 *>(p.ws_o + (base + q0) * 128 + c0);
+        const float4 *s1 = reinterpret_cast<const float4 *>(p.ws_o + (base + q0 + (two ? 1 : 0)) * 128 + c0);
+        float4 x0[8], x1[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            x0[k] = s0[k];
+            x1[k] = s1[k];
+        }
+        const float mn = fmaxf(m, fmaxf(l0, l1));
+        if (mn == -INFINITY) continue;
+        const float a = exp2f(m - mn), w0 = exp2f(l0 - mn), w1 = exp2f(l1 - mn);
+        wsum = wsum * a + w0 + w1;
+        m = mn;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            acc[4 * k] = acc[4 * k] * a + w0 * x0[k].x + w1 * x1[k].x;
+            acc[4 * k + 1] = acc[4 * k + 1] * a + w0 * x0[k].y + w1 * x1[k].y;
+            acc[4 * k + 2] = acc[4 * k + 2] * a + w0 * x0[k].z + w1 * x1[k].z;
+            acc[4 * k + 3] = acc[4 * k + 3] * a + w0 * x0[k].w + w1 * x1[k].w;
+        }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((static_cast<int64_t>(b) * nq + tq) * p.Hq + h_q) * 128 + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const __nv_bfloat162 v2 = __floats2bfloat162_rn(acc[8 * q + 2 * kk] * inv, acc[8 * q + 2 * kk + 1] * inv);
+            w4[kk] = *reinterpret_cast<const uint32_t *>(&v2);
+        }
+        dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+    if (c0 == 0 && p.lse) p.lse[orow] = wsum > 0.f ? (m + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
 }
 
 cudaError_t launch_gqa_decode(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p,
@@ -893,10 +1160,11 @@ cudaError_t launch_gqa_decode(const CUtensorMap &tk, const CUtensorMap &tv, cons
         }
     }
     // Persistent: one CTA per SM (shared memory and the 512 TMEM columns allow no
-    // more), each walking the units blockIdx.x, blockIdx.x + grid, ...
-    const int n_units = p.B * p.Hkv * p.num_splits;
-    const int grid = n_units < sms ? n_units : sms;
-    qk4v8_gqa_decode_kernel<<<grid, kGdThreads, GdSmem::kBytes, stream>>>(tk, tv, p);
+    // more); the kernel schedules the work over the grid itself.
+    qk4v8_gqa_decode_kernel<<<sms, kGdThreads, GdSmem::kBytes, stream>>>(tk, tv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !p.direct_out || p.num_splits < 2) return e;
+    qk4v8_gqa_merge_kernel<<<p.B * p.Hkv, 256, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -37,7 +37,8 @@ struct AttnParams {
     float *lse;               // prefill [B][Hq][Sq] (natural log), nullable
     float *ws_o;              // decode partial outputs [B][Hq][nq][splits][128]
     float *ws_lse;            // decode partial log2-sum-exp [B][Hq][nq][splits]
-    int direct_out;           // swap-AB decode with one split: write out [B][nq][Hq][128] and lse directly
+    int direct_out;           // decode: write out [B][nq][Hq][128] and lse directly
+    int32_t *piece_counts;    // GQA decode with splits: [B][Hkv] pieces of each sequence (0: written whole)
     int32_t *status;          // nullable
     int test_stall;           // test hook: the producer withholds the Q-ready signal
     float *test_dump_s;       // test hook: CTA 0 writes its first raw score tile [128 lanes][128 keys]
@@ -67,7 +68,8 @@ constexpr int kDecodeMaxRows = 64;
 cudaError_t launch_decode(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p, int grid,
                           cudaStream_t stream);
 // GQA decode kernel for kGqaMinRows..kDecodeMaxRows query rows per KV head
-// (persistent over the (sequence, KV head, split) units; packed MXFP4 queries).
+// (persistent, one CTA per SM; packed MXFP4 queries), followed, for a
+// direct-output call with splits, by the merge of the cut sequences.
 constexpr int kGqaMinRows = 33;
 cudaError_t launch_gqa_decode(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p,
                               cudaStream_t stream);

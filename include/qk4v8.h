@@ -148,7 +148,12 @@ QK4V8_API int qk4v8_attention_prefill(const uint8_t *q_codes, const uint8_t *q_s
                             const int32_t *seqlens_k, int causal, float softmax_scale,
                             void *out, float *lse, int32_t *dev_status, void *stream);
 
-/* Workspace bytes for qk4v8_attention_decode with these sizes. */
+/*
+ * Workspace bytes for qk4v8_attention_decode with these sizes: the split
+ * partials float O[B][Hq][nq][splits][128], then float lse2[B][Hq][nq][splits],
+ * then int32 [B][Hq] piece counts (the GQA decode kernel records there which
+ * sequences it cut, for its merge launch).
+ */
 QK4V8_API size_t qk4v8_decode_workspace_bytes(int B, int Hq, int nq, int num_splits);
 
 /*
@@ -163,9 +168,10 @@ QK4V8_API int qk4v8_decode_default_splits(int B, int Hq, int Hkv, int nq, int ma
 /*
  * The two stages of qk4v8_attention_decode, as separate launches.
  *
- * qk4v8_attention_decode_splitkv: one CTA per (sequence, KV head, split) runs
- * the tiled QK4V8 attention over its contiguous slice of the cache. It writes
- * the split's normalised partial output and log2-sum-exp to `workspace`:
+ * qk4v8_attention_decode_splitkv: for every (sequence, KV head, split) the
+ * split kernel runs the tiled QK4V8 attention over the split's contiguous
+ * slice of the cache. It writes the split's normalised partial output and
+ * log2-sum-exp to `workspace`:
  *     float O[B][Hq][nq][splits][128], then float lse2[B][Hq][nq][splits].
  * A split with no key writes O = 0 and lse2 = -inf. Arguments as for
  * qk4v8_attention_decode.
@@ -198,7 +204,17 @@ QK4V8_API int qk4v8_decode_merge(const void *workspace, size_t workspace_bytes, 
  *            unused (and may be null) when the call runs one split with
  *            (Hq / Hkv) * nq <= 64, as the split kernel then writes out itself
  *   out      bf16 [B][nq][Hq][128]; lse float [B][Hq][nq] (nullable)
- * Requires (Hq / Hkv) * nq <= 128.
+ * Requires (Hq / Hkv) * nq <= 128. Kernels by query rows per KV head:
+ *   - up to 32: the swap-AB split kernel, then the merge (one launch when one
+ *     split);
+ *   - 33..64: the GQA decode kernel, one CTA per SM, which writes out and lse
+ *     for every sequence it does not cut. When splits >= 2 and no sequence
+ *     would be cut into more than `splits` pieces, it spreads the key tiles of
+ *     all sequences evenly over the CTAs instead of cutting every sequence
+ *     into `splits` equal parts; a sequence is then cut only where a CTA's
+ *     share ends. With splits >= 2 a second, short launch merges the pieces of
+ *     the cut sequences from the workspace.
+ *   - 65..128: the 128-row split kernel, then the merge.
  */
 QK4V8_API int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
                            const uint8_t *k_codes, const uint8_t *k_scales,
@@ -212,9 +228,12 @@ QK4V8_API int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_sc
  * MXFP4 scales are computed as it is loaded, inside the attention call).
  * Same result, bit for bit, as qk4v8_quantize_qk (capacity 128) followed by
  * qk4v8_attention_decode, in one call and usually one launch:
- *   - (Hq / Hkv) * nq <= 64: the split kernel reads the bf16 query rows and
+ *   - (Hq / Hkv) * nq <= 32: the split kernel reads the bf16 query rows and
  *     encodes them to MXFP4 itself; with one split it also writes out and lse
  *     directly, so there is no merge launch and no workspace.
+ *   - 33..64: the nq query rows of each head are quantized into the front of
+ *     the workspace (capacity 128 tokens), then the GQA decode kernel writes
+ *     out and lse.
  *   - larger groups: the queries are quantized into the front of the
  *     workspace, then the 128-row split kernel and the merge run.
  *   q        bf16 [B][nq][Hq][128] (device), element strides q_stride_b,
@@ -252,10 +271,10 @@ QK4V8_API int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, 
  *   - The first call on each device looks up the array's device address, with
  *     that device current. Make that first call before any stream capture.
  *   - Every call shares the one array, and the array keeps the last call's
- *     contents. Nothing in it has to start at zero: the split-KV kernel writes
- *     every slot the merge reads. Calls that overlap on the GPU (different
- *     streams, or different host threads without ordering) race on the array;
- *     serialise them.
+ *     contents. Nothing in it has to start at zero: the split kernels write
+ *     every partial slot before a merge reads it. Calls that overlap on the GPU
+ *     (different streams, or different host threads without ordering) race on
+ *     the array; serialise them.
  *   - It allocates nothing (no cudaMalloc, no cudaFree, no allocating library
  *     call). Arguments and results as for qk4v8_attention_decode.
  */

@@ -51,7 +51,7 @@ def test_size_helpers(lib):
     assert lib.qk4v8_mxfp4_codes_bytes(2, 3, 256) == 2 * 3 * 256 * 64
     assert lib.qk4v8_mxfp8_codes_bytes(2, 3, 256) == 2 * 3 * 128 * 256
     assert lib.qk4v8_scales_bytes(2, 3, 256) == 2 * 3 * 2 * 512
-    assert lib.qk4v8_decode_workspace_bytes(4, 8, 2, 3) == 4 * 8 * 2 * 3 * 129 * 4
+    assert lib.qk4v8_decode_workspace_bytes(4, 8, 2, 3) == 4 * 8 * 2 * 3 * 129 * 4 + 4 * 8 * 4
     assert lib.qk4v8_decode_workspace_bytes(0, 8, 2, 3) == 0
     # KV bytes per token per kv-head: 64 (E2M1 codes) + 128 (E4M3) + 4 + 4 (scales) = 200
     cap = 8192

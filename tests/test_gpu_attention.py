@@ -328,3 +328,32 @@ def test_gqa_decode_o_rescale_path():
         assert_close(out, ref, f"GQA decode O rescale, splits={splits}")
         l = lse.cpu().numpy().transpose(0, 2, 1)
         assert np.abs(l - rlse).max() < 1e-2 + 1e-5 * np.abs(rlse).max()
+
+
+@pytest.mark.parametrize("B,nq,L,Hq,Hkv,splits,lens", [
+    # 8 x 8 sequences of 32 tiles over one CTA per SM: each CTA's even share of
+    # the 2048 tiles is 13 or 14, so sequences are cut into up to 4 pieces.
+    (8, 8, 4096, 64, 8, 4, None),
+    # Mixed lengths (empty, one key, a few tiles, long): whole sequences, pieces
+    # spread over up to 17 CTAs, and empty sequences inside the tile list.
+    (16, 8, 4096, 16, 2, 20, [4096, 0, 1, 129, 4096, 3000, 0, 255, 4000, 17, 2048, 4096, 1024, 0, 3500, 640]),
+])
+def test_gqa_decode_balanced_schedule(B, nq, L, Hq, Hkv, splits, lens):
+    """GQA decode with the balanced schedule: key tiles of all sequences spread
+    evenly over the CTAs, sequences cut at the CTA range boundaries merged by
+    the follow-up launch. Checked against the oracle, and against a one-split
+    run of the same kernel (each sequence whole in one CTA)."""
+    gen = make_gen(B, nq, L, Hq, Hkv, seed=L + B + splits, lens=lens, k_out=4)
+    (ref, rlse), _ = oracle_attention_from(gen, True)
+    out, lse, _ = run_decode(gen, True, splits)
+    one, one_lse, _ = run_decode(gen, True, 1)
+    assert_close(out, ref, f"balanced GQA decode B{B} splits{splits}")
+    assert_close(one, ref, f"one-split GQA decode B{B}")
+    fin = np.isfinite(rlse)
+    for got in (lse, one_lse):
+        l = got.cpu().numpy().transpose(0, 2, 1)
+        assert np.array_equal(np.isfinite(l), fin)
+        assert np.abs(l[fin] - rlse[fin]).max() < 1e-2
+    # The same call twice gives the same bits.
+    again, _, _ = run_decode(gen, True, splits)
+    assert torch.equal(out, again)
