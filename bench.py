@@ -183,8 +183,17 @@ def decode_kernel_name(rows: int) -> str:
     if rows <= 32:
         return "qk4v8_decode_kernel<32,32,16,6,1> (swap-AB split-KV decode)"
     if rows <= 64:
-        return "qk4v8_decode_kernel<64,64,16,6,1> (swap-AB split-KV decode)"
+        return "qk4v8_gqa_decode_kernel (row-owner GQA decode, key tiles balanced over one CTA per SM)"
     return "qk4v8_attention_kernel<true> (128-row split-KV decode)"
+
+
+def decode_launches(rows: int, splits: int) -> int:
+    """Kernel launches of one qk4v8_attention_decode_bf16 call."""
+    if rows <= 32:
+        return 1 if splits == 1 else 2               # split kernel (+ merge)
+    if rows <= 64:
+        return 2 if splits == 1 else 3               # query quantize, GQA decode kernel (+ merge of cut sequences)
+    return 3                                         # query quantize, 128-row split kernel, merge
 
 
 def run_decode(args, world, rank):
@@ -215,7 +224,7 @@ def run_decode(args, world, rank):
     # The K timed steps run as one CUDA graph, so host launch overhead does not
     # pace the device; two events bracket the whole replay.
     rows = wl.G * wl.Sq
-    launches = (1 if rows <= 64 else 2) + (0 if splits == 1 and rows <= 64 else 1)
+    launches = decode_launches(rows, splits)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for _ in range(args.steps):
@@ -333,12 +342,11 @@ def run_decode_workload(name, steps, warmup, hbm_gbs):
     kv_bytes = int(lens.sum()) * wl.Hkv * KV_BYTES_PER_TOKEN_HEAD   # the packed cache each step streams
     gbs = kv_bytes / (ms * 1e-3) / 1e9
     rows = wl.G * wl.Sq
-    one_launch = rows <= 64 and splits == 1
     return {
         "workload": name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "nq": wl.Sq, "kv_len_mean": float(lens.mean()),
         "kv_len_max": max_len, "kv_splits": splits, "ms_per_step": ms, "value": gbs, "unit": "GB/s",
         "tokens_per_s": wl.B * wl.Sq / (ms * 1e-3),
-        "launches_per_step": 1 if one_launch else (2 if rows <= 64 else 3),
+        "launches_per_step": decode_launches(rows, splits),
         "roofline": {"bound": "hbm", "kernel": decode_kernel_name(rows), "achieved": gbs, "peak": hbm_gbs,
                      "unit": "GB/s", "frac": gbs / hbm_gbs, "algorithmic_bytes_per_step": kv_bytes,
                      "note": "step time (all launches of the call); the split kernel dominates it"},
