@@ -273,11 +273,20 @@ size_t qk4v8_decode_workspace_bytes(int B, int Hq, int nq, int num_splits) {
 }
 
 int qk4v8_decode_default_splits(int B, int Hq, int Hkv, int nq, int max_seqlen) {
-    // Wave cost model: a launch of units * s CTAs over `slots` resident CTA
-    // slots takes ceil(units * s / slots) waves, each as long as one split
+    // For 33..64 query rows per KV head the GQA decode kernel is persistent and
+    // can spread the key tiles of all sequences evenly over the CTAs; it does so
+    // when no sequence would be cut into more pieces than there are splits.
+    // With at most half as many sequences as CTAs (where whole sequences would
+    // leave many CTAs idle), plan for that: for sequences of at least half the
+    // maximum length each CTA's share is at least range/2 tiles (range = units
+    // * tiles / slots), and a sequence meets at most ceil(tiles / (range/2)) + 1
+    // shares. Otherwise (and for problems of less than two tiles per CTA, and
+    // other group sizes) use the wave cost model: a launch of units * s CTAs
+    // over `slots` resident CTA slots
+    // takes ceil(units * s / slots) waves, each as long as one split
     // (ceil(tiles / s) key tiles of 128) plus a fixed cost of about
-    // kSplitOverheadTiles tiles for the prologue, pipeline fill and epilogue.
-    // Pick the cheapest s, the smallest on ties.
+    // kSplitOverheadTiles tiles for the prologue, pipeline fill and epilogue;
+    // the cheapest s, the smallest on ties.
     constexpr int kSplitOverheadTiles = 3;
     constexpr int kMaxSplits = 64;
     if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv || nq <= 0) return 1;
@@ -291,6 +300,12 @@ int qk4v8_decode_default_splits(int B, int Hq, int Hkv, int nq, int max_seqlen) 
     const int64_t slots = static_cast<int64_t>(sms) * (rows <= 16 ? 2 : 1);
     const int64_t units = static_cast<int64_t>(B) * Hkv;
     const int tiles = max_seqlen > 0 ? (max_seqlen + 127) / 128 : 1;
+    if (rows >= qk4v8::kGqaMinRows && rows <= qk4v8::kDecodeMaxRows && 2 * units <= slots &&
+        units * tiles >= 2 * slots) {
+        const int64_t half = units * tiles / slots / 2;
+        const int64_t s = (tiles + half - 1) / half + 1;
+        return static_cast<int>(s < kMaxSplits ? s : kMaxSplits);
+    }
     int best = 1;
     int64_t best_cost = INT64_MAX;
     for (int s = 1; s <= kMaxSplits && s <= tiles; ++s) {
@@ -365,8 +380,7 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
     const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen);
     // Direct output: the swap-AB kernel with one split, and the GQA decode kernel
     // always (with splits, its own merge launch finishes the cut sequences).
-    const bool gqa = gqa_rows(Hq, Hkv, nq);
-    const bool direct_out = out && ((splits == 1 && swap_ab_rows(Hq, Hkv, nq)) || gqa);
+    const bool direct_out = out && ((splits == 1 && swap_ab_rows(Hq, Hkv, nq)) || gqa_rows(Hq, Hkv, nq));
     if (out && !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
     const size_t need = (direct_out && splits == 1) ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
     if (need && (!workspace || !aligned16(workspace) || workspace_bytes < need))

@@ -73,6 +73,9 @@ cudaError_t launch_decode(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, 
 constexpr int kGqaMinRows = 33;
 cudaError_t launch_gqa_decode(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p,
                               cudaStream_t stream);
+// Merge of the sequences a persistent decode kernel cut (direct output, splits >= 2,
+// <= 64 rows per KV head), from the partials and the recorded piece counts.
+cudaError_t launch_cut_merge(const AttnParams &p, cudaStream_t stream);
 cudaError_t launch_decode_merge(const float *ws_o, const float *ws_lse, int B, int Hq, int nq, int splits,
                                 __nv_bfloat16 *out, float *lse, cudaStream_t stream);
 

@@ -61,18 +61,24 @@ def test_size_helpers(lib):
 
 
 def test_default_splits(lib):
-    """Wave cost model, 148 SMs without a device: waves * (tiles per split + 3).
-    Worked by hand: B=32, Hkv=8, 4 rows (two CTAs per SM, 296 slots), 64 tiles:
-    s=1 costs 1 * 67, s=2 costs 2 * 35. B=8, Hkv=8, 8 rows, 1024 tiles: s=9 is
-    576 CTAs in 2 waves of 114 + 3 = 234, below s=4 (259) and s=18 (240).
-    B=64, Hkv=8, 64 rows (one CTA per SM), 128 tiles: s=2 is 7 waves of 67 =
-    469, below s=1 (4 * 131) and s=4 (14 * 35)."""
+    """148 SMs without a device. For 33..64 rows per KV head (the persistent GQA
+    decode kernel), with at most half as many sequences as CTAs and at least two
+    key tiles per CTA: enough splits for its balanced schedule with sequences of
+    half the maximum length, ceil(tiles / half) + 1 with half = units * tiles /
+    slots / 2. Worked by hand: B=8, Hkv=8, 64 rows (one CTA per SM, 148 slots),
+    1024 tiles: half = 65536 / 148 / 2 = 221, so 5 + 1 = 6. Otherwise the wave
+    cost model, waves * (tiles per split + 3): B=32, Hkv=8, 4 rows (two CTAs per
+    SM, 296 slots), 64 tiles: s=1 costs 1 * 67, s=2 costs 2 * 35. B=8, Hkv=8,
+    8 rows, 1024 tiles: s=9 is 576 CTAs in 2 waves of 114 + 3 = 234, below s=4
+    (259) and s=18 (240). B=64, Hkv=8, 64 rows, 128 tiles: s=2 is 7 waves of
+    67 = 469, below s=1 (4 * 131) and s=4 (14 * 35)."""
     f = lib.qk4v8_decode_default_splits
     assert f(32, 32, 8, 1, 8192) == 1
     assert f(8, 64, 8, 1, 131072) == 9
+    assert f(8, 64, 8, 8, 131072) == 6
     assert f(64, 64, 8, 8, 16384) == 2
     assert f(1, 1, 1, 1, 100) == 1
-    assert f(2, 8, 2, 1, 1000) == 8          # never more splits than tiles
+    assert f(2, 8, 2, 1, 1000) == 8          # wave model; never more splits than tiles
     for bad in ((0, 8, 8, 1, 100), (1, 30, 8, 1, 100), (1, 8, 8, 0, 100)):
         assert f(*bad) == 1
 
