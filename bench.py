@@ -156,13 +156,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest x over the ranks (the step time of a multi-GPU run is the slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_gbs(bytes_per_rank_step: int, steps: int, world: int, elapsed_ms: float) -> float:
+    """Whole-job throughput: the bytes every rank streamed over the slowest rank's time (weak scaling)."""
+    return bytes_per_rank_step * steps * world / (elapsed_ms * 1e-3) / 1e9
 
 
 def to_dev(bits):
@@ -581,11 +588,10 @@ def main():
     d = run_decode(args, world, rank)
     wl = d["wl"]
     steps = args.steps
-    total_bytes = d["kv_bytes"] * steps * world
-    value = total_bytes / (d["elapsed_ms"] * 1e-3) / 1e9
+    value = aggregate_gbs(d["kv_bytes"], steps, world, d["elapsed_ms"])
     ms_per_step = d["elapsed_ms"] / steps
     achieved = d["kv_bytes"] / (d["attn_avg_ms"] * 1e-3) / 1e9
-    e2e_value = d["kv_bytes"] * d["e2e_steps"] * world / (d["e2e_ms"] * 1e-3) / 1e9
+    e2e_value = aggregate_gbs(d["kv_bytes"], d["e2e_steps"], world, d["e2e_ms"])
 
     line = {
         "metric": METRIC,
