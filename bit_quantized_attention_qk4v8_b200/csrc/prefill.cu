@@ -342,62 +342,74 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
     } else if (warp == kPfMmaWarp) {
         // -------------------------------------------------------------- MMA issuer
-        // The whole warp runs the loop and waits, so the descriptors stay
-        // warp-uniform; one elected lane issues the tcgen05 instructions.
+        // Every tcgen05 instruction of this role (copies of scale atoms, MMAs,
+        // commits) is issued by a single thread, so one elected thread runs the
+        // whole loop: its waits need no warp votes and its issue path no
+        // reconvergence. That path sets the pace of the QK^T stage.
         uint32_t pred;
         asm volatile(
             "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\tselp.u32 %0, 1, 0, e;\n\t}"
             : "=r"(pred));
-        const bool leader = pred != 0;
-        const uint32_t sb = smem_u32(smem);
-        // Descriptors for stage / buffer 0; the others are fixed offsets of the
-        // 14-bit start-address field (16-byte units).
-        const uint64_t dQ0 = smem_desc(sb + S::kQ, 16, 512, 4);
-        const uint64_t dK0 = smem_desc(sb + S::kK, 16, 512, 4);
-        const uint64_t dV0 = smem_desc(sb + S::kV, 16, 1024, 2);
-        const uint64_t dP0 = smem_desc(sb + S::kP, 16, 1024, 2);
-        const uint64_t dSfQ0 = smem_desc(sb + S::kSfQ, 0, 128, 0);
-        const uint64_t dSfK0 = smem_desc(sb + S::kSfK, 0, 128, 0);
-        const uint64_t dSfV0 = smem_desc(sb + S::kSfV, 0, 128, 0);
-        const uint64_t dSfP0 = smem_desc(sb + S::kSfP, 0, 128, 0);
-        const uint32_t tO = tmem + kPfColO;
-        bool ok = true;
-        if (!kStageQK) {
-            // The ones row's scale, for both V scale buffers, once.
-            if (leader) {
+        if (pred != 0) {
+            const uint32_t sb = smem_u32(smem);
+            // Descriptors for stage / buffer 0; the others are fixed offsets of the
+            // 14-bit start-address field (16-byte units).
+            const uint64_t dQ0 = smem_desc(sb + S::kQ, 16, 512, 4);
+            const uint64_t dK0 = smem_desc(sb + S::kK, 16, 512, 4);
+            const uint64_t dV0 = smem_desc(sb + S::kV, 16, 1024, 2);
+            const uint64_t dP0 = smem_desc(sb + S::kP, 16, 1024, 2);
+            const uint64_t dSfQ0 = smem_desc(sb + S::kSfQ, 0, 128, 0);
+            const uint64_t dSfK0 = smem_desc(sb + S::kSfK, 0, 128, 0);
+            const uint64_t dSfV0 = smem_desc(sb + S::kSfV, 0, 128, 0);
+            const uint64_t dSfP0 = smem_desc(sb + S::kSfP, 0, 128, 0);
+            const uint32_t tO = tmem + kPfColO;
+            bool ok = true;
+            if (!kStageQK) {
+                // The ones row's scale, for both V scale buffers, once.
                 const uint64_t dOne = smem_desc(sb + S::kSfOne, 0, 128, 0);
                 tc_cp_32x128b_warpx4(tmem + pf_col_sf_v(0) + 4, dOne);
                 tc_cp_32x128b_warpx4(tmem + pf_col_sf_v(1) + 4, dOne);
             }
-            __syncwarp();
-        }
-        int g = 0, c = 0, n_patch = 0;
-        for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
-            const PfUnit u = pf_unit(p, un);
-            const int T = u.T;
-            if (T <= 0) continue;
-            const int qb = c & 1;
-            const bool last_partial = !kStageQK && (u.L & 127) != 0 && T == (u.L + 127) / 128;
-            ok = __all_sync(0xffffffffu, wait_bar(&q_full[qb], (c >> 1) & 1, abort_flag, p.status));
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t tSfQ = tmem + pf_col_sf_q(qb);
-            const uint64_t dQ = dQ0 + static_cast<uint64_t>(qb * (S::kQBytes >> 4));
-            if (leader) tc_cp_32x128b_warpx4(tSfQ, dSfQ0 + static_cast<uint64_t>(qb * 32));
-            __syncwarp();
-            // S(gi) = Q K(gi)^T into S buffer gi & 1, once K(gi) has landed and the
-            // warps of parity gi & 1 have read S(gi-2) out of that buffer.
-            auto issue_qk = [&](int i) -> bool {
-                const int gi = g + i;
-                const int st = gi % kPfKStages;
-                bool w = wait_bar(&k_full[st], (gi / kPfKStages) & 1, abort_flag, p.status);
-                if (w && gi >= 2) w = wait_bar(&s_free[gi & 1], ((gi - 2) >> 1) & 1, abort_flag, p.status);
-                if (!__all_sync(0xffffffffu, w)) return false;
+            int g = 0, c = 0, n_patch = 0;
+            // The next unit's description is worked out while this unit's first S
+            // computes, off the issue path of the unit transition.
+            PfUnit nu = pf_unit(p, blockIdx.x);
+            for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
+                const PfUnit u = nu;
+                const int T = u.T;
+                if (T <= 0) {
+                    if (un + static_cast<int>(gridDim.x) < n_units) nu = pf_unit(p, un + gridDim.x);
+                    continue;
+                }
+                const int qb = c & 1;
+                const bool last_partial = !kStageQK && (u.L & 127) != 0 && T == (u.L + 127) / 128;
+                ok = mbar_test_wait(&q_full[qb], (c >> 1) & 1) ||
+                     wait_bar(&q_full[qb], (c >> 1) & 1, abort_flag, p.status);
+                if (!ok) break;
                 tc_fence_after();
-                const uint32_t tSfK = tmem + pf_col_sf_k(gi & 1);
-                const uint64_t dK = dK0 + static_cast<uint64_t>(st * (S::kKBytes >> 4));
-                const uint32_t tS = tmem + pf_col_s(gi & 1);
-                if (leader) {
+                const uint32_t tSfQ = tmem + pf_col_sf_q(qb);
+                const uint64_t dQ = dQ0 + static_cast<uint64_t>(qb * (S::kQBytes >> 4));
+                tc_cp_32x128b_warpx4(tSfQ, dSfQ0 + static_cast<uint64_t>(qb * 32));
+                // S(gi) = Q K(gi)^T into S buffer gi & 1, once K(gi) has landed and the
+                // warps of parity gi & 1 have read S(gi-2) out of that buffer.
+                auto issue_qk = [&](int i) -> bool {
+                    const int gi = g + i;
+                    const int st = gi % kPfKStages;
+                    const uint32_t kpar = (gi / kPfKStages) & 1;
+                    const uint32_t spar = ((gi - 2) >> 1) & 1;
+                    // Both inputs are usually ready by now: one probe of the two
+                    // barriers, the bounded waits only when it fails.
+                    bool w = gi >= 2 ? mbar_test_wait2(&k_full[st], kpar, &s_free[gi & 1], spar)
+                                     : mbar_test_wait(&k_full[st], kpar);
+                    if (!w) {
+                        w = wait_bar(&k_full[st], kpar, abort_flag, p.status);
+                        if (w && gi >= 2) w = wait_bar(&s_free[gi & 1], spar, abort_flag, p.status);
+                    }
+                    if (!w) return false;
+                    tc_fence_after();
+                    const uint32_t tSfK = tmem + pf_col_sf_k(gi & 1);
+                    const uint64_t dK = dK0 + static_cast<uint64_t>(st * (S::kKBytes >> 4));
+                    const uint32_t tS = tmem + pf_col_s(gi & 1);
                     tc_cp_32x128b_warpx4(tSfK, dSfK0 + static_cast<uint64_t>(st * 32));
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk)
@@ -405,28 +417,32 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                     tSfK | ((2u * kk) << 30), kk > 0 ? 1u : 0u);
                     tc_commit(&s_full[gi & 1]);
                     tc_commit(&k_empty[st]);
-                }
-                __syncwarp();
-                return true;
-            };
-            // O += P(gi) V(gi), once V(gi) has landed and the warps of parity gi & 1
-            // have written P(gi); the unit's first one overwrites O, once the previous
-            // unit's epilogue has read it.
-            auto issue_pv = [&](int i) -> bool {
-                const int gi = g + i;
-                const int sv = gi % kPfVStages;
-                bool w = wait_bar(&v_full[sv], (gi / kPfVStages) & 1, abort_flag, p.status);
-                if (w && last_partial && i == T - 1) w = wait_bar(patch, n_patch & 1, abort_flag, p.status);
-                if (w && i == 0 && c >= 1) w = wait_bar(o_free, (c - 1) & 1, abort_flag, p.status);
-                if (w) w = wait_bar(&p_full[gi & 1], (gi >> 1) & 1, abort_flag, p.status);
-                if (!__all_sync(0xffffffffu, w)) return false;
-                tc_fence_after();
-                const uint32_t tSfV = tmem + pf_col_sf_v(gi & 1);
-                const uint32_t tSfP = tmem + pf_col_sf_p(gi & 1);
-                const uint64_t dV = dV0 + static_cast<uint64_t>(sv * (S::kVBytes >> 4));
-                const uint64_t dPhi = dP0 + static_cast<uint64_t>((gi & 1) * (S::kPBuf >> 4));
-                const uint64_t dPlo = dPhi + static_cast<uint64_t>((128 * 128) >> 4);
-                if (leader) {
+                    return true;
+                };
+                // O += P(gi) V(gi), once V(gi) has landed and the warps of parity gi & 1
+                // have written P(gi); the unit's first one overwrites O, once the
+                // previous unit's epilogue has read it.
+                auto issue_pv = [&](int i) -> bool {
+                    const int gi = g + i;
+                    const int sv = gi % kPfVStages;
+                    const uint32_t vpar = (gi / kPfVStages) & 1;
+                    const uint32_t ppar = (gi >> 1) & 1;
+                    const bool need_patch = last_partial && i == T - 1;
+                    const bool need_ofree = i == 0 && c >= 1;
+                    bool w = !need_patch && !need_ofree && mbar_test_wait2(&v_full[sv], vpar, &p_full[gi & 1], ppar);
+                    if (!w) {
+                        w = wait_bar(&v_full[sv], vpar, abort_flag, p.status);
+                        if (w && need_patch) w = wait_bar(patch, n_patch & 1, abort_flag, p.status);
+                        if (w && need_ofree) w = wait_bar(o_free, (c - 1) & 1, abort_flag, p.status);
+                        if (w) w = wait_bar(&p_full[gi & 1], ppar, abort_flag, p.status);
+                    }
+                    if (!w) return false;
+                    tc_fence_after();
+                    const uint32_t tSfV = tmem + pf_col_sf_v(gi & 1);
+                    const uint32_t tSfP = tmem + pf_col_sf_p(gi & 1);
+                    const uint64_t dV = dV0 + static_cast<uint64_t>(sv * (S::kVBytes >> 4));
+                    const uint64_t dPhi = dP0 + static_cast<uint64_t>((gi & 1) * (S::kPBuf >> 4));
+                    const uint64_t dPlo = dPhi + static_cast<uint64_t>((128 * 128) >> 4);
                     tc_cp_32x128b_warpx4(tSfV, dSfV0 + static_cast<uint64_t>(sv * 32));
                     tc_cp_32x128b_warpx4(tSfP, dSfP0 + static_cast<uint64_t>((gi & 1) * 32));
 #pragma unroll
@@ -439,35 +455,34 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                     tSfV | (k << 30), 1u);
                     tc_commit(&pv_done[gi & 1]);
                     tc_commit(&v_empty[sv]);
+                    return true;
+                };
+                // The tensor pipe runs in issue order, so the issue order follows the
+                // order in which the softmax warps release their inputs: S(i) is read
+                // early in tile i, while P(i-1) is written at the end of tile i-1 by the
+                // other warp, later. So: S(0), S(1), then per tile i: S(i+2) once S(i)
+                // has been read, then P(i-1) V(i-1). S(i+2) then never queues behind a
+                // P V.
+                ok = issue_qk(0);
+                if (ok && T > 1) ok = issue_qk(1);
+                if (un + static_cast<int>(gridDim.x) < n_units) nu = pf_unit(p, un + gridDim.x);
+                for (int i = 0; i < T && ok; ++i) {
+                    if (i + 2 < T) ok = issue_qk(i + 2);
+                    if (ok && !kStageQK && i >= 1) ok = issue_pv(i - 1);
                 }
-                __syncwarp();
-                return true;
-            };
-            // The tensor pipe runs in issue order, so the issue order follows the order
-            // in which the softmax warps release their inputs: S(i) is read early in
-            // tile i, while P(i-1) is written at the end of tile i-1 by the other
-            // warp, later. So: S(0), S(1), then per tile i: S(i+2) once S(i) has been
-            // read, then P(i-1) V(i-1). S(i+2) then never queues behind a P V.
-            ok = issue_qk(0);
-            if (ok && T > 1) ok = issue_qk(1);
-            for (int i = 0; i < T && ok; ++i) {
-                if (i + 2 < T) ok = issue_qk(i + 2);
-                if (ok && !kStageQK && i >= 1) ok = issue_pv(i - 1);
-            }
-            if (ok && !kStageQK) ok = issue_pv(T - 1);
-            if (!ok) break;
-            if (leader) {
+                if (ok && !kStageQK) ok = issue_pv(T - 1);
+                if (!ok) break;
                 tc_commit(&q_empty[qb]);  // Q buffer and its scale columns free for unit c + 2
                 if (!kStageQK) tc_commit(o_full);
+                if (last_partial) ++n_patch;
+                g += T;
+                ++c;
             }
-            __syncwarp();
-            if (last_partial) ++n_patch;
-            g += T;
-            ++c;
+            // Every tcgen05 operation issued above has completed once `drain` does,
+            // also when the loop unwound early, so TMEM is freed with nothing in
+            // flight.
+            tc_commit(drain);
         }
-        // Every tcgen05 operation issued above has completed once `drain` does, also
-        // when the loop unwound early, so TMEM is freed with nothing in flight.
-        if (leader) tc_commit(drain);
         __syncwarp();
         (void)wait_peers(drain, 0);
     } else if (warp < kPfSoftmaxWarps) {
