@@ -34,8 +34,9 @@
 // ones, so O column 128 accumulates the softmax denominator sum(P_hi + P_lo)
 // in the same MMAs.
 //
-// Warp roles (320 threads): warps 0..7 softmax and epilogue, warp 8 TMA
-// producer, warp 9 TMEM allocator and MMA issuer.
+// Warp roles (352 threads): warps 0..7 softmax and epilogue, warp 8 Q/K
+// producer (TMA), warp 9 TMEM allocator and MMA issuer, warp 10 V producer
+// (TMA). The producers and the MMA issuer each run on one elected thread.
 //
 // kStageQK builds the QK^T stage alone over the same tile schedule: Q/K loads
 // with their scales, the mxf4 MMAs and the TMEM drain with the row max. It
@@ -56,13 +57,14 @@ namespace qk4v8 {
 
 namespace {
 
-constexpr int kPfKStages = 4;               // K tiles in flight (freed when QK^T of the tile completes)
+constexpr int kPfKStages = 6;               // K tiles in flight (freed when QK^T of the tile completes)
 constexpr int kPfVStages = 4;               // V tiles in flight (freed when P V of the tile completes)
 constexpr int kPfSoftmaxWarps = 8;          // two per TMEM lane quarter, alternate key tiles
-// Warps 0..7 softmax, then the producer and the MMA issuer.
-constexpr int kPfThreads = 32 * kPfSoftmaxWarps + 64;
-constexpr int kPfProducerWarp = 8;
+// Warps 0..7 softmax, then the Q/K producer, the MMA issuer and the V producer.
+constexpr int kPfThreads = 32 * kPfSoftmaxWarps + 96;
+constexpr int kPfProducerWarp = 8;          // Q and K tiles with their scales
 constexpr int kPfMmaWarp = 9;
+constexpr int kPfVWarp = 10;                // V tiles with their scales
 constexpr float kPfTau = 8.0f;              // m_w moves once a score passes it by 2^8
 constexpr int kPfEMax = 64;                 // largest e = m_w - m_O before O is rescaled
 constexpr float kPfMaxMove = 16777216.0f;   // cap on one move of m_w, keeps it an exact integer
@@ -125,23 +127,56 @@ struct PfUnit {
     int b, h_q, h_kv, q0, L, T;
 };
 
+// Integer quotient a / b for 0 <= a, 1 <= b through the float reciprocal rb of
+// b, corrected to the exact value by the integer remainder. A unit's
+// description is worked out on the issue paths of the producer and the MMA
+// warp at every unit change, where the emulated integer divisions cost
+// hundreds of cycles.
+__device__ __forceinline__ int pf_div(int a, int b, float rb) {
+    int q = static_cast<int>(static_cast<float>(a) * rb);
+    int r = a - q * b;
+    while (r < 0) {
+        --q;
+        r += b;
+    }
+    while (r >= b) {
+        ++q;
+        r -= b;
+    }
+    return q;
+}
+
+struct PfDecode {
+    int per;           // units per query tile row: B * Hq
+    float r_per, r_hq, r_g;
+};
+
+__device__ __forceinline__ PfDecode pf_decode(const AttnParams &p) {
+    PfDecode d;
+    d.per = p.B * p.Hq;
+    d.r_per = 1.0f / static_cast<float>(d.per);
+    d.r_hq = 1.0f / static_cast<float>(p.Hq);
+    d.r_g = 1.0f / static_cast<float>(p.G);
+    return d;
+}
+
 // Work unit `idx`: one query head and 128 query tokens. Units are numbered
 // longest first (the last query tiles of a causal prefill see the most keys).
-__device__ __forceinline__ PfUnit pf_unit(const AttnParams &p, int idx) {
+__device__ __forceinline__ PfUnit pf_unit(const AttnParams &p, const PfDecode &d, int idx) {
     PfUnit u;
-    const int per = p.B * p.Hq;
-    const int qt = p.n_qtiles - 1 - idx / per;
-    const int rem = idx % per;
-    u.b = rem / p.Hq;
-    u.h_q = rem % p.Hq;
-    u.h_kv = u.h_q / p.G;
+    const int row = pf_div(idx, d.per, d.r_per);
+    const int qt = p.n_qtiles - 1 - row;
+    const int rem = idx - row * d.per;
+    u.b = pf_div(rem, p.Hq, d.r_hq);
+    u.h_q = rem - u.b * p.Hq;
+    u.h_kv = pf_div(u.h_q, p.G, d.r_g);
     u.q0 = qt * 128;
     const int R = imin(128, p.Sq - u.q0);
     const int L = p.seqlens ? p.seqlens[u.b] : p.Lk;
     u.L = imax(0, imin(L, p.kv_cap));
     int kv_end = u.L;
     if (p.causal) kv_end = imin(u.L, u.q0 + R + u.L - p.Sq);
-    u.T = kv_end > 0 ? (kv_end + 127) / 128 : 0;
+    u.T = kv_end > 0 ? (kv_end + 127) >> 7 : 0;
     return u;
 }
 
@@ -157,6 +192,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n_units = p.B * p.Hq * p.n_qtiles;
+    const PfDecode dc = pf_decode(p);
 
     // Softmax thread identity (warps 0..7): lane quarter, warp parity, row in the tile.
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
@@ -221,7 +257,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tmem_alloc(tmem_slot, kPfTmemCols);
         tmem_relinquish();
     }
-    if (!kStageQK && warp == kPfProducerWarp) {
+    if (!kStageQK && warp == kPfVWarp) {
         // Constant V rows: row 128 = 1.0 (E4M3 0x38), rows 129..143 = 0, and a
         // scale atom of 2^0 for them. TMA never writes these rows.
         for (int s = 0; s < kPfVStages; ++s)
@@ -240,95 +276,58 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kPfProducerWarp) {
-        // ---------------------------------------------------------------- producer
-        if (lane == 0) {
+        // ----------------------------------------------------------- Q/K producer
+        // One elected thread: each step is a probe of one barrier and three copy
+        // instructions, and this thread's pace bounds the QK^T stage's.
+        uint32_t pred;
+        asm volatile(
+            "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\tselp.u32 %0, 1, 0, e;\n\t}"
+            : "=r"(pred));
+        if (pred != 0) {
             prefetch_tensormap(&tmap_q);
             prefetch_tensormap(&tmap_k);
-            if (!kStageQK) prefetch_tensormap(&tmap_v);
-        }
-        const int nblk = p.kv_cap / 128;
-        int g = 0, c = 0;  // tiles and units so far (units with at least one tile)
-        int gk_issued = 0, gv_issued = 0, q_issued = 0;  // copies issued (global tile / unit counts)
-        bool ok = true;
-        for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
-            const PfUnit u = pf_unit(p, un);
-            const int T = u.T;
-            if (T <= 0) continue;
-            const int kvh = u.b * p.Hkv + u.h_kv;
-            const int qb = c & 1;
-            // Q of this unit (TMA; rows past Sq are padding in the packed format) and
-            // its scale atom. The MMA warp frees the buffer after the unit's last QK^T.
-            ok = __all_sync(0xffffffffu, wait_bar(&q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status));
-            if (!ok) break;
-            if (lane == 0 && !(p.test_stall && c == 0)) {
-                const int qhead = u.b * p.Hq + u.h_q;
-                mbar_arrive_expect_tx(&q_full[qb], S::kQBytes + 512);
-                tma_load_3d(smem + S::kQ + qb * S::kQBytes, &tmap_q, 0, u.q0, qhead, &q_full[qb]);
-                bulk_load(smem + S::kSfQ + qb * 512,
-                          p.q_scales + (static_cast<int64_t>(qhead) * (p.q_cap / 128) + u.q0 / 128) * 512, 512,
-                          &q_full[qb]);
-            }
-            if (!(p.test_stall && c == 0)) q_issued = c + 1;
-            const bool last_partial = !kStageQK && (u.L & 127) != 0 && T == (u.L + 127) / 128;
-            // K runs one tile ahead of V: the K ring frees as soon as QK^T of a tile
-            // completes, the V ring only after its P V.
-            for (int it = 0; it <= T && ok; ++it) {
-                if (it < T) {
+            const int nblk = p.kv_cap / 128;
+            int g = 0, c = 0;  // tiles and units so far (units with at least one tile)
+            int gk_issued = 0, q_issued = 0;  // copies issued (global tile / unit counts)
+            bool ok = true;
+            for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
+                const PfUnit u = pf_unit(p, dc, un);
+                const int T = u.T;
+                if (T <= 0) continue;
+                const int kvh = u.b * p.Hkv + u.h_kv;
+                const int qb = c & 1;
+                // Q of this unit (TMA; rows past Sq are padding in the packed format)
+                // and its scale atom. The MMA warp frees the buffer after the unit's
+                // last QK^T.
+                const uint32_t qpar = ((c >> 1) & 1) ^ 1;
+                ok = mbar_test_wait(&q_empty[qb], qpar) || wait_bar(&q_empty[qb], qpar, abort_flag, p.status);
+                if (!ok) break;
+                if (!(p.test_stall && c == 0)) {
+                    const int qhead = u.b * p.Hq + u.h_q;
+                    mbar_arrive_expect_tx(&q_full[qb], S::kQBytes + 512);
+                    tma_load_3d(smem + S::kQ + qb * S::kQBytes, &tmap_q, 0, u.q0, qhead, &q_full[qb]);
+                    bulk_load(smem + S::kSfQ + qb * 512,
+                              p.q_scales + (static_cast<int64_t>(qhead) * (p.q_cap / 128) + u.q0 / 128) * 512, 512,
+                              &q_full[qb]);
+                    q_issued = c + 1;
+                }
+                // K tiles: the ring frees as soon as QK^T of a tile completes.
+                for (int it = 0; it < T; ++it) {
                     const int gk = g + it;
                     const int st = gk % kPfKStages;
-                    ok = __all_sync(0xffffffffu,
-                                    wait_bar(&k_empty[st], ((gk / kPfKStages) & 1) ^ 1, abort_flag, p.status));
+                    const uint32_t kpar = ((gk / kPfKStages) & 1) ^ 1;
+                    ok = mbar_test_wait(&k_empty[st], kpar) || wait_bar(&k_empty[st], kpar, abort_flag, p.status);
                     if (!ok) break;
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&k_full[st], S::kKBytes + 512);
-                        tma_load_3d(smem + S::kK + st * S::kKBytes, &tmap_k, 0, it * 128, kvh, &k_full[st]);
-                        bulk_load(smem + S::kSfK + st * 512,
-                                  p.k_scales + (static_cast<int64_t>(kvh) * nblk + it) * 512, 512, &k_full[st]);
-                    }
+                    mbar_arrive_expect_tx(&k_full[st], S::kKBytes + 512);
+                    tma_load_3d(smem + S::kK + st * S::kKBytes, &tmap_k, 0, it * 128, kvh, &k_full[st]);
+                    bulk_load(smem + S::kSfK + st * 512, p.k_scales + (static_cast<int64_t>(kvh) * nblk + it) * 512,
+                              512, &k_full[st]);
                     gk_issued = gk + 1;
                 }
-                const int jt = it - 1;  // V tile issued in this round
-                if (kStageQK || jt < 0) continue;
-                const int gv = g + jt;
-                const int sv = gv % kPfVStages;
-                const uint32_t ph = (gv / kPfVStages) & 1;
-                ok = __all_sync(0xffffffffu, wait_bar(&v_empty[sv], ph ^ 1, abort_flag, p.status));
-                if (!ok) break;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&v_full[sv], S::kVTmaBytes + 512);
-                    tma_load_3d(smem + S::kV + sv * S::kVBytes, &tmap_v, jt * 128, 0, kvh, &v_full[sv]);
-                    bulk_load(smem + S::kSfV + sv * 512, p.v_scales + (static_cast<int64_t>(kvh) * nblk + jt) * 512,
-                              512, &v_full[sv]);
-                }
-                gv_issued = gv + 1;
-                if (last_partial && jt == T - 1) {
-                    // Keys at or past L may hold anything (a reused buffer). Their P is
-                    // zero, but a NaN code or scale in V would still poison O: zero them
-                    // once the tile has landed, and tell the MMA warp.
-                    ok = __all_sync(0xffffffffu, wait_bar(&v_full[sv], ph, abort_flag, p.status));
-                    if (!ok) break;
-                    const int jv = u.L - jt * 128;  // valid keys in this tile, 1..127
-                    uint8_t *vt = smem + S::kV + sv * S::kVBytes;
-                    for (int cc = lane; cc < 128 * 8; cc += 32) {
-                        const int r = cc >> 3, q = cc & 7;
-                        if (16 * q + 16 <= jv) continue;
-                        uint8_t *chunk = vt + r * 128 + ((q ^ (r & 7)) << 4);
-                        for (int e = 0; e < 16; ++e)
-                            if (16 * q + e >= jv) chunk[e] = 0;
-                    }
-                    uint8_t *sfv = smem + S::kSfV + sv * 512;
-                    for (int r = lane; r < 128; r += 32)
-                        for (int gq = (jv + 31) / 32; gq < 4; ++gq) sfv[(r & 31) * 16 + (r >> 5) * 4 + gq] = 0;
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(patch);
-                }
+                g += T;
+                ++c;
             }
-            g += T;
-            ++c;
-        }
-        // Let every issued copy land before the CTA can retire.
-        if (lane == 0) {
+            // Let every issued copy land before the CTA can retire.
             auto settle = [&](uint64_t *bar, uint32_t parity) {
                 const uint64_t t0 = globaltimer_ns();
                 while (!mbar_try_wait(bar, parity))
@@ -336,10 +335,77 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             };
             for (int gk = imax(0, gk_issued - kPfKStages); gk < gk_issued; ++gk)
                 settle(&k_full[gk % kPfKStages], (gk / kPfKStages) & 1);
-            for (int gv = imax(0, gv_issued - kPfVStages); gv < gv_issued; ++gv)
-                settle(&v_full[gv % kPfVStages], (gv / kPfVStages) & 1);
             for (int cq = imax(0, q_issued - 2); cq < q_issued; ++cq) settle(&q_full[cq & 1], (cq >> 1) & 1);
         }
+        __syncwarp();
+    } else if (warp == kPfVWarp) {
+        // ------------------------------------------------------------- V producer
+        // One elected thread, like the Q/K producer: a whole warp waiting here
+        // takes issue slots from the softmax warps that share its scheduler.
+        uint32_t pred;
+        asm volatile(
+            "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\tselp.u32 %0, 1, 0, e;\n\t}"
+            : "=r"(pred));
+        if (!kStageQK && pred != 0) {
+            prefetch_tensormap(&tmap_v);
+            const int nblk = p.kv_cap / 128;
+            int g = 0;
+            int gv_issued = 0;
+            bool ok = true;
+            for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
+                const PfUnit u = pf_unit(p, dc, un);
+                const int T = u.T;
+                if (T <= 0) continue;
+                const int kvh = u.b * p.Hkv + u.h_kv;
+                const bool last_partial = (u.L & 127) != 0 && T == (u.L + 127) / 128;
+                // V tiles: the ring frees only after P V of a tile.
+                for (int jt = 0; jt < T && ok; ++jt) {
+                    const int gv = g + jt;
+                    const int sv = gv % kPfVStages;
+                    const uint32_t ph = (gv / kPfVStages) & 1;
+                    ok = mbar_test_wait(&v_empty[sv], ph ^ 1) || wait_bar(&v_empty[sv], ph ^ 1, abort_flag, p.status);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&v_full[sv], S::kVTmaBytes + 512);
+                    tma_load_3d(smem + S::kV + sv * S::kVBytes, &tmap_v, jt * 128, 0, kvh, &v_full[sv]);
+                    bulk_load(smem + S::kSfV + sv * 512, p.v_scales + (static_cast<int64_t>(kvh) * nblk + jt) * 512,
+                              512, &v_full[sv]);
+                    gv_issued = gv + 1;
+                    if (last_partial && jt == T - 1) {
+                        // Keys at or past L may hold anything (a reused buffer). Their P
+                        // is zero, but a NaN code or scale in V would still poison O:
+                        // zero them once the tile has landed, and tell the MMA warp.
+                        ok = wait_bar(&v_full[sv], ph, abort_flag, p.status);
+                        if (!ok) break;
+                        const int jv = u.L - jt * 128;  // valid keys in this tile, 1..127
+                        uint8_t *vt = smem + S::kV + sv * S::kVBytes;
+                        const int q0 = jv >> 4;  // 16-byte chunk (of each channel row) holding key jv
+                        for (int r = 0; r < 128; ++r) {
+                            for (int q = q0; q < 8; ++q) {
+                                uint8_t *chunk = vt + r * 128 + ((q ^ (r & 7)) << 4);
+                                if (16 * q >= jv) {
+                                    *reinterpret_cast<uint4 *>(chunk) = make_uint4(0, 0, 0, 0);
+                                } else {
+                                    for (int e = jv - 16 * q; e < 16; ++e) chunk[e] = 0;
+                                }
+                            }
+                        }
+                        uint8_t *sfv = smem + S::kSfV + sv * 512;
+                        for (int r = 0; r < 128; ++r)
+                            for (int gq = (jv + 31) / 32; gq < 4; ++gq) sfv[(r & 31) * 16 + (r >> 5) * 4 + gq] = 0;
+                        fence_proxy_async_smem();
+                        mbar_arrive(patch);
+                    }
+                }
+                g += T;
+            }
+            // Let every issued copy land before the CTA can retire.
+            for (int gv = imax(0, gv_issued - kPfVStages); gv < gv_issued; ++gv) {
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(&v_full[gv % kPfVStages], (gv / kPfVStages) & 1))
+                    if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
+            }
+        }
+        __syncwarp();
     } else if (warp == kPfMmaWarp) {
         // -------------------------------------------------------------- MMA issuer
         // Every tcgen05 instruction of this role (copies of scale atoms, MMAs,
@@ -373,12 +439,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             int g = 0, c = 0, n_patch = 0;
             // The next unit's description is worked out while this unit's first S
             // computes, off the issue path of the unit transition.
-            PfUnit nu = pf_unit(p, blockIdx.x);
+            PfUnit nu = pf_unit(p, dc, blockIdx.x);
             for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
                 const PfUnit u = nu;
                 const int T = u.T;
                 if (T <= 0) {
-                    if (un + static_cast<int>(gridDim.x) < n_units) nu = pf_unit(p, un + gridDim.x);
+                    if (un + static_cast<int>(gridDim.x) < n_units) nu = pf_unit(p, dc, un + gridDim.x);
                     continue;
                 }
                 const int qb = c & 1;
@@ -465,7 +531,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 // P V.
                 ok = issue_qk(0);
                 if (ok && T > 1) ok = issue_qk(1);
-                if (un + static_cast<int>(gridDim.x) < n_units) nu = pf_unit(p, un + gridDim.x);
+                if (un + static_cast<int>(gridDim.x) < n_units) nu = pf_unit(p, dc, un + gridDim.x);
                 for (int i = 0; i < T && ok; ++i) {
                     if (i + 2 < T) ok = issue_qk(i + 2);
                     if (ok && !kStageQK && i >= 1) ok = issue_pv(i - 1);
@@ -500,7 +566,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int g = 0, c = 0;  // tiles and units so far (units with at least one tile)
         bool ok = true;
         for (int un = blockIdx.x; un < n_units && ok; un += gridDim.x) {
-            const PfUnit u = pf_unit(p, un);
+            const PfUnit u = pf_unit(p, dc, un);
             const int T = u.T;
             const int qi = u.q0 + row;
             const bool row_valid = qi < p.Sq;
