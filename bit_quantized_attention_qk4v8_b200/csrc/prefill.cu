@@ -90,8 +90,11 @@ struct PfSmem {
     // (tile parity 0 only) the reference m_O.
     static constexpr int kHsE = kSfOne + 512;                      // int [4][2][32]
     static constexpr int kHsM = kHsE + 4 * 2 * 32 * 4;             // float [4][2][32]
-    static constexpr int kXmax = kHsM + 4 * 2 * 32 * 4;            // float [unit parity][warp parity][128] (QK stage)
-    static constexpr int kBar = kXmax + 2 * 2 * 128 * 4;
+    // QK stage: row maxima [unit slot][warp parity][128] and arrival counters
+    // [quarter][unit slot]; 8 unit slots, more than one parity can lead the other.
+    static constexpr int kXmax = kHsM + 4 * 2 * 32 * 4;
+    static constexpr int kXcnt = kXmax + 8 * 2 * 128 * 4;
+    static constexpr int kBar = kXcnt + 4 * 8 * 4;
     // k_full/k_empty, v_full/v_empty per stage; q_full/q_empty per Q buffer;
     // patch; s_full, s_free, p_full, pv_done per parity; o_full, o_free, drain;
     // handshake [4 quarters][2]; m_O handshake [4 quarters]; unit end [4 quarters].
@@ -248,6 +251,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mbar_init(&mo_bar[g], 1);
             mbar_init(&ue_bar[g], 2);
         }
+        if (kStageQK)
+            for (int i = 0; i < 4 * 8; ++i) reinterpret_cast<int *>(smem + S::kXcnt)[i] = 0;
         // A status already set by another launch or CTA: unwind at once (every
         // wait returns false), uniformly for the whole CTA.
         *abort_flag = (p.status && *reinterpret_cast<const volatile int32_t *>(p.status) != 0) ? 1u : 0u;
@@ -561,6 +566,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         uint64_t *hs = hs_bar + quarter * 2;
         uint8_t *pbuf = smem + S::kP + pp * S::kPBuf;
         float *xmax = reinterpret_cast<float *>(smem + S::kXmax);
+        int *xcnt = reinterpret_cast<int *>(smem + S::kXcnt);
         const int swz = row & 7;
         const float sc = p.scale_log2;
         int g = 0, c = 0;  // tiles and units so far (units with at least one tile)
@@ -780,7 +786,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
             // -------------------------------------------------------------- epilogue
             if (kStageQK) {
-                xmax[((c & 1) * 2 + pp) * 128 + row] = qk_rowmax;
+                // Each warp of the quarter posts its rows' maxima; the second to arrive
+                // combines the two and writes them, so neither waits for the other.
+                // A parity runs at most a few tiles (so units) ahead of the other,
+                // well within the 8 slots.
+                const int slot = c & 7;
+                xmax[(slot * 2 + pp) * 128 + row] = qk_rowmax;
+                __threadfence_block();
+                __syncwarp();
+                int second = 0;
+                if (lane == 0) second = atomicAdd(&xcnt[quarter * 8 + slot], 1);
+                second = __shfl_sync(0xffffffffu, second, 0);
+                if (second) {
+                    __threadfence_block();
+                    const float m = fmaxf(xmax[(slot * 2) * 128 + row], xmax[(slot * 2 + 1) * 128 + row]);
+                    if (row_valid && p.lse) p.lse[(static_cast<int64_t>(u.b) * p.Hq + u.h_q) * p.Sq + qi] = m;
+                    __syncwarp();
+                    if (lane == 0) xcnt[quarter * 8 + slot] = 0;
+                }
+                g += T;
+                ++c;
+                continue;
             } else {
                 ok = __all_sync(0xffffffffu, wait_bar(o_full, c & 1, abort_flag, p.status));
                 if (!ok) break;
@@ -819,15 +845,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(o_free);  // the next unit's first P V may overwrite O
             }
-            // Both warps of the quarter are done with this unit (its handshake slots,
-            // and in the QK stage its row maxima).
+            // Both warps of the quarter are done with this unit (its handshake slots).
             __syncwarp();
             if (lane == 0) mbar_arrive(&ue_bar[quarter]);
             ok = __all_sync(0xffffffffu, wait_bar(&ue_bar[quarter], c & 1, abort_flag, p.status));
             if (!ok) break;
-            if (kStageQK && pp == 0 && row_valid && p.lse)
-                p.lse[(static_cast<int64_t>(u.b) * p.Hq + u.h_q) * p.Sq + qi] =
-                    fmaxf(xmax[((c & 1) * 2) * 128 + row], xmax[((c & 1) * 2 + 1) * 128 + row]);
             g += T;
             ++c;
         }
