@@ -90,6 +90,7 @@ def test_scores_tile_matches_dequantized_dot_products():
     (2, 128, 4, 1, False),     # non-causal, GQA 4
     (1, 384, 8, 2, True),      # several key tiles
     (1, 1, 1, 1, True),        # a single token
+    (4, 256, 64, 8, True),     # 512 units: several per CTA, Q buffers and the K and V rings reused across units
 ])
 def test_prefill_parity(B, S, Hq, Hkv, causal):
     gen = make_gen(B, S, S, Hq, Hkv, seed=S + Hq)
@@ -252,6 +253,10 @@ def dequantized_scores(qp, kp, Sq, Lk):
     (1, 384, 4, 2, True, None),
     (2, 200, 2, 1, False, [200, 77]),
     (2, 130, 2, 2, True, [130, 0]),
+    # several units per CTA (512 units on at most 148 CTAs), of one and two key
+    # tiles, so the two tile parities of a CTA drift apart across units
+    (4, 256, 64, 8, True, None),
+    (8, 256, 32, 8, False, [256, 1, 129, 128, 0, 77, 255, 3]),
 ])
 def test_prefill_stage_qk_row_max(B, S, Hq, Hkv, causal, lens):
     """The QK^T-stage build: each row's largest allowed scaled score, exactly as the scores' max."""
