@@ -21,46 +21,75 @@ namespace qk4v8 {
 // ------------------------------------------------------------------ MXFP4
 
 // 16 lanes per token row (128 channels), 8 channels per lane, 4 lanes per group
-// of 32. Rows are visited in input order (b, t, h) so loads are contiguous.
-// Tokens 0 .. row_len-1 of each sequence are visited: row_len = cap writes the
-// whole capacity (zero codes and scales past the valid length), row_len = S
-// only the rows of the input.
+// of 32; a warp takes two rows per step, each half-warp one. blockIdx.y is the
+// batch entry; its rows (t, h) are visited in input order (t major), so loads
+// are contiguous. Tokens 0 .. row_len-1 of each sequence are visited: row_len =
+// cap writes the whole capacity (zero codes and scales past the valid length),
+// row_len = S only the rows of the input. Each half-warp steps its (t, h)
+// position by a fixed amount and keeps two rows in flight: the kernel is meant
+// to be bound by memory, and an integer division per row would make it bound by
+// instruction issue instead.
+__device__ __forceinline__ void qk_store_row(uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int64_t head,
+                                             int cap, int t, int sub, uint32_t packed, int X, bool valid) {
+    reinterpret_cast<uint32_t *>(codes + (head * cap + t) * 64)[sub] = packed;
+    if ((sub & 3) == 0) {
+        const int g = sub >> 2;
+        uint8_t *blk = scales + (head * (cap / 128) + t / 128) * 512;
+        blk[(t & 31) * 16 + ((t & 127) >> 5) * 4 + g] = valid ? static_cast<uint8_t>(X + 127) : 0;
+    }
+}
+
 __global__ void __launch_bounds__(256) quantize_qk_kernel(const __nv_bfloat16 *__restrict__ x, int B, int S, int H,
                                                           int64_t sb, int64_t ss, int64_t sh,
                                                           const int32_t *__restrict__ seqlens, int cap,
                                                           int row_len, uint8_t *__restrict__ codes,
                                                           uint8_t *__restrict__ scales) {
     const int sub = threadIdx.x & 15;  // lane within the row
-    const int64_t n_rows = static_cast<int64_t>(B) * row_len * H;
-    const int64_t row_step = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 4);
+    const int hw = (threadIdx.x >> 4) & 1;
+    const int b = blockIdx.y;
+    const int rows = row_len * H;  // rows of this batch entry (the launcher keeps this below 2^30)
+    int valid_len = S;
+    if (seqlens) {
+        const int L = seqlens[b];
+        valid_len = L < valid_len ? L : valid_len;
+    }
+    const int step = static_cast<int>(gridDim.x) * (blockDim.x >> 5) * 2;  // rows per grid step
+    const int step_t = step / H, step_h = step - step_t * H;
     // The loop bound is taken per warp (two rows) so every lane reaches the shuffles.
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 4) + ((threadIdx.x >> 5) << 1);
-         base < n_rows; base += row_step) {
-        const int64_t row_raw = base + ((threadIdx.x >> 4) & 1);
-        const bool in_range = row_raw < n_rows;
-        const int64_t row = in_range ? row_raw : base;
-        const int h = static_cast<int>(row % H);
-        const int64_t bt = row / H;
-        const int t = static_cast<int>(bt % row_len);
-        const int b = static_cast<int>(bt / row_len);
-        int valid_len = S;
-        if (seqlens) {
-            int L = seqlens[b];
-            valid_len = L < valid_len ? L : valid_len;
+    int base = (static_cast<int>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 2;
+    int t = (base + hw) / H;
+    int h = (base + hw) - t * H;
+    const __nv_bfloat16 *xb = x + b * sb;
+    const int64_t head_b = static_cast<int64_t>(b) * H;
+    auto advance = [&](int &tt, int &hh) {
+        tt += step_t;
+        hh += step_h;
+        if (hh >= H) {
+            hh -= H;
+            ++tt;
         }
-        const bool valid = in_range && t < valid_len;
-        uint4 raw = make_uint4(0, 0, 0, 0);
-        if (valid) raw = *reinterpret_cast<const uint4 *>(x + b * sb + t * ss + h * sh + sub * 8);
-        int X;
-        const uint32_t packed = mxfp4_encode8(raw, valid, X);
-        if (!in_range) continue;
-        const int64_t head = static_cast<int64_t>(b) * H + h;
-        reinterpret_cast<uint32_t *>(codes + (head * cap + t) * 64)[sub] = packed;
-        if ((sub & 3) == 0) {
-            const int g = sub >> 2;
-            uint8_t *blk = scales + (head * (cap / 128) + t / 128) * 512;
-            blk[(t & 31) * 16 + ((t & 127) >> 5) * 4 + g] = valid ? static_cast<uint8_t>(X + 127) : 0;
+    };
+    for (; base < rows; base += 2 * step) {
+        // Two rows of this half-warp: base + hw and base + hw + step.
+        int t1 = t, h1 = h;
+        advance(t1, h1);
+        const bool in0 = base + hw < rows, in1 = base + step + hw < rows;
+        const bool v0 = in0 && t < valid_len, v1 = in1 && t1 < valid_len;
+        uint4 raw0 = make_uint4(0, 0, 0, 0), raw1 = make_uint4(0, 0, 0, 0);
+        if (v0) raw0 = *reinterpret_cast<const uint4 *>(xb + t * ss + h * sh + sub * 8);
+        if (v1) raw1 = *reinterpret_cast<const uint4 *>(xb + t1 * ss + h1 * sh + sub * 8);
+        int X0, X1;
+        const uint32_t p0 = mxfp4_encode8(raw0, v0, X0);
+        if (in0) qk_store_row(codes, scales, head_b + h, cap, t, sub, p0, X0, v0);
+        // The second pair of rows is encoded by the whole warp too (shuffles),
+        // when the warp's first row of it exists.
+        if (base + step < rows) {
+            const uint32_t p1 = mxfp4_encode8(raw1, v1, X1);
+            if (in1) qk_store_row(codes, scales, head_b + h1, cap, t1, sub, p1, X1, v1);
         }
+        t = t1;
+        h = h1;
+        advance(t, h);
     }
 }
 
@@ -156,13 +185,16 @@ cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, i
                                const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
                                cudaStream_t stream, bool pad_to_cap) {
     const int row_len = pad_to_cap ? cap : S;
-    const int64_t rows = static_cast<int64_t>(B) * row_len * H;
-    const int rows_per_cta = 256 / 16;
-    int64_t grid = (rows + rows_per_cta - 1) / rows_per_cta;
-    const int64_t max_grid = 148 * 16;
-    if (grid > max_grid) grid = max_grid;
-    if (grid < 1) grid = 1;
-    quantize_qk_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+    const int64_t rows = static_cast<int64_t>(row_len) * H;  // per batch entry
+    if (rows >= (int64_t{1} << 30) || B > 65535) return cudaErrorInvalidValue;
+    // About one wave over all batch entries: 6 CTAs (48 warps, 40 registers a
+    // thread) per SM, each warp with two pairs of rows in flight.
+    const int64_t rows_per_cta = 256 / 16;
+    int64_t gx = (rows + rows_per_cta - 1) / rows_per_cta;
+    const int64_t wave = (148 * 6 + B - 1) / B;
+    if (gx > wave) gx = wave;
+    if (gx < 1) gx = 1;
+    quantize_qk_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(B)), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(x), B, S, H, sb, ss, sh, seqlens, cap, row_len, codes, scales);
     return cudaGetLastError();
 }
