@@ -27,8 +27,9 @@
 //     further power of two 2^-x, also in its scale byte: 127 + e + x.
 //   - If some e passes 2^64, the tile's owner scales the row of O by 2^-E
 //     (after P V of the previous tile, before its own) and lowers e by E.
-//     The owner of the next tile learns E (and, after tile 0, m_O) through a
-//     one-way handshake posted early in each tile.
+//     The owner of the next tile learns E through a one-way handshake
+//     posted at the end of each tile, and m_O through one posted early in the
+//     unit's first tile.
 // P is kept as two E4M3 terms with the same scales: P_hi = E4M3(p) and
 // P_lo = E4M3(p - P_hi), about 8 significant bits. V carries an extra row of
 // ones, so O column 128 accumulates the softmax denominator sum(P_hi + P_lo)
