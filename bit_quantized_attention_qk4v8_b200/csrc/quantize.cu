@@ -186,7 +186,7 @@ cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, i
                                cudaStream_t stream, bool pad_to_cap) {
     const int row_len = pad_to_cap ? cap : S;
     const int64_t rows = static_cast<int64_t>(row_len) * H;  // per batch entry
-    if (rows >= (int64_t{1} << 30) || B > 65535) return cudaErrorInvalidValue;
+    if (rows >= (int64_t{1} << 30)) return cudaErrorInvalidValue;
     // About one wave over all batch entries: 6 CTAs (48 warps, 40 registers a
     // thread) per SM, each warp with two pairs of rows in flight.
     const int64_t rows_per_cta = 256 / 16;
@@ -194,9 +194,18 @@ cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, i
     const int64_t wave = (148 * 6 + B - 1) / B;
     if (gx > wave) gx = wave;
     if (gx < 1) gx = 1;
-    quantize_qk_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(B)), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(x), B, S, H, sb, ss, sh, seqlens, cap, row_len, codes, scales);
-    return cudaGetLastError();
+    // The grid's y extent is at most 65535: larger batches go in chunks.
+    const int64_t codes_per_b = static_cast<int64_t>(H) * cap * 64;
+    const int64_t scales_per_b = static_cast<int64_t>(H) * (cap / 128) * 512;
+    for (int b0 = 0; b0 < B; b0 += 65535) {
+        const int nb = B - b0 < 65535 ? B - b0 : 65535;
+        quantize_qk_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(nb)), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16 *>(x) + b0 * sb, nb, S, H, sb, ss, sh, seqlens ? seqlens + b0 : nullptr,
+            cap, row_len, codes + b0 * codes_per_b, scales + b0 * scales_per_b);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t launch_quantize_v(const void *v, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
