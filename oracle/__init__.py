@@ -64,6 +64,16 @@ def _load():
         lib.oracle_attention.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                          ctypes.c_double, vp, i64, vp, vp]
         lib.oracle_attention.restype = i32
+        lib.oracle_attention_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                                ctypes.c_double, vp, i64, vp, vp]
+        lib.oracle_attention_window.restype = i32
+        lib.oracle_hadamard_rows.argtypes = [vp, i64, vp]
+        lib.oracle_hadamard_rows.restype = i32
+        lib.oracle_quantize_rows_f32.argtypes = [vp, i64, i64, vp, i32, vp, vp]
+        lib.oracle_quantize_rows_f32.restype = i32
+        lib.oracle_attention_ref.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                             ctypes.c_double, vp, i64, vp, vp]
+        lib.oracle_attention_ref.restype = i32
         lib.oracle_num_threads.restype = i32
         _lib = lib
     return _lib
@@ -146,12 +156,14 @@ def quantize_v(v_bits: np.ndarray, seqlens=None):
     return quantize_rows(vt, E4M3, valid)
 
 
-def attention(qc, qs, kc, ks, vc, vs, seqlens=None, causal=True, scale=None, sel=None):
+def attention(qc, qs, kc, ks, vc, vs, seqlens=None, causal=True, scale=None, sel=None, window=0):
     """fp64 attention over the dequantized MX tensors.
 
     qc/qs [B,Hq,Sq,d]/[B,Hq,Sq,d/32]; kc/ks [B,Hkv,Lk,d]/[B,Hkv,Lk,d/32];
     vc/vs [B,Hkv,d,Lk]/[B,Hkv,d,ceil(Lk/32)].
     sel: int32 [n,3] rows (b, h_q, i) or None for all rows.
+    window > 0: each row sees only the last `window` keys before the query
+    block and the block itself (the C function's visible_keys rule).
     Returns (out, lse): out [B,Sq,Hq,d] and lse [B,Sq,Hq] when sel is None,
     else out [n,d] and lse [n].
     """
@@ -162,23 +174,109 @@ def attention(qc, qs, kc, ks, vc, vs, seqlens=None, causal=True, scale=None, sel
         scale = 1.0 / math.sqrt(d)
     arrs = [np.ascontiguousarray(a, dtype=np.uint8) for a in (qc, qs, kc, ks, vc, vs)]
     sl = None if seqlens is None else np.ascontiguousarray(seqlens, dtype=np.int32)
-    if sel is None:
-        n = B * Sq * Hq
-        selp = None
-    else:
-        sela = np.ascontiguousarray(sel, dtype=np.int32).reshape(-1, 3)
-        n = sela.shape[0]
-        selp = sela.ctypes.data
+    n, selp, sela = _selection(sel, B * Sq * Hq)
     out = np.empty((n, d), dtype=np.float64)
     lse = np.empty((n,), dtype=np.float64)
-    rc = lib.oracle_attention(*[a.ctypes.data for a in arrs], sl.ctypes.data if sl is not None else None,
-                              B, Hq, Hkv, Sq, Lk, d, int(bool(causal)), float(scale), selp, n,
-                              out.ctypes.data, lse.ctypes.data)
+    rc = lib.oracle_attention_window(*[a.ctypes.data for a in arrs], sl.ctypes.data if sl is not None else None,
+                                     B, Hq, Hkv, Sq, Lk, d, int(bool(causal)), int(window), float(scale), selp, n,
+                                     out.ctypes.data, lse.ctypes.data)
     if rc != 0:
-        raise RuntimeError(f"oracle_attention failed ({rc})")
+        raise RuntimeError(f"oracle_attention_window failed ({rc})")
     if sel is None:
         return out.reshape(B, Sq, Hq, d), lse.reshape(B, Sq, Hq)
     return out, lse
+
+
+def _selection(sel, n_all):
+    if sel is None:
+        return n_all, None, None
+    sela = np.ascontiguousarray(sel, dtype=np.int32).reshape(-1, 3)
+    return sela.shape[0], sela.ctypes.data, sela
+
+
+def attention_ref(q, k, v, seqlens=None, causal=True, scale=None, sel=None, window=0):
+    """fp64 softmax attention over UNQUANTIZED inputs (the context reference).
+
+    q [B,Sq,Hq,d], k and v [B,Lk,Hkv,d]: float32 arrays, or uint16 bf16 bit
+    patterns (converted exactly). Masking as for `attention`. Returns (out,
+    lse) shaped like `attention`'s.
+    """
+    lib = _load()
+    q, k, v = (_as_f32(t) for t in (q, k, v))
+    B, Sq, Hq, d = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    sl = None if seqlens is None else np.ascontiguousarray(seqlens, dtype=np.int32)
+    n, selp, sela = _selection(sel, B * Sq * Hq)
+    out = np.empty((n, d), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    rc = lib.oracle_attention_ref(q.ctypes.data, k.ctypes.data, v.ctypes.data,
+                                  sl.ctypes.data if sl is not None else None, B, Hq, Hkv, Sq, Lk, d,
+                                  int(bool(causal)), int(window), float(scale), selp, n, out.ctypes.data,
+                                  lse.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_ref failed ({rc})")
+    if sel is None:
+        return out.reshape(B, Sq, Hq, d), lse.reshape(B, Sq, Hq)
+    return out, lse
+
+
+def _as_f32(t):
+    """float32 array as is; uint16 bf16 bit patterns widened to float32 (a bit shift, exact)."""
+    t = np.asarray(t)
+    if t.dtype == np.uint16:
+        return np.ascontiguousarray((t.astype(np.uint32) << 16).view(np.float32))
+    return np.ascontiguousarray(t, dtype=np.float32)
+
+
+def hadamard_rows(x_bits: np.ndarray) -> np.ndarray:
+    """Rotation of 128-channel rows (bf16 bits [..., 128]) by H/sqrt(128), in fp32 (oracle.c)."""
+    lib = _load()
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    if x.shape[-1] != 128:
+        raise ValueError("rows of 128 channels")
+    y = np.empty(x.shape, dtype=np.float32)
+    if lib.oracle_hadamard_rows(x.ctypes.data, x.size // 128, y.ctypes.data) != 0:
+        raise RuntimeError("oracle_hadamard_rows failed")
+    return y
+
+
+def quantize_rows_f32(x: np.ndarray, fmt: int, valid=None):
+    """quantize_rows for float32 values (last axis, groups of 32)."""
+    lib = _load()
+    xf = np.ascontiguousarray(x, dtype=np.float32)
+    n_cols = xf.shape[-1]
+    ng = (n_cols + 31) // 32
+    codes = np.empty(xf.shape, dtype=np.uint8)
+    scales = np.empty(xf.shape[:-1] + (ng,), dtype=np.uint8)
+    vv = None
+    if valid is not None:
+        vv = np.ascontiguousarray(np.broadcast_to(valid, xf.shape[:-1]), dtype=np.int32)
+    rc = lib.oracle_quantize_rows_f32(xf.ctypes.data, xf.size // n_cols, n_cols,
+                                      vv.ctypes.data if vv is not None else None, fmt, codes.ctypes.data,
+                                      scales.ctypes.data)
+    if rc != 0:
+        raise RuntimeError("oracle_quantize_rows_f32 failed")
+    return codes, scales
+
+
+def quantize_qk_hadamard(x_bits: np.ndarray, seqlens=None):
+    """MXFP4 quantization of Hadamard-rotated Q or K, bf16 bits [B, T, H, d].
+
+    Each (token, head) row is rotated by H/sqrt(128) in fp32 and then
+    quantized like quantize_qk. Tokens at or past seqlens[b] (when given) get
+    zero codes and scales. Returns codes [B, H, T, d] and scales [B, H, T, d/32].
+    """
+    xt = np.ascontiguousarray(np.transpose(x_bits, (0, 2, 1, 3)))
+    y = hadamard_rows(xt)
+    valid = None
+    if seqlens is not None:
+        B, H, T, d = xt.shape
+        lens = np.asarray(seqlens, dtype=np.int64)
+        valid = np.where(np.arange(T)[None, None, :] < lens[:, None, None], d, 0).astype(np.int32)
+        valid = np.broadcast_to(valid, (B, H, T))
+    return quantize_rows_f32(y, E2M1, valid)
 
 
 def quantize_workload(gen: dict):

@@ -183,20 +183,48 @@ int oracle_dequantize_rows(const uint8_t *codes, const uint8_t *scales, int64_t 
 }
 
 /*
+ * Keys visible to query row i (of Sq) of a sequence of L keys: lo <= j < hi.
+ *   hi = L, or with causal = 1, min(L, i + (L - Sq) + 1): bottom-right
+ *        alignment, so the Sq queries are the last Sq positions;
+ *   lo = 0, or with window > 0, max(0, L - Sq - window): the draft-block
+ *        attention of the MiMo DFlash article (section "DFlash块扩散推测解码")
+ *        uses sliding-window attention over the most recent 1024 context
+ *        tokens; the reading taken is that every row of the block sees the
+ *        last `window` keys before the block and all keys of the block.
+ */
+static void visible_keys(int L, int Sq, int i, int causal, int window, int *lo, int *hi) {
+    int h = L;
+    if (causal) {
+        int lim = i + (L - Sq) + 1;
+        if (lim < h) h = lim;
+    }
+    if (h < 0) h = 0;
+    int l = 0;
+    if (window > 0) {
+        l = L - Sq - window;
+        if (l < 0) l = 0;
+    }
+    if (l > h) l = h;
+    *lo = l;
+    *hi = h;
+}
+
+/*
  * Attention over the dequantized tensors, in fp64.
  *
  * qc, qs  [B][Hq][Sq][d] codes, [B][Hq][Sq][d/32] scales   (E2M1)
  * kc, ks  [B][Hkv][Lk][d] codes, [B][Hkv][Lk][d/32] scales (E2M1)
  * vc, vs  [B][Hkv][d][Lk] codes, [B][Hkv][d][ceil(Lk/32)] scales (E4M3)
  * seqlens [B] KV length per sequence (NULL: Lk)
+ * causal, window  the visible keys of each row (visible_keys above)
  * sel     [n_sel][3] rows (b, h_q, i) to compute; NULL computes every row in
  *         (b, i, h_q) order, n_sel = B*Sq*Hq
  * out     [n_sel][d]; lse [n_sel] natural-log log-sum-exp of the scaled scores
  */
-int oracle_attention(const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, const uint8_t *ks,
-                     const uint8_t *vc, const uint8_t *vs, const int32_t *seqlens,
-                     int B, int Hq, int Hkv, int Sq, int Lk, int d, int causal, double scale,
-                     const int32_t *sel, int64_t n_sel, double *out, double *lse) {
+int oracle_attention_window(const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, const uint8_t *ks,
+                            const uint8_t *vc, const uint8_t *vs, const int32_t *seqlens,
+                            int B, int Hq, int Hkv, int Sq, int Lk, int d, int causal, int window, double scale,
+                            const int32_t *sel, int64_t n_sel, double *out, double *lse) {
     if (d % 32 || Hkv <= 0 || Hq % Hkv) return -1;
     const int G = Hq / Hkv;
     const int dg = d / 32;
@@ -230,7 +258,7 @@ int oracle_attention(const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, co
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t u = 0; u < n_units; ++u) {
         if (cnt[u + 1] == cnt[u]) continue;
-        const int b = (int)(u / Hkv), hk = (int)(u % Hkv);
+        const int b = (int)(u / Hkv);
         int L = seqlens ? seqlens[b] : Lk;
         if (L > Lk) L = Lk;
         if (L < 0) L = 0;
@@ -262,20 +290,16 @@ int oracle_attention(const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, co
             const int64_t qrow = (((int64_t)b * Hq + h) * Sq + i);
             for (int c = 0; c < d; ++c)
                 qd[c] = ldexp(oracle_decode(ORACLE_E2M1, qc[qrow * d + c]), (int)qs[qrow * dg + c / 32] - 127);
-            int jmax = L; /* exclusive bound on allowed keys */
-            if (causal) {
-                int lim = i + (L - Sq) + 1;
-                if (lim < jmax) jmax = lim;
-            }
-            if (jmax < 0) jmax = 0;
+            int jmin, jmax; /* allowed keys: jmin <= j < jmax */
+            visible_keys(L, Sq, i, causal, window, &jmin, &jmax);
             double *o = out + r * d;
-            if (jmax == 0) {
+            if (jmax <= jmin) {
                 for (int c = 0; c < d; ++c) o[c] = 0.0;
                 if (lse) lse[r] = -INFINITY;
                 continue;
             }
             double m = -INFINITY;
-            for (int j = 0; j < jmax; ++j) {
+            for (int j = jmin; j < jmax; ++j) {
                 double s = 0.0;
                 const double *kr = kd + (int64_t)j * d;
                 for (int c = 0; c < d; ++c) s += qd[c] * kr[c];
@@ -284,9 +308,9 @@ int oracle_attention(const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, co
                 if (s > m) m = s;
             }
             double l = 0.0;
-            for (int j = 0; j < jmax; ++j) { p[j] = exp(p[j] - m); l += p[j]; }
+            for (int j = jmin; j < jmax; ++j) { p[j] = exp(p[j] - m); l += p[j]; }
             for (int c = 0; c < d; ++c) o[c] = 0.0;
-            for (int j = 0; j < jmax; ++j) {
+            for (int j = jmin; j < jmax; ++j) {
                 const double w = p[j] / l;
                 const double *vr = vd + (int64_t)j * d;
                 for (int c = 0; c < d; ++c) o[c] += w * vr[c];
@@ -297,6 +321,163 @@ int oracle_attention(const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, co
     }
     free(cnt);
     free(order);
+    return err;
+}
+
+/* oracle_attention_window with no window: every key up to the causal bound. */
+int oracle_attention(const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, const uint8_t *ks,
+                     const uint8_t *vc, const uint8_t *vs, const int32_t *seqlens,
+                     int B, int Hq, int Hkv, int Sq, int Lk, int d, int causal, double scale,
+                     const int32_t *sel, int64_t n_sel, double *out, double *lse) {
+    return oracle_attention_window(qc, qs, kc, ks, vc, vs, seqlens, B, Hq, Hkv, Sq, Lk, d, causal, 0, scale, sel,
+                                   n_sel, out, lse);
+}
+
+/*
+ * Hadamard rotation of 128-channel rows before MXFP4 quantization.
+ *
+ * The MpFA article (section 3.1, and the outlier discussion of section 2.1)
+ * expects outlier channels to be handled by a light rotation applied per group
+ * before the 4-bit quantization. Q.K^T is unchanged by an orthonormal rotation
+ * R applied to both Q and K, because (qR).(kR) = q R R^T k^T = q.k.
+ * Reading taken: R = H / sqrt(128) with H the 128 x 128 Sylvester Hadamard
+ * matrix, H[i][j] = (-1)^popcount(i & j), applied to each (token, head) row
+ * of 128 channels, so that one outlier channel is spread over all four MX
+ * groups of the row.
+ *
+ * The rotated values decide the quantized codes, so they are computed in the
+ * precision the GPU kernel uses: fp32, as the fast Walsh-Hadamard transform
+ * (butterfly stages of stride 1, 2, 4, ..., 64; each stage maps the pair
+ * (a, b) at indices (i, i + stride) to (a + b, a - b)), then one fp32 multiply
+ * by the fp32 value nearest to 2^-3.5 = 1/sqrt(128).
+ * x  [n_rows][128] bf16 bit patterns;  y  [n_rows][128] fp32.
+ */
+#define ORACLE_RSQRT128_F32 0x1.6a09e6p-4f
+
+int oracle_hadamard_rows(const uint16_t *x, int64_t n_rows, float *y) {
+    if (!x || !y || n_rows < 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        float *yr = y + r * 128;
+        for (int c = 0; c < 128; ++c) {
+            uint32_t u = (uint32_t)x[r * 128 + c] << 16;
+            memcpy(&yr[c], &u, 4);
+        }
+        for (int stride = 1; stride < 128; stride *= 2)
+            for (int i = 0; i < 128; ++i) {
+                if (i & stride) continue;
+                const float a = yr[i], b = yr[i + stride];
+                yr[i] = a + b;
+                yr[i + stride] = a - b;
+            }
+        for (int c = 0; c < 128; ++c) yr[c] = yr[c] * ORACLE_RSQRT128_F32;
+    }
+    return 0;
+}
+
+/*
+ * oracle_quantize_rows for fp32 inputs (the rotated rows): the same OCP MX
+ * rule, group amax, shared exponent and nearest-even encode, in fp64 on the
+ * exact fp32 values.
+ */
+int oracle_quantize_rows_f32(const float *x, int64_t n_rows, int64_t n_cols, const int32_t *valid,
+                             int fmt, uint8_t *codes, uint8_t *scales) {
+    if (!x || !codes || !scales || n_cols <= 0 || n_rows < 0) return -1;
+    const int64_t ng = (n_cols + 31) / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const float *xr = x + r * n_cols;
+        uint8_t *cr = codes + r * n_cols;
+        uint8_t *sr = scales + r * ng;
+        int64_t nv = valid ? (int64_t)valid[r] : n_cols;
+        if (nv > n_cols) nv = n_cols;
+        if (nv < 0) nv = 0;
+        for (int64_t g = 0; g < ng; ++g) {
+            int64_t c0 = g * 32, c1 = c0 + 32 < n_cols ? c0 + 32 : n_cols;
+            int64_t cv = c1 < nv ? c1 : nv;
+            if (cv <= c0) {
+                sr[g] = 0;
+                for (int64_t c = c0; c < c1; ++c) cr[c] = 0;
+                continue;
+            }
+            double amax = 0.0;
+            for (int64_t c = c0; c < cv; ++c) {
+                double a = fabs((double)xr[c]);
+                if (a > amax) amax = a;
+            }
+            int X = oracle_shared_exponent(fmt, amax);
+            sr[g] = (uint8_t)(X + 127);
+            for (int64_t c = c0; c < cv; ++c) cr[c] = (uint8_t)oracle_encode(fmt, ldexp((double)xr[c], -X));
+            for (int64_t c = cv; c < c1; ++c) cr[c] = 0;
+        }
+    }
+    return 0;
+}
+
+/*
+ * Softmax attention over unquantized inputs, in fp64: the reference the
+ * quantized method is compared against (the error against it is context, not
+ * a pass/fail bar). Also the visible-key rule with a window, shared with
+ * oracle_attention_window.
+ *
+ * q [B][Sq][Hq][d], k and v [B][Lk][Hkv][d], fp32 values (bf16 inputs are
+ * exact in fp32). For sequence b of length L (seqlens, NULL: Lk) query row i
+ * attends keys j with lo <= j < hi, where
+ *   hi = L, or with causal = 1, min(L, i + (L - Sq) + 1) (bottom-right);
+ *   lo = 0, or with window > 0, max(0, L - Sq - window): the last `window`
+ *        keys before the query block, and every key of the block.
+ * sel, out, lse as for oracle_attention.
+ */
+int oracle_attention_ref(const float *q, const float *k, const float *v, const int32_t *seqlens,
+                         int B, int Hq, int Hkv, int Sq, int Lk, int d, int causal, int window, double scale,
+                         const int32_t *sel, int64_t n_sel, double *out, double *lse) {
+    if (Hkv <= 0 || Hq % Hkv || d <= 0) return -1;
+    const int G = Hq / Hkv;
+    if (!sel) n_sel = (int64_t)B * Sq * Hq;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t r = 0; r < n_sel; ++r) {
+        int b, h, i;
+        if (sel) { b = sel[3 * r]; h = sel[3 * r + 1]; i = sel[3 * r + 2]; }
+        else { b = (int)(r / ((int64_t)Sq * Hq)); i = (int)((r / Hq) % Sq); h = (int)(r % Hq); }
+        int L = seqlens ? seqlens[b] : Lk;
+        if (L > Lk) L = Lk;
+        if (L < 0) L = 0;
+        int lo, hi;
+        visible_keys(L, Sq, i, causal, window, &lo, &hi);
+        double *o = out + r * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        if (hi <= lo) {
+            if (lse) lse[r] = -INFINITY;
+            continue;
+        }
+        double *p = (double *)malloc((size_t)(hi - lo) * sizeof(double));
+        if (!p) {
+#pragma omp atomic write
+            err = -2;
+            continue;
+        }
+        const int hk = h / G;
+        const float *qr = q + (((int64_t)b * Sq + i) * Hq + h) * d;
+        double m = -INFINITY;
+        for (int j = lo; j < hi; ++j) {
+            const float *kr = k + (((int64_t)b * Lk + j) * Hkv + hk) * d;
+            double s = 0.0;
+            for (int c = 0; c < d; ++c) s += (double)qr[c] * (double)kr[c];
+            s *= scale;
+            p[j - lo] = s;
+            if (s > m) m = s;
+        }
+        double l = 0.0;
+        for (int j = lo; j < hi; ++j) { p[j - lo] = exp(p[j - lo] - m); l += p[j - lo]; }
+        for (int j = lo; j < hi; ++j) {
+            const double w = p[j - lo] / l;
+            const float *vr = v + (((int64_t)b * Lk + j) * Hkv + hk) * d;
+            for (int c = 0; c < d; ++c) o[c] += w * (double)vr[c];
+        }
+        if (lse) lse[r] = m + log(l);
+        free(p);
+    }
     return err;
 }
 

@@ -339,3 +339,221 @@ def test_sampled_rows_match_full():
     for r, (b, h, i) in enumerate(sel):
         assert np.array_equal(o2[r], out[b, i, h])
         assert l2[r] == lse[b, i, h]
+
+
+# ------------------------------------------------- unquantized reference attention
+
+def naive_attention_window(q, k, v, seqlens, causal, scale, window):
+    """Softmax attention from the definition with the draft-block window:
+    row i of the Sq-row block sees the last `window` keys before the block and
+    every key of the block (causal: only keys up to its own position)."""
+    B, Sq, Hq, d = q.shape
+    Hkv = k.shape[2]
+    out = np.zeros((B, Sq, Hq, d))
+    lse = np.full((B, Sq, Hq), -np.inf)
+    for b in range(B):
+        L = int(seqlens[b])
+        for h in range(Hq):
+            hk = h // (Hq // Hkv)
+            for i in range(Sq):
+                keys = [j for j in range(L)
+                        if (not causal or j <= i + L - Sq) and (window <= 0 or j >= L - Sq - window)]
+                if not keys:
+                    continue
+                s = scale * (k[b, keys, hk, :] @ q[b, i, h, :])
+                m = s.max()
+                p = np.exp(s - m)
+                out[b, i, h] = (p @ v[b, keys, hk, :]) / p.sum()
+                lse[b, i, h] = m + np.log(p.sum())
+    return out, lse
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Lk,causal,lens,window", [
+    (1, 1, 1, 5, 5, True, None, 0),
+    (2, 4, 2, 3, 7, True, [7, 4], 0),
+    (2, 6, 2, 8, 8, False, [8, 3], 0),
+    (3, 4, 4, 2, 70, True, [70, 1, 35], 0),
+    (2, 4, 1, 8, 60, False, [60, 20], 16),
+    (2, 4, 2, 8, 90, True, [90, 9], 5),
+    (1, 2, 1, 1, 40, False, [40], 1),
+])
+def test_reference_attention_matches_naive(B, Hq, Hkv, Sq, Lk, causal, lens, window):
+    rng = np.random.default_rng(B * 1000 + Hq * 10 + Lk + window)
+    q = f32_to_bf16_bits(rng.standard_normal((B, Sq, Hq, 128)).astype(np.float32) * 2)
+    k = f32_to_bf16_bits(rng.standard_normal((B, Lk, Hkv, 128)).astype(np.float32) * 2)
+    v = f32_to_bf16_bits(rng.standard_normal((B, Lk, Hkv, 128)).astype(np.float32))
+    sl = np.array(lens if lens else [Lk] * B, dtype=np.int32)
+    out, lse = oracle.attention_ref(q, k, v, sl, causal=causal, window=window)
+    ref, rlse = naive_attention_window(bf16_bits_to_f64(q), bf16_bits_to_f64(k), bf16_bits_to_f64(v), sl, causal,
+                                       1 / math.sqrt(128), window)
+    assert np.allclose(out, ref, rtol=0, atol=1e-12)
+    assert np.array_equal(np.isinf(lse), np.isinf(rlse))
+    fin = np.isfinite(rlse)
+    assert np.allclose(lse[fin], rlse[fin], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,window", [(True, 0), (False, 12), (True, 3)])
+def test_windowed_oracle_matches_naive_on_dequantized(causal, window):
+    rng = np.random.default_rng(77 + window)
+    B, Sq, Hq, Hkv, Lk = 2, 8, 4, 2, 100
+    gen = dict(q=f32_to_bf16_bits(rng.standard_normal((B, Sq, Hq, 128)).astype(np.float32) * 2),
+               k=f32_to_bf16_bits(rng.standard_normal((B, Lk, Hkv, 128)).astype(np.float32) * 2),
+               v=f32_to_bf16_bits(rng.standard_normal((B, Lk, Hkv, 128)).astype(np.float32)),
+               seqlens=np.array([100, 37], dtype=np.int32))
+    qz = oracle.quantize_workload(gen)
+    out, lse = oracle.attention(qz["qc"], qz["qs"], qz["kc"], qz["ks"], qz["vc"], qz["vs"], gen["seqlens"],
+                                causal=causal, window=window)
+    qd, kd, vd = dequantized_inputs(qz)
+    ref, rlse = naive_attention_window(qd, kd, vd, gen["seqlens"], causal, 1 / math.sqrt(128), window)
+    assert np.allclose(out, ref, rtol=0, atol=1e-12)
+    assert np.allclose(lse, rlse, rtol=0, atol=1e-12)
+
+
+def test_window_closed_forms():
+    """A window of W keys before a one-row block sees exactly W + 1 keys; a window
+    at least the sequence length changes nothing."""
+    rng = np.random.default_rng(4)
+    L = 50
+    q = np.zeros((1, 1, 1, 128), np.uint16)  # Q = 0: uniform weights over the visible keys
+    k = f32_to_bf16_bits(rng.standard_normal((1, L, 1, 128)).astype(np.float32))
+    v = f32_to_bf16_bits(rng.standard_normal((1, L, 1, 128)).astype(np.float32))
+    sl = np.array([L], np.int32)
+    vv = bf16_bits_to_f64(v)
+    for W in (1, 7, 49):
+        out, lse = oracle.attention_ref(q, k, v, sl, causal=True, window=W)
+        assert np.allclose(out[0, 0, 0], vv[0, L - 1 - W:, 0].mean(axis=0), atol=1e-14)
+        assert abs(lse[0, 0, 0] - math.log(W + 1)) < 1e-13
+    o1, l1 = oracle.attention_ref(q, k, v, sl, causal=True, window=L)
+    o0, l0 = oracle.attention_ref(q, k, v, sl, causal=True, window=0)
+    assert np.array_equal(o1, o0) and np.array_equal(l1, l0)
+
+
+def test_grid_inputs_quantized_oracle_equals_reference():
+    """On MX-grid inputs quantization is the identity, so the quantized oracle and
+    the unquantized reference must agree (pins one against the other)."""
+    rng = np.random.default_rng(6)
+    B, Sq, Hq, Hkv, Lk = 2, 4, 4, 2, 96
+    q = _grid_tensor(rng, (B, Sq, Hq, 128), oracle.E2M1)
+    k = _grid_tensor(rng, (B, Lk, Hkv, 128), oracle.E2M1)
+    v = np.transpose(_grid_tensor(rng, (B, Hkv, 128, Lk), oracle.E4M3), (0, 3, 1, 2))
+    gen = dict(q=f32_to_bf16_bits(q.astype(np.float32)), k=f32_to_bf16_bits(k.astype(np.float32)),
+               v=f32_to_bf16_bits(v.astype(np.float32)), seqlens=np.array([96, 70], np.int32))
+    out, lse, _ = run_oracle(gen, True, 1 / 64.0)
+    ref, rlse = oracle.attention_ref(gen["q"], gen["k"], gen["v"], gen["seqlens"], causal=True, scale=1 / 64.0)
+    assert np.allclose(out, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+    assert np.allclose(lse, rlse, rtol=0, atol=1e-12 * np.abs(rlse).max())
+
+
+# ------------------------------------------------------------ Hadamard rotation
+
+def hadamard_matrix(n=128):
+    """Sylvester Hadamard matrix from its closed form H[i][j] = (-1)^popcount(i & j)."""
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    pc = np.vectorize(lambda x: bin(int(x)).count("1"))(i & j)
+    return np.where(pc % 2 == 0, 1.0, -1.0)
+
+
+RSQRT128_F32 = np.float32(2.0 ** -3.5)  # fp32 nearest to 1/sqrt(128)
+
+
+def test_hadamard_matrix_is_orthogonal():
+    H = hadamard_matrix()
+    assert np.array_equal(H @ H.T, 128 * np.eye(128))
+
+
+def test_hadamard_one_hot_rows():
+    """x = e_j gives c * (row j of H): every entry +-c with the popcount sign."""
+    H = hadamard_matrix()
+    for j in (0, 1, 5, 64, 127):
+        x = np.zeros((1, 128), np.uint16)
+        x[0, j] = f32_to_bf16_bits(np.float32(1.0))
+        y = oracle.hadamard_rows(x)[0]
+        assert np.array_equal(y, (H[j] * RSQRT128_F32).astype(np.float32)), j
+
+
+def test_hadamard_integer_inputs_exact():
+    """Small integers sum exactly in fp32, so the transform equals the integer
+    matrix product, rounded once by the final fp32 multiply."""
+    rng = np.random.default_rng(12)
+    H = hadamard_matrix()
+    xi = rng.integers(-100, 101, size=(64, 128))
+    y = oracle.hadamard_rows(f32_to_bf16_bits(xi.astype(np.float32)))
+    expect = (xi @ H.T).astype(np.float32) * RSQRT128_F32
+    assert np.array_equal(y, expect)
+
+
+def test_hadamard_random_inputs_within_fp32_bound():
+    rng = np.random.default_rng(13)
+    H = hadamard_matrix()
+    x = rng.standard_normal((256, 128)) * np.exp2(rng.integers(-8, 8, size=(256, 128)))
+    bits = f32_to_bf16_bits(x.astype(np.float32))
+    xb = bf16_bits_to_f64(bits)
+    y = oracle.hadamard_rows(bits).astype(np.float64)
+    exact = xb @ H.T / math.sqrt(128)
+    # seven butterfly stages and one multiply, each within 2^-24 relative of a partial sum <= sum|x|
+    bound = 9 * 2.0 ** -24 * np.abs(xb).sum(axis=1, keepdims=True)
+    assert np.all(np.abs(y - exact) <= bound)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(xb, axis=1), rtol=1e-6)
+
+
+def test_quantize_rows_f32_brute_force():
+    """The fp32-input quantizer against the numpy nearest-grid search, on values
+    that are not bf16 (rotated rows are general fp32)."""
+    rng = np.random.default_rng(14)
+    for fmt in (oracle.E2M1, oracle.E4M3):
+        x = (rng.standard_normal((2048, 32)) * np.exp2(rng.integers(-30, 30, size=(2048, 1)))).astype(np.float32)
+        x[::7, 3] = 0.0
+        x[::11] = 0.0
+        codes, scales = oracle.quantize_rows_f32(x, fmt)
+        emax = 2 if fmt == oracle.E2M1 else 8
+        amax = np.abs(x.astype(np.float64)).max(axis=1)
+        _, e = np.frexp(amax)
+        X = np.where(amax > 0, np.clip(e - 1 - emax, -127, 127), -127)
+        assert np.array_equal(scales[:, 0].astype(np.int64), X + 127)
+        y = x.astype(np.float64) * np.exp2(-X)[:, None]
+        expect = _brute_force_codes(y.ravel(), fmt).reshape(y.shape)
+        assert np.array_equal(codes, expect)
+
+
+def test_quantize_rows_f32_equals_bf16_path_on_bf16_values():
+    rng = np.random.default_rng(15)
+    bits = f32_to_bf16_bits((rng.standard_normal((512, 128)) * 3).astype(np.float32))
+    for fmt in (oracle.E2M1, oracle.E4M3):
+        c1, s1 = oracle.quantize_rows(bits, fmt)
+        c2, s2 = oracle.quantize_rows_f32(bf16_bits_to_f64(bits).astype(np.float32), fmt)
+        assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+
+
+def test_rotation_leaves_unquantized_attention_unchanged():
+    """(qR).(kR) = q.k: unquantized attention over rotated Q and K equals the
+    unrotated one up to the fp32 rounding of the rotation."""
+    rng = np.random.default_rng(16)
+    B, Sq, Hq, Hkv, Lk = 2, 6, 4, 2, 80
+    q = f32_to_bf16_bits(rng.standard_normal((B, Sq, Hq, 128)).astype(np.float32))
+    k = f32_to_bf16_bits(rng.standard_normal((B, Lk, Hkv, 128)).astype(np.float32))
+    v = f32_to_bf16_bits(rng.standard_normal((B, Lk, Hkv, 128)).astype(np.float32))
+    sl = np.array([80, 33], np.int32)
+    base, blse = oracle.attention_ref(q, k, v, sl, causal=True)
+    rot, rlse = oracle.attention_ref(oracle.hadamard_rows(q), oracle.hadamard_rows(k), v, sl, causal=True)
+    assert np.abs(rot - base).max() < 1e-5
+    assert np.abs(rlse - blse).max() < 1e-5
+
+
+def test_rotation_spreads_an_outlier_channel():
+    """A channel 16x larger than the rest dominates its MX group; after the
+    rotation it is spread over every group, so the rotated row's quantization
+    error of the non-outlier content is smaller (the article's reason for it)."""
+    rng = np.random.default_rng(17)
+    x = rng.standard_normal((512, 128)).astype(np.float32)
+    x[:, 5] *= 16.0
+    bits = f32_to_bf16_bits(x)
+    xb = bf16_bits_to_f64(bits)
+    c, s = oracle.quantize_rows(bits, oracle.E2M1)
+    err_plain = np.abs(oracle.dequantize_rows(c, s, oracle.E2M1) - xb)
+    y = oracle.hadamard_rows(bits)
+    cr, sr = oracle.quantize_rows_f32(y, oracle.E2M1)
+    H = hadamard_matrix()
+    back = oracle.dequantize_rows(cr, sr, oracle.E2M1) @ H / math.sqrt(128)  # rotate back
+    err_rot = np.abs(back - xb)
+    assert err_rot[:, 0:32].mean() < 0.7 * err_plain[:, 0:32].mean()
