@@ -82,8 +82,12 @@ def _seqlens(seqlens, B, device):
     return seqlens
 
 
-def quantize_qk(x: torch.Tensor, cap: Optional[int] = None, seqlens=None, out: Optional[MXFP4] = None) -> MXFP4:
-    """MXFP4-quantize Q or K ([B, T, H, 128] bf16) into the packed layout."""
+def quantize_qk(x: torch.Tensor, cap: Optional[int] = None, seqlens=None, out: Optional[MXFP4] = None,
+                hadamard: bool = False) -> MXFP4:
+    """MXFP4-quantize Q or K ([B, T, H, 128] bf16) into the packed layout.
+
+    hadamard=True rotates each row by H/sqrt(128) first (qk4v8_quantize_qk_hadamard);
+    rotate both Q and K, or neither."""
     _check_bf16(x, "x")
     B, T, H, _ = x.shape
     cap = round_cap(T) if cap is None else int(cap)
@@ -91,8 +95,10 @@ def quantize_qk(x: torch.Tensor, cap: Optional[int] = None, seqlens=None, out: O
     if out is None:
         out = MXFP4(torch.empty((B, H, cap, 64), dtype=torch.uint8, device=x.device),
                     torch.empty((B, H, cap // 128, 512), dtype=torch.uint8, device=x.device), B, H, cap, T)
-    check(lib().qk4v8_quantize_qk(x.data_ptr(), B, T, H, D, x.stride(0), x.stride(1), x.stride(2), _ptr(sl), cap,
-                                  out.codes.data_ptr(), out.scales.data_ptr(), _stream(x.device)), "qk4v8_quantize_qk")
+    fn, name = ((lib().qk4v8_quantize_qk_hadamard, "qk4v8_quantize_qk_hadamard") if hadamard
+                else (lib().qk4v8_quantize_qk, "qk4v8_quantize_qk"))
+    check(fn(x.data_ptr(), B, T, H, D, x.stride(0), x.stride(1), x.stride(2), _ptr(sl), cap,
+             out.codes.data_ptr(), out.scales.data_ptr(), _stream(x.device)), name)
     out.length = T
     return out
 
@@ -112,8 +118,12 @@ def quantize_v(v: torch.Tensor, cap: Optional[int] = None, seqlens=None, out: Op
     return out
 
 
-def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seqlens_k=None, q_cap=None, kv_cap=None):
-    """Quantize contiguous Q [B,Sq,Hq,128], K and V [B,Sk,Hkv,128] in one library call."""
+def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seqlens_k=None, q_cap=None, kv_cap=None,
+             hadamard: bool = False):
+    """Quantize contiguous Q [B,Sq,Hq,128], K and V [B,Sk,Hkv,128] in one library call.
+
+    hadamard=True quantizes Q and K after their Hadamard rotation (three launches:
+    qk4v8_quantize_qk_hadamard for Q and K, qk4v8_quantize_v for V)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check_bf16(t, n)
         if not t.is_contiguous():
@@ -124,6 +134,11 @@ def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seqlens_k=None, 
     kv_cap = round_cap(Sk) if kv_cap is None else int(kv_cap)
     dev = q.device
     sl = _seqlens(seqlens_k, B, dev)
+    if hadamard:
+        qp = quantize_qk(q, cap=q_cap, hadamard=True)
+        kp = quantize_qk(k, cap=kv_cap, seqlens=sl, hadamard=True)
+        vp = quantize_v(v, cap=kv_cap, seqlens=sl)
+        return qp, kp, vp
     qp = MXFP4(torch.empty((B, Hq, q_cap, 64), dtype=torch.uint8, device=dev),
                torch.empty((B, Hq, q_cap // 128, 512), dtype=torch.uint8, device=dev), B, Hq, q_cap, Sq)
     kp = MXFP4(torch.empty((B, Hkv, kv_cap, 64), dtype=torch.uint8, device=dev),

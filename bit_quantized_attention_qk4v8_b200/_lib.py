@@ -23,6 +23,7 @@ SIGNATURES = {
     "qk4v8_mxfp8_codes_bytes": ([_i32, _i32, _i32], _sz),
     "qk4v8_scales_bytes": ([_i32, _i32, _i32], _sz),
     "qk4v8_quantize_qk": ([_vp, _i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp], _i32),
+    "qk4v8_quantize_qk_hadamard": ([_vp, _i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp], _i32),
     "qk4v8_quantize_v": ([_vp, _i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp], _i32),
     "qk4v8_quantize": ([_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _i32,
                         _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i32),

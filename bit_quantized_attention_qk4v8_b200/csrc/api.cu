@@ -165,6 +165,18 @@ int qk4v8_quantize_qk(const void *x, int B, int S, int H, int d, int64_t stride_
     return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "quantize_qk launch");
 }
 
+int qk4v8_quantize_qk_hadamard(const void *x, int B, int S, int H, int d, int64_t stride_b, int64_t stride_s,
+                               int64_t stride_h, const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
+                               void *stream) {
+    int st = validate_quant_args(x, B, S, H, d, stride_b, stride_s, stride_h, cap, codes, scales);
+    if (st) return st;
+    if ((st = check_device())) return st;
+    cudaError_t e = qk4v8::launch_quantize_qk(x, B, S, H, stride_b, stride_s, stride_h, seqlens, cap, codes, scales,
+                                              static_cast<cudaStream_t>(stream), /*pad_to_cap=*/true,
+                                              /*rotate=*/true);
+    return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "quantize_qk_hadamard launch");
+}
+
 int qk4v8_quantize_v(const void *v, int B, int S, int H, int d, int64_t stride_b, int64_t stride_s,
                      int64_t stride_h, const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
                      void *stream) {
@@ -619,21 +631,53 @@ namespace {
 std::mutex g_noalloc_mu;
 constexpr int kNoAllocMaxDevices = 64;
 void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kNoAllocMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique id of the current CUDA context (0 when it cannot be had). A context
+// destroyed by cudaDeviceReset and created again gets a new id, even if its
+// handle value is reused, so a cached device address is looked up again.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
 
 // Device address of the scratch array on the current device. In host code the
 // array's name only stands in for the symbol and is not a device address, so
-// the address is looked up once per device, with that device current.
+// the address is looked up with the device current, once per device and
+// context (again after a cudaDeviceReset, which reloads the module).
 int noalloc_scratch_address(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
     if (dev < 0 || dev >= kNoAllocMaxDevices) return set_error(QK4V8_ERR_UNSUPPORTED, "device index %d too large", dev);
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
         void *ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, qk4v8_noalloc_scratch);
         if (e != cudaSuccess) return cuda_error(e, "cudaGetSymbolAddress(decode scratch)");
         g_noalloc_ptr[dev] = ptr;
+        // The id is read again: the symbol lookup may have created the context.
+        g_noalloc_ctx[dev] = current_context_id();
     }
     *out = g_noalloc_ptr[dev];
     return QK4V8_OK;
@@ -650,9 +694,14 @@ int qk4v8_attention_decode_noalloc(const uint8_t *q_codes, const uint8_t *q_scal
                                    float softmax_scale, int num_splits, void *out, float *lse, int32_t *dev_status,
                                    void *stream) {
     if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq < 1 || nq > 8 || (Hq / Hkv) * nq > 128)
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad sizes B=%d Hq=%d Hkv=%d nq=%d", B, Hq, Hkv, nq);
     const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen);
-    const size_t need = qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
-    if (need == 0 || need > QK4V8_NOALLOC_SCRATCH_BYTES)
+    // One split with up to 64 query rows per KV head: the split kernel writes
+    // the output itself and needs no scratch (qk4v8_attention_decode's rule).
+    const bool direct = splits == 1 && (Hq / Hkv) * nq <= qk4v8::kDecodeMaxRows;
+    const size_t need = direct ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
+    if (need > QK4V8_NOALLOC_SCRATCH_BYTES)
         return set_error(QK4V8_ERR_INVALID_ARG,
                          "decode scratch of %zu bytes (B=%d Hq=%d nq=%d splits=%d) exceeds the fixed %zu-byte "
                          "array of qk4v8_attention_decode_noalloc; use qk4v8_attention_decode with a workspace",
@@ -662,7 +711,7 @@ int qk4v8_attention_decode_noalloc(const uint8_t *q_codes, const uint8_t *q_scal
     if (st) return st;
     return qk4v8_attention_decode(q_codes, q_scales, B, Hq, nq, q_cap, k_codes, k_scales, v_codes, v_scales, Hkv,
                                   kv_cap, seqlens_k, max_seqlen, causal_in_block, softmax_scale, splits, scratch,
-                                  need, out, lse, dev_status, stream);
+                                  QK4V8_NOALLOC_SCRATCH_BYTES, out, lse, dev_status, stream);
 }
 
 }  // extern "C"

@@ -57,4 +57,59 @@ __device__ __forceinline__ uint32_t mxfp4_encode8(uint4 raw, bool valid, int &X)
     return valid ? (cvt_e2m1x8(v) | sign) : 0u;
 }
 
+// MXFP4 encode of eight fp32 values (the rotated rows), same lane layout and
+// contract as mxfp4_encode8; the sign of each code is the sign bit of the
+// float.
+__device__ __forceinline__ uint32_t mxfp4_encode8_f32(const float (&x)[8], bool valid, int &X) {
+    float v[8];
+    float amax = 0.f;
+    uint32_t sign = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        sign |= (__float_as_uint(x[i]) >> 31) << (4 * i + 3);
+        amax = fmaxf(amax, fabsf(x[i]));
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    X = shared_exponent(amax, 2);
+    const float f = pow2_neg(X);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = fabsf(x[i]) * f;  // exact: power-of-two scaling
+    return valid ? (cvt_e2m1x8(v) | sign) : 0u;
+}
+
+// Rotation of a 128-channel row by H / sqrt(128), H the Sylvester Hadamard
+// matrix (MpFA article, sections 2.1 and 3.1: a light rotation before the
+// 4-bit quantization spreads outlier channels over the row). The row is held
+// by 16 lanes, 8 consecutive channels each (lane sub = lane & 15 holds
+// channels 8 sub .. 8 sub + 7). Fast Walsh-Hadamard transform in fp32:
+// butterfly stages of stride 1, 2 and 4 inside the lane, then 8, 16, 32 and 64
+// across lanes (lane xor 1, 2, 4, 8); each stage maps the pair (a, b) at
+// channels (i, i + stride) to (a + b, a - b). Then one multiply by the fp32
+// value nearest 2^-3.5. All 32 lanes of the warp must call it together.
+__device__ __forceinline__ void hadamard128_rows(float (&v)[8], int sub) {
+#pragma unroll
+    for (int s = 1; s < 8; s *= 2) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (i & s) continue;
+            const float a = v[i], b = v[i + s];
+            v[i] = a + b;
+            v[i + s] = a - b;
+        }
+    }
+#pragma unroll
+    for (int m = 1; m < 16; m *= 2) {
+        const bool upper = (sub & m) != 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float other = __shfl_xor_sync(0xffffffffu, v[i], m);
+            v[i] = upper ? other - v[i] : v[i] + other;
+        }
+    }
+    constexpr float kRsqrt128 = 0x1.6a09e6p-4f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = v[i] * kRsqrt128;
+}
+
 }  // namespace qk4v8

@@ -46,9 +46,10 @@ struct AttnParams {
 
 // pad_to_cap: write all `cap` token rows of each sequence (rows past the valid
 // length get zero codes and scales); otherwise only the S input rows.
+// rotate: quantize each row after its rotation by H / sqrt(128).
 cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                                const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
-                               cudaStream_t stream, bool pad_to_cap = true);
+                               cudaStream_t stream, bool pad_to_cap = true, bool rotate = false);
 cudaError_t launch_quantize_v(const void *v, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                               const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
                               cudaStream_t stream);

@@ -39,6 +39,22 @@ __device__ __forceinline__ void qk_store_row(uint8_t *__restrict__ codes, uint8_
     }
 }
 
+// With kRotate, each row is first rotated by H / sqrt(128) (hadamard128_rows)
+// and the rotated fp32 values are quantized.
+__device__ __forceinline__ uint32_t qk_encode_row(uint4 raw, bool valid, int sub, bool rotate, int &X) {
+    if (!rotate) return mxfp4_encode8(raw, valid, X);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+    hadamard128_rows(v, sub);
+    return mxfp4_encode8_f32(v, valid, X);
+}
+
+template <bool kRotate>
 __global__ void __launch_bounds__(256) quantize_qk_kernel(const __nv_bfloat16 *__restrict__ x, int B, int S, int H,
                                                           int64_t sb, int64_t ss, int64_t sh,
                                                           const int32_t *__restrict__ seqlens, int cap,
@@ -79,12 +95,12 @@ __global__ void __launch_bounds__(256) quantize_qk_kernel(const __nv_bfloat16 *_
         if (v0) raw0 = *reinterpret_cast<const uint4 *>(xb + t * ss + h * sh + sub * 8);
         if (v1) raw1 = *reinterpret_cast<const uint4 *>(xb + t1 * ss + h1 * sh + sub * 8);
         int X0, X1;
-        const uint32_t p0 = mxfp4_encode8(raw0, v0, X0);
+        const uint32_t p0 = qk_encode_row(raw0, v0, sub, kRotate, X0);
         if (in0) qk_store_row(codes, scales, head_b + h, cap, t, sub, p0, X0, v0);
         // The second pair of rows is encoded by the whole warp too (shuffles),
         // when the warp's first row of it exists.
         if (base + step < rows) {
-            const uint32_t p1 = mxfp4_encode8(raw1, v1, X1);
+            const uint32_t p1 = qk_encode_row(raw1, v1, sub, kRotate, X1);
             if (in1) qk_store_row(codes, scales, head_b + h1, cap, t1, sub, p1, X1, v1);
         }
         t = t1;
@@ -183,7 +199,7 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__
 
 cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                                const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
-                               cudaStream_t stream, bool pad_to_cap) {
+                               cudaStream_t stream, bool pad_to_cap, bool rotate) {
     const int row_len = pad_to_cap ? cap : S;
     const int64_t rows = static_cast<int64_t>(row_len) * H;  // per batch entry
     if (rows >= (int64_t{1} << 30)) return cudaErrorInvalidValue;
@@ -199,9 +215,15 @@ cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, i
     const int64_t scales_per_b = static_cast<int64_t>(H) * (cap / 128) * 512;
     for (int b0 = 0; b0 < B; b0 += 65535) {
         const int nb = B - b0 < 65535 ? B - b0 : 65535;
-        quantize_qk_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(nb)), 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16 *>(x) + b0 * sb, nb, S, H, sb, ss, sh, seqlens ? seqlens + b0 : nullptr,
-            cap, row_len, codes + b0 * codes_per_b, scales + b0 * scales_per_b);
+        const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(nb));
+        const __nv_bfloat16 *xs = static_cast<const __nv_bfloat16 *>(x) + b0 * sb;
+        const int32_t *ls = seqlens ? seqlens + b0 : nullptr;
+        if (rotate)
+            quantize_qk_kernel<true><<<grid, 256, 0, stream>>>(xs, nb, S, H, sb, ss, sh, ls, cap, row_len,
+                                                               codes + b0 * codes_per_b, scales + b0 * scales_per_b);
+        else
+            quantize_qk_kernel<false><<<grid, 256, 0, stream>>>(xs, nb, S, H, sb, ss, sh, ls, cap, row_len,
+                                                                codes + b0 * codes_per_b, scales + b0 * scales_per_b);
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

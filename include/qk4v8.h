@@ -104,6 +104,25 @@ QK4V8_API int qk4v8_quantize_qk(const void *x, int B, int S, int H, int d,
                       uint8_t *codes, uint8_t *scales, void *stream);
 
 /*
+ * MXFP4 quantization of Q or K after a Hadamard rotation of each row (MpFA
+ * article, section 3.1, and the outlier discussion of section 2.1: a light
+ * rotation ahead of the per-group 4-bit quantization spreads outlier channels
+ * over the whole row). Each (token, head) row x of 128 channels becomes
+ * y = x H / sqrt(128), H the Sylvester Hadamard matrix
+ * (H[i][j] = (-1)^popcount(i & j)), computed in fp32 as the fast
+ * Walsh-Hadamard transform (butterfly strides 1, 2, ..., 64) followed by one
+ * multiply by the fp32 value nearest 2^-3.5; y is then quantized exactly as by
+ * qk4v8_quantize_qk. The rotation is orthonormal, so quantizing both Q and K
+ * this way leaves Q K^T, and the attention calls, unchanged: pass the rotated
+ * packed Q and K to them as they are (V is not rotated). Arguments, layout and
+ * errors as for qk4v8_quantize_qk.
+ */
+QK4V8_API int qk4v8_quantize_qk_hadamard(const void *x, int B, int S, int H, int d,
+                               int64_t stride_b, int64_t stride_s, int64_t stride_h,
+                               const int32_t *seqlens, int cap,
+                               uint8_t *codes, uint8_t *scales, void *stream);
+
+/*
  * MXFP8-E4M3 quantization of V, groups of 32 along the token axis (article
  * section 2.2: V stays at 8 bits).
  *   v        bf16 [B][S][H][128] (device), strides in elements
@@ -166,7 +185,10 @@ QK4V8_API size_t qk4v8_decode_workspace_bytes(int B, int Hq, int nq, int num_spl
 QK4V8_API int qk4v8_decode_default_splits(int B, int Hq, int Hkv, int nq, int max_seqlen);
 
 /*
- * The two stages of qk4v8_attention_decode, as separate launches.
+ * The two stages of qk4v8_attention_decode, as separate launches (MpFA
+ * article, sections 1.3 and 3.3: the memory-bound decode attention with its
+ * FP32 online softmax, here split over the KV length; the splits' partial
+ * (max, sum, O) are combined afterwards).
  *
  * qk4v8_attention_decode_splitkv: for every (sequence, KV head, split) the
  * split kernel runs the tiled QK4V8 attention over the split's contiguous
@@ -194,6 +216,11 @@ QK4V8_API int qk4v8_decode_merge(const void *workspace, size_t workspace_bytes, 
 
 /*
  * Split-KV decode and speculative block verify over a packed KV cache.
+ * MpFA article, section 1.3: in decode, attention is memory bound, so the
+ * packed cache (4-bit K, 8-bit V) is streamed once, split across CTAs, at HBM
+ * rate. MiMo DFlash article, section on block-diffusion speculative decoding
+ * (block_size 8): the backbone verifies a whole draft block in one forward,
+ * hence up to nq = 8 query tokens per sequence, causal within the block.
  *   q_*      packed MXFP4 Q, [B][Hq][q_cap] with nq (1..8) query tokens
  *   k_*, v_* packed cache, [B][Hkv][kv_cap]
  *   seqlens_k int32 [B] (device, required), each <= kv_cap
@@ -270,6 +297,10 @@ QK4V8_API int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, 
  *     the size.
  *   - The first call on each device looks up the array's device address, with
  *     that device current. Make that first call before any stream capture.
+ *     The address is cached per device and CUDA context; after a
+ *     cudaDeviceReset the next call looks it up again.
+ *   - One split with up to 64 query rows per KV head needs no scratch, so such
+ *     calls are never refused for size.
  *   - Every call shares the one array, and the array keeps the last call's
  *     contents. Nothing in it has to start at zero: the split kernels write
  *     every partial slot before a merge reads it. Calls that overlap on the GPU

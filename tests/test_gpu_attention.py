@@ -208,6 +208,67 @@ def test_decode_poisoned_padding_does_not_leak():
     assert torch.equal(clean, dirty)
 
 
+def _poison_padding(kp, vp, lens):
+    """Overwrite every cache byte past each sequence's length with NaN patterns:
+    codes, whole scale atoms past the last block, and the scale entries of the
+    padding rows and groups inside the last block."""
+    for b, L in enumerate(lens):
+        vp.codes[b, :, :, L:] = 0xFF          # E4M3 NaN
+        kp.codes[b, :, L:] = 0xFF
+        blk0 = L // 128
+        vp.scales[b, :, blk0 + 1:] = 0xFF
+        kp.scales[b, :, blk0 + 1:] = 0xFF
+        jv = L - blk0 * 128
+        if blk0 >= vp.scales.shape[2]:
+            continue
+        if jv == 0:   # block blk0 starts at L: all of it is padding
+            vp.scales[b, :, blk0] = 0xFF
+            kp.scales[b, :, blk0] = 0xFF
+            continue
+        idx = torch.tensor([(c % 32) * 16 + (c // 32) * 4 + g for c in range(128) for g in range((jv + 31) // 32, 4)],
+                           dtype=torch.long, device="cuda")
+        if idx.numel():
+            vp.scales[b, :, blk0, idx] = 0xFF
+        tidx = torch.tensor([(t % 32) * 16 + (t // 32) * 4 + g for t in range(jv, 128) for g in range(4)],
+                            dtype=torch.long, device="cuda")
+        kp.scales[b, :, blk0, tidx] = 0xFF
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_prefill_poisoned_padding_does_not_leak(causal):
+    """Prefill over a cache whose bytes past each length are NaN patterns: the
+    output must equal the one over clean (zero) padding, bit for bit."""
+    lens = [300, 45, 256]
+    gen = make_gen(3, 64, 512, 8, 2, seed=14, lens=lens, k_out=2)
+    qp, kp, vp, sl = quantize_on_gpu(gen)
+    clean = qk.attention_prefill(qp, kp, vp, seqlens_k=sl, causal=causal)
+    torch.cuda.synchronize()
+    clean = clean.clone()
+    _poison_padding(kp, vp, lens)
+    dirty = qk.attention_prefill(qp, kp, vp, seqlens_k=sl, causal=causal)
+    torch.cuda.synchronize()
+    assert torch.isfinite(dirty.float()).all()
+    assert torch.equal(clean, dirty)
+    (ref, _), _ = oracle_attention_from(gen, causal)
+    assert_close(dirty, ref, f"poisoned prefill causal={causal}")
+
+
+@pytest.mark.parametrize("Hq,Hkv,nq,splits", [(64, 8, 8, 3), (16, 1, 8, 2)])
+def test_decode_poisoned_padding_larger_groups(Hq, Hkv, nq, splits):
+    """The GQA decode kernel (64 rows) and the 128-row kernel over NaN padding."""
+    lens = [300, 45, 129]
+    gen = make_gen(3, nq, 512, Hq, Hkv, seed=15, lens=lens, k_out=4)
+    qp, kp, vp, sl = quantize_on_gpu(gen)
+    clean = qk.attention_decode(qp, kp, vp, sl, max_seqlen=300, num_splits=splits)
+    torch.cuda.synchronize()
+    clean = clean.clone()
+    _poison_padding(kp, vp, lens)
+    dirty = qk.attention_decode(qp, kp, vp, sl, max_seqlen=300, num_splits=splits)
+    torch.cuda.synchronize()
+    assert torch.isfinite(dirty.float()).all()
+    assert torch.equal(clean, dirty)
+
+
 def test_deterministic():
     gen = make_gen(2, 8, 1500, 16, 2, seed=9, k_out=4)
     qp, kp, vp, sl = quantize_on_gpu(gen)

@@ -153,3 +153,26 @@ def test_workload_quantize_bit_exact(name):
         vc, vs = oracle.quantize_v(gen["v"][b:b + 1], lens[b:b + 1])
         assert np.array_equal(vp.codes[b:b + 1].cpu().numpy()[..., :wl.Lk], vc)
         assert np.array_equal(v_scales_logical(vp.scales[b:b + 1].cpu().numpy(), wl.Lk), vs)
+
+
+@pytest.mark.timeout(300)
+def test_qk_batch_beyond_grid_y_limit():
+    """B = 65537 sequences: the launcher runs the batch in chunks of 65535 grid
+    rows, offsetting inputs, lengths, codes and scales per chunk. Entries on both
+    sides of the chunk boundary and the last one must match the oracle."""
+    B = 65537
+    rng = np.random.default_rng(21)
+    bits = f32_to_bf16_bits(rng.standard_normal((B, 1, 1, 128)).astype(np.float32) * 4)
+    lens = np.ones((B,), np.int32)
+    lens[65535] = 0   # first entry of the second chunk is empty
+    xp = qk.quantize_qk(to_dev(bits), cap=128, seqlens=torch.from_numpy(lens).cuda())
+    torch.cuda.synchronize()
+    oc, os_ = oracle.quantize_qk(bits)
+    oc[lens == 0] = 0
+    os_[lens == 0] = 0
+    for b in (0, 1, 65534, 65535, 65536):
+        codes = xp.codes[b].cpu().numpy()
+        scales = xp.scales[b].cpu().numpy()
+        assert np.array_equal(unpack_e2m1(codes[None, :, :1])[0], oc[b]), b
+        assert np.array_equal(qk_scales_logical(scales[None], 1)[0], os_[b]), b
+        assert not codes[:, 1:].any()

@@ -79,3 +79,33 @@ def test_noalloc_rejects_oversized_scratch():
         sl.data_ptr(), max_len, 1, ctypes.c_float(0.0), 100, out.data_ptr(), None, None, stream)
     assert rc == 1
     assert b"exceeds the fixed" in _lib.lib().qk4v8_last_error()
+
+
+def test_noalloc_gqa_kernel_after_other_contents():
+    """33..64 query rows per KV head run on the GQA decode kernel, which keeps
+    per-sequence piece counts in the scratch. A different call first leaves
+    its own partials in the shared array; then two GQA problems in a row (splits
+    >= 2, and the library's default) must still match qk4v8_attention_decode."""
+    qp, kp, vp, sl, max_len = _problem(3, 16, 4, 2, 1500, 41)
+    _noalloc(qp, kp, vp, sl, max_len, 4)          # fills the array with swap-AB partials
+    torch.cuda.synchronize()
+    for B, Hq, Hkv, nq, L, seed, splits in [(2, 64, 8, 8, 1200, 42, 3), (3, 48, 8, 8, 2000, 43, 0),
+                                            (2, 64, 8, 8, 900, 44, 2)]:
+        qp, kp, vp, sl, max_len = _problem(B, Hq, Hkv, nq, L, seed)
+        ref = qk.attention_decode(qp, kp, vp, sl, max_seqlen=max_len, num_splits=splits)
+        out, status = _noalloc(qp, kp, vp, sl, max_len, splits)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        d = (out.float() - ref.float()).abs()
+        assert torch.isfinite(out.float()).all()
+        assert d.max().item() <= MAX_ABS_TOL and d.mean().item() <= MEAN_ABS_TOL, (d.max().item(), d.mean().item())
+
+
+def test_noalloc_single_split_needs_no_scratch():
+    """One split with up to 64 rows writes the output directly: no size limit applies."""
+    qp, kp, vp, sl, max_len = _problem(2, 32, 8, 1, 800, 45)
+    ref = qk.attention_decode(qp, kp, vp, sl, max_seqlen=max_len, num_splits=1)
+    out, status = _noalloc(qp, kp, vp, sl, max_len, 1)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(out, ref)
