@@ -7,22 +7,33 @@ outlier channels x16 in Q and K. The step is one library call,
 qk4v8_attention_decode_bf16: the split-KV block-scaled tcgen05 attention over
 the pre-quantized MXFP4-K / MXFP8-V cache, which MXFP4-quantizes the step's
 bf16 query rows itself. With one KV split (the library's choice for this
-workload) that is a single launch that also writes the bf16 output; with
-more splits a merge launch follows.
+workload) that is a single launch that also writes the bf16 output.
 `value` is the packed KV bytes streamed per second, summed over all ranks
 (weak scaling: every rank runs its own copy of the workload, with no
 collective on the data path).
 
-The JSON line also carries these sub-objects:
-  - roofline: the attention kernel's achieved GB/s against the measured HBM
-    copy bandwidth;
-  - e2e: the same step through the public API with pinned host buffers, the
-    query copied in and the output copied back every step;
+The JSON line also carries one flat object per other workload or measurement:
+  - roofline: the headline decode kernel's achieved GB/s against the measured
+    HBM copy bandwidth (and the 8 TB/s specification);
+  - e2e: the headline step through the public API with pinned host buffers,
+    the query copied in and the output copied back every step;
+  - decode_long, verify: the long-context decode (B=8, Hq=64, L in
+    [65536, 131072]) and 8-token speculative verify (B=64, Hq=64, L=16384)
+    workloads, each one library call per step;
   - prefill: the causal GQA prefill workload B=4, Hq=32, Hkv=8, S=8192,
-    quantization of Q, K and V included, in TFLOPS;
-  - cpu_baseline: the CPU oracle on a bounded sample of the same decode
-    workload.
-`--impl reference` times the CPU oracle alone on the decode workload.
+    quantization of Q, K and V included, in TFLOPS, with its QK^T-stage build
+    against the measured block-scaled FP4 peak of the best MMA shape;
+  - prefill_small: the causal prefill B=1, Hq=Hkv=2, S=256;
+  - quantize: the MXFP4 (plain and Hadamard-rotated) and MXFP8 quantize
+    kernels in HBM GB/s;
+  - mma_peaks: the measured tensor-pipe peaks of the block-scaled MMA shapes;
+  - cpu_baseline (and cpu_* keys in each workload object): the CPU fp64
+    oracle on the machine's host cores, on the whole workload (configs 1, 2, 4, 5)
+    or a stated subset (the S=8192 prefill), extrapolated linearly;
+  - error keys (err_*): the GPU output against the oracle, and, as context,
+    against fp64 attention over the unquantized bf16 inputs; hadamard_* keys
+    give the same for Q and K quantized after their Hadamard rotation.
+`--impl reference` times the CPU oracle alone on the headline decode workload.
 """
 from __future__ import annotations
 
@@ -43,10 +54,23 @@ if ROOT not in sys.path:
 
 METRIC = "QK4V8 attn: prefill TFLOPS & decode KV GB/s, % of B200 roofline"
 DECODE_WORKLOAD = "decode_gqa_b32_hq32_hkv8_l8192"
+LONG_WORKLOAD = "decode_long_b8_hq64_hkv8_l64k_128k"
+VERIFY_WORKLOAD = "verify_b64_nq8_hq64_hkv8_l16384"
 PREFILL_WORKLOAD = "prefill_gqa_b4_hq32_hkv8_s8192"
+SMALL_PREFILL_WORKLOAD = "prefill_b1_h2_s256"
 KV_BYTES_PER_TOKEN_HEAD = 64 + 128 + 4 + 4   # E2M1 K codes, E4M3 V codes, K and V E8M0 scales
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+SPEC_HBM_GBS = 8000.0      # B200 HBM3e, DGX figure
+SPEC_FP4_TFLOPS = 9000.0   # dense block-scaled FP4
+L2_BYTES = 126 * 2 ** 20
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
+# kernel, from its committed ncu capture; None until a capture of the kernel as
+# it stands exists.
+NCU_TRAFFIC = {
+    DECODE_WORKLOAD: None,
+}
 
 
 def parse_args():
@@ -65,8 +89,11 @@ def parse_args():
                     help="decode workload of the main measurement (a profiling aid; the headline is the default)")
     ap.add_argument("--no-decode", action="store_true",
                     help="prefill only (a profiling aid): prints the prefill object alone")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the CPU oracle leg (baselines and error reports)")
+    ap.add_argument("--no-hadamard", action="store_true", help="skip the Hadamard-rotated runs")
+    ap.add_argument("--quantize-only", action="store_true",
+                    help="quantize kernels only (a profiling aid): prints the quantize object alone")
     return ap.parse_args()
 
 
@@ -75,9 +102,9 @@ def load_peaks():
     try:
         with open(path) as f:
             pk = json.load(f)
-        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), "measured"
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
 class ClockSampler:
@@ -102,16 +129,19 @@ class ClockSampler:
         except Exception:
             self.nv = None
 
-    def _run(self):
+    def _sample(self):
         nv = self.nv
         get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
             getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+            self.reasons |= int(get_reasons(self.h))
+        except Exception:
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                self.reasons |= int(get_reasons(self.h))
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def __enter__(self):
@@ -124,6 +154,8 @@ class ClockSampler:
         if self._thread is not None:
             self._stop.set()
             self._thread.join()
+            if not self.samples:
+                self._sample()
 
     def summary(self):
         if not self.samples:
@@ -172,9 +204,42 @@ def aggregate_gbs(bytes_per_rank_step: int, steps: int, world: int, elapsed_ms: 
     return bytes_per_rank_step * steps * world / (elapsed_ms * 1e-3) / 1e9
 
 
+def headline_config(world: int) -> dict:
+    """The `config` object of the headline line; both arms print the same one."""
+    import synth
+    wl = synth.WORKLOADS[DECODE_WORKLOAD]
+    kv = wl.B * wl.Hkv * wl.Lk * KV_BYTES_PER_TOKEN_HEAD
+    return {"workload": DECODE_WORKLOAD, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "nq": wl.Sq, "L": wl.Lk, "d": 128,
+            "parallelism": f"dp{world}: independent replicas, no collective on the data path",
+            "l2": f"no flush: the packed KV cache ({kv / 1e6:.0f} MB) is larger than L2 (126 MB)"}
+
+
 def to_dev(bits):
     import torch
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def graph_time_ms(step, steps, warmup, stream):
+    """Runs `step` warmup times, captures `steps` calls in one CUDA graph, replays
+    it once untimed, then times one replay with events. Returns (ms per step, clocks)."""
+    import torch
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(steps):
+            step()
+    graph.replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    del graph
+    return t0.elapsed_time(t1) / steps, clk.summary()
 
 
 # ----------------------------------------------------------------------------- decode
@@ -203,6 +268,26 @@ def decode_launches(rows: int, splits: int) -> int:
     return 3                                         # query quantize, 128-row split kernel, merge
 
 
+def rotated_decode(k_dev, q_dev, vp, sl, cap, max_len, splits, steps, warmup):
+    """Q and K quantized after their Hadamard rotation, then the packed decode.
+    Returns (host output [B, nq, Hq, 128], ms per step of quantize(Q) + decode)."""
+    import torch
+    import bit_quantized_attention_qk4v8_b200 as qk
+    kp_r = qk.quantize_qk(k_dev, cap=cap, seqlens=sl, hadamard=True)
+    qp_r = qk.quantize_qk(q_dev, hadamard=True)
+    B, nq, Hq, _ = q_dev.shape
+    ws = torch.empty((max(16, qk.decode_workspace_bytes(B, Hq, nq, splits)),), dtype=torch.uint8, device="cuda")
+    out = torch.empty((B, nq, Hq, 128), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        qk.quantize_qk(q_dev, hadamard=True, out=qp_r)
+        qk.attention_decode(qp_r, kp_r, vp, sl, max_seqlen=max_len, num_splits=splits, workspace=ws, out=out)
+
+    ms, _ = graph_time_ms(step, steps, warmup, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), ms
+
+
 def run_decode(args, world, rank):
     import torch
     import bit_quantized_attention_qk4v8_b200 as qk
@@ -212,8 +297,10 @@ def run_decode(args, world, rank):
     q_host = torch.from_numpy(gen["q"].view(np.int16)).view(torch.bfloat16).pin_memory()
     q = q_host.cuda()
     sl = torch.from_numpy(gen["seqlens"]).cuda()
-    kp = qk.quantize_qk(to_dev(gen["k"]), seqlens=sl)      # the cache: quantized once, outside the timing
-    vp = qk.quantize_v(to_dev(gen["v"]), seqlens=sl)
+    cap = qk.round_cap(wl.Lk)
+    k = to_dev(gen["k"])
+    kp = qk.quantize_qk(k, cap=cap, seqlens=sl)      # the cache: quantized once, outside the timing
+    vp = qk.quantize_v(to_dev(gen["v"]), cap=cap, seqlens=sl)
     max_len = int(gen["seqlens"].max())
     splits = args.splits if args.splits > 0 else qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, max_len)
     ws_bytes = qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)
@@ -256,16 +343,16 @@ def run_decode(args, world, rank):
         attn_timing = "timed region / steps (one launch per step)"
     else:
         # Several launches per step: a second replay with an event pair (graph
-        # event-record nodes) around each attention call times the kernel alone.
+        # event-record nodes) around each attention call times the call alone.
         ev = [(torch.cuda.Event(enable_timing=True, external=True),
                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
         g2 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g2):
-            cap = torch.cuda.current_stream()
+            cap_s = torch.cuda.current_stream()
             for i in range(args.steps):
-                ev[i][0].record(cap)
+                ev[i][0].record(cap_s)
                 step()
-                ev[i][1].record(cap)
+                ev[i][1].record(cap_s)
         g2.replay()
         torch.cuda.synchronize()
         attn_avg_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
@@ -294,14 +381,19 @@ def run_decode(args, world, rank):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    out_np = out.float().cpu().numpy()
 
+    rot = None
+    if world == 1 and not args.no_hadamard:
+        rot = rotated_decode(k, q, vp, sl, cap, max_len, splits, 50, 3)
+    del k
     return dict(wl=wl, gen=gen, kv_bytes=kv_bytes, splits=splits, elapsed_ms=elapsed_ms, attn_avg_ms=attn_avg_ms,
                 launches_per_step=launches, attn_timing=attn_timing,
                 clocks=clk.summary(), e2e_ms=e2e_ms, e2e_steps=e2e_steps,
-                h2d=q_host.numel() * 2, d2h=out_host.numel() * 2)
+                h2d=q_host.numel() * 2, d2h=out_host.numel() * 2, out=out_np, rot=rot)
 
 
-def run_decode_workload(name, steps, warmup, hbm_gbs):
+def run_decode_workload(name, steps, warmup, hbm_gbs, hadamard):
     """One of the other decode workloads (long context, speculative verify): one
     qk4v8_attention_decode_bf16 call per step over its pre-quantized cache."""
     import torch
@@ -315,10 +407,11 @@ def run_decode_workload(name, steps, warmup, hbm_gbs):
     cap = qk.round_cap(wl.Lk)
     k = to_dev(gen["k"])
     kp = qk.quantize_qk(k, cap=cap, seqlens=sl)
-    del k
+    if not hadamard:
+        del k
     v = to_dev(gen["v"])
     vp = qk.quantize_v(v, cap=cap, seqlens=sl)
-    del v, gen
+    del v
     max_len = int(lens.max())
     splits = qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, max_len)
     ws_bytes = qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)
@@ -328,49 +421,44 @@ def run_decode_workload(name, steps, warmup, hbm_gbs):
     def step():
         qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=max_len, num_splits=splits, workspace=ws, out=out)
 
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for _ in range(steps):
-            step()
-    graph.replay()
-    torch.cuda.synchronize()
-    stream = torch.cuda.current_stream()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        t0.record(stream)
-        graph.replay()
-        t1.record(stream)
-        torch.cuda.synchronize()
-    del graph
-    ms = t0.elapsed_time(t1) / steps
+    ms, clocks = graph_time_ms(step, steps, warmup, torch.cuda.current_stream())
+    out_np = out.float().cpu().numpy()
+    rot = None
+    if hadamard:
+        del kp
+        rot = rotated_decode(k, q, vp, sl, cap, max_len, splits, steps, 3)
+        del k
     kv_bytes = int(lens.sum()) * wl.Hkv * KV_BYTES_PER_TOKEN_HEAD   # the packed cache each step streams
     gbs = kv_bytes / (ms * 1e-3) / 1e9
     rows = wl.G * wl.Sq
-    return {
+    res = {
         "workload": name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "nq": wl.Sq, "kv_len_mean": float(lens.mean()),
-        "kv_len_max": max_len, "kv_splits": splits, "ms_per_step": ms, "value": gbs, "unit": "GB/s",
-        "tokens_per_s": wl.B * wl.Sq / (ms * 1e-3),
-        "launches_per_step": decode_launches(rows, splits),
-        "roofline": {"bound": "hbm", "kernel": decode_kernel_name(rows), "achieved": gbs, "peak": hbm_gbs,
-                     "unit": "GB/s", "frac": gbs / hbm_gbs, "algorithmic_bytes_per_step": kv_bytes,
-                     "note": "step time (all launches of the call); the split kernel dominates it"},
-        "clocks": clk.summary(),
+        "kv_len_max": max_len, "kv_splits": splits, "ms_per_step": ms, "steps": steps, "value": gbs,
+        "unit": "GB/s", "tokens_per_s": wl.B * wl.Sq / (ms * 1e-3),
+        "launches_per_step": decode_launches(rows, splits), "kernel": decode_kernel_name(rows),
+        "roofline_bound": "hbm", "algorithmic_bytes_per_step": kv_bytes, "roofline_peak_gbs": hbm_gbs,
+        "roofline_frac": gbs / hbm_gbs, "roofline_frac_of_spec_8tbs": gbs / SPEC_HBM_GBS,
+        "roofline_timing": "step time (all launches of the call); the split kernel dominates it",
+        "clocks_sm_mhz": clocks["sm_mhz"], "clocks_reasons": ",".join(clocks["reasons"]) or "none",
     }
+    if rot is not None:
+        res["hadamard_ms_per_step"] = rot[1]
+        res["hadamard_step"] = "quantize_qk_hadamard(Q) + qk4v8_attention_decode over the rotated K cache"
+    return dict(res=res, gen=gen, out=out_np, rot=None if rot is None else rot[0], wl=wl)
 
 
 # ---------------------------------------------------------------------------- prefill
 
-def run_prefill(args):
+PREFILL_SUBSET_HEADS = list(range(0, 32, 4))   # (b = 0, one query head per KV head): the CPU subset
+
+
+def run_prefill(args, hadamard):
     import torch
     import bit_quantized_attention_qk4v8_b200 as qk
     import synth
     wl = synth.WORKLOADS[PREFILL_WORKLOAD]
     gen = wl.generate()
     q, k, v = to_dev(gen["q"]), to_dev(gen["k"]), to_dev(gen["v"])
-    del gen
     stream = torch.cuda.current_stream()
     qp, kp, vp = qk.quantize(q, k, v)
     out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
@@ -399,6 +487,7 @@ def run_prefill(args):
         torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / n
     attn_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    out_sub = out[0][:, PREFILL_SUBSET_HEADS].float().cpu().numpy()      # [S, 8, 128]
 
     # The QK^T stage alone: the same kernel built without exp, P and P.V, same tile schedule.
     for _ in range(3):
@@ -412,19 +501,114 @@ def run_prefill(args):
     torch.cuda.synchronize()
     stage_ms = s0.elapsed_time(s1) / n
 
+    rot_sub, rot_ms = None, None
+    if hadamard:
+        def rstep():
+            qr, kr, vr = qk.quantize(q, k, v, hadamard=True)
+            qk.attention_prefill(qr, kr, vr, causal=True, out=out)
+
+        for _ in range(2):
+            rstep()
+        torch.cuda.synchronize()
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        for _ in range(n):
+            rstep()
+        r1.record(stream)
+        torch.cuda.synchronize()
+        rot_ms = r0.elapsed_time(r1) / n
+        rot_sub = out[0][:, PREFILL_SUBSET_HEADS].float().cpu().numpy()
+
     # FlashAttention-style FLOP count of causal attention: 4 * B * Hq * d * (S(S+1)/2)
     pairs = wl.Sq * (wl.Sq + 1) / 2
     flops = 4.0 * wl.B * wl.Hq * 128 * pairs
-    qk_flops = flops / 2
     # Executed work: every 128 x 128 tile on or below the causal diagonal is computed in full.
     nt = (wl.Sq + 127) // 128
     tiles = wl.B * wl.Hq * nt * (nt + 1) // 2
-    return dict(wl=wl, ms=ms, attn_ms=attn_ms, stage_ms=stage_ms, flops=flops, qk_flops=qk_flops, tiles=tiles,
-                clocks=clk.summary())
+    return dict(wl=wl, gen=gen, ms=ms, attn_ms=attn_ms, stage_ms=stage_ms, flops=flops, qk_flops=flops / 2,
+                tiles=tiles, clocks=clk.summary(), out_sub=out_sub, rot_sub=rot_sub, rot_ms=rot_ms)
 
 
-def run_mma_peaks(kinds=(0, 1), iters=200000):
-    """Tensor-pipe peak (TFLOP/s) of the attention's own MMA shapes, one CTA per SM, CUDA-event timed."""
+def run_prefill_small(steps=200):
+    """The causal prefill B=1, Hq=Hkv=2, S=256: quantize Q, K, V + attention per step."""
+    import torch
+    import bit_quantized_attention_qk4v8_b200 as qk
+    import synth
+    wl = synth.WORKLOADS[SMALL_PREFILL_WORKLOAD]
+    gen = wl.generate()
+    q, k, v = to_dev(gen["q"]), to_dev(gen["k"]), to_dev(gen["v"])
+    out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
+    qp, kp, vp = qk.quantize(q, k, v)
+
+    # One graph of library calls on fixed output buffers: quantize Q, K, V, attention.
+    def step_fixed():
+        qk.quantize_qk(q, out=qp)
+        qk.quantize_qk(k, out=kp)
+        qk.quantize_v(v, out=vp)
+        qk.attention_prefill(qp, kp, vp, causal=True, out=out)
+
+    ms, clocks = graph_time_ms(step_fixed, steps, 5, torch.cuda.current_stream())
+    pairs = wl.Sq * (wl.Sq + 1) / 2
+    flops = 4.0 * wl.B * wl.Hq * 128 * pairs
+    res = {"workload": SMALL_PREFILL_WORKLOAD, "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOPS",
+           "ms_per_step": ms, "steps": steps, "launches_per_step": 4,
+           "step": "quantize Q, K, V + causal prefill attention (latency-bound; no roofline fraction)",
+           "clocks_sm_mhz": clocks["sm_mhz"]}
+    return dict(res=res, gen=gen, out=out.float().cpu().numpy(), wl=wl, flops=flops)
+
+
+def run_quantize_kernels(hbm_gbs, gen, reps=10):
+    """HBM throughput of the quantize kernels on the S=8192 prefill workload's
+    tensors (`gen`); L2 is flushed (a 256 MB write) before every timed launch."""
+    import torch
+    import bit_quantized_attention_qk4v8_b200 as qk
+    import synth
+    wl = synth.WORKLOADS[PREFILL_WORKLOAD]
+    q, k, v = to_dev(gen["q"]), to_dev(gen["k"]), to_dev(gen["v"])
+    flush = torch.empty((256 * 2 ** 20,), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    qp = qk.quantize_qk(q)
+    kp = qk.quantize_qk(k)
+    vp = qk.quantize_v(v)
+    cases = [
+        ("quantize_qk_q", "quantize_qk_kernel<false> (Q)", lambda: qk.quantize_qk(q, out=qp),
+         wl.B * wl.Sq * wl.Hq * (256 + 68)),
+        ("quantize_qk_hadamard_q", "quantize_qk_kernel<true> (Q, rotated)",
+         lambda: qk.quantize_qk(q, out=qp, hadamard=True), wl.B * wl.Sq * wl.Hq * (256 + 68)),
+        ("quantize_qk_k", "quantize_qk_kernel<false> (K)", lambda: qk.quantize_qk(k, out=kp),
+         wl.B * wl.Sq * wl.Hkv * (256 + 68)),
+        ("quantize_v", "quantize_v_kernel (V)", lambda: qk.quantize_v(v, out=vp),
+         wl.B * wl.Sq * wl.Hkv * (256 + 132)),
+    ]
+    res = {"workload": PREFILL_WORKLOAD, "unit": "GB/s", "peak_gbs": hbm_gbs,
+           "bytes": "algorithmic: 256 B bf16 read + 64 B codes + 4 B scales written per Q/K token-head row; "
+                    "256 B read + 128 B codes + 4 B scales per V token-head",
+           "l2": "flushed (256 MB write) before each timed launch"}
+    for key, kname, fn, nbytes in cases:
+        fn()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[f"{key}_us"] = ms * 1e3
+        res[f"{key}_gbs"] = gbs
+        res[f"{key}_frac"] = gbs / hbm_gbs
+        res[f"{key}_frac_of_spec_8tbs"] = gbs / SPEC_HBM_GBS
+        res[f"{key}_bytes"] = nbytes
+        res[f"{key}_kernel"] = kname
+    return res
+
+
+def run_mma_peaks(kinds=(0, 1, 2, 3), iters=200000):
+    """Tensor-pipe peak (TFLOP/s) of block-scaled MMA shapes, one CTA per SM, CUDA-event timed."""
     import torch
     import bit_quantized_attention_qk4v8_b200 as qk
     sms = torch.cuda.get_device_properties(0).multi_processor_count
@@ -446,127 +630,244 @@ def run_mma_peaks(kinds=(0, 1), iters=200000):
     return res
 
 
+def prefill_object(p, peaks):
+    """Flat summary of the S=8192 prefill run against the measured MMA peaks."""
+    import torch
+    fp4_own = peaks["mxf4_m128n128k64"]       # the QK^T instruction's own shape
+    fp8_own = peaks["mxf8f6f4_m128n144k32"]   # the P.V instruction's own shape
+    fp4_best = max(v for k, v in peaks.items() if k.startswith("mxf4"))
+    fp8_best = max(v for k, v in peaks.items() if k.startswith("mxf8"))
+    best_fp4_shape = max((v, k) for k, v in peaks.items() if k.startswith("mxf4"))[1]
+    # Roofline time of the executed MMAs: QK^T in FP4; P.V twice (P_hi and P_lo terms) in FP8 at
+    # N = 144 (128 channels, the ones row that sums P, padding to a multiple of 16).
+    t_own = p["qk_flops"] / (fp4_own * 1e12) + 2 * p["qk_flops"] * (144 / 128) / (fp8_own * 1e12)
+    t_best = p["qk_flops"] / (fp4_best * 1e12) + 2 * p["qk_flops"] / (fp8_best * 1e12)
+    attn_s = p["attn_ms"] * 1e-3
+    clocks = p["clocks"]
+    sm_hz = (clocks.get("sm_mhz") or 1965.0) * 1e6
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    mufu_s = p["tiles"] * 128 * 128 / (16.0 * sms * sm_hz)   # one ex2 per executed score, 16 per clock per SM
+    stage_tf = p["qk_flops"] / (p["stage_ms"] * 1e-3) / 1e12
+    res = {
+        "workload": PREFILL_WORKLOAD, "value": p["flops"] / (p["ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
+        "ms_per_step": p["ms"], "steps": p.get("steps"),
+        "step": "quantize Q,K,V + causal prefill attention (FlashAttention FLOP count 2.199e12)",
+        "launches_per_step": 4,
+        "attention_ms": p["attn_ms"], "attention_tflops": p["flops"] / attn_s / 1e12,
+        "kernel": "qk4v8_prefill_kernel<false>", "roofline_bound": "tensor",
+        "roofline_frac": t_best / attn_s,
+        "roofline_peak_tflops": p["flops"] / t_best / 1e12,
+        "roofline_peak_source": "measured tcgen05 peaks of the fastest mxf4 and mxf8f6f4 shapes (mma_peaks)",
+        "roofline_frac_own_shapes": t_own / attn_s,
+        "qk_stage_kernel": "qk4v8_prefill_kernel<true> (QK^T stage build)",
+        "qk_stage_ms": p["stage_ms"], "qk_stage_tflops": stage_tf,
+        "qk_stage_frac_of_best_fp4": stage_tf / fp4_best, "qk_stage_best_fp4_shape": best_fp4_shape,
+        "qk_stage_frac_of_n128_fp4": stage_tf / fp4_own,
+        "qk_stage_frac_of_spec_fp4_9pf": stage_tf / SPEC_FP4_TFLOPS,
+        "mufu_bound_ms": mufu_s * 1e3, "mufu_frac": mufu_s / attn_s,
+        "clocks_sm_mhz": clocks["sm_mhz"], "clocks_reasons": ",".join(clocks["reasons"]) or "none",
+    }
+    if p.get("rot_ms") is not None:
+        res["hadamard_ms_per_step"] = p["rot_ms"]
+        res["hadamard_step"] = "quantize (Q, K rotated) + causal prefill attention"
+    return res
+
+
 # ------------------------------------------------------------------------ CPU oracle
+# Everything below runs the CPU oracle: the baselines (timed on the host cores)
+# and the error reports. It is the benchmark's cpu_baseline leg.
 
-def oracle_decode_sample(gen, wl, target_s: float, max_units=None):
-    """Time the CPU oracle on whole (b, h_kv) units of the decode workload.
+def _errs(got, ref, prefix):
+    d = np.abs(np.asarray(got, np.float64) - np.asarray(ref, np.float64))
+    return {f"{prefix}_max_abs": float(d.max()), f"{prefix}_mean_abs": float(d.mean())}
 
-    Per unit: MXFP4 quantization of the unit's query rows and fp64 attention
-    over the unit's cache, the same work as one GPU step restricted to that
-    unit. The cache is quantized beforehand, as it is on the GPU path.
-    Returns (kv_bytes_processed, seconds, units, threads)."""
+
+def cpu_decode_leg(gen, wl, out_gpu, rot_gpu):
+    """Oracle on the whole decode workload (cache pre-quantized untimed, as on the
+    GPU; Q quantize + attention timed), the GPU output's error against it, and
+    the context errors against unquantized attention on three batch entries."""
     import oracle
-    B, Hkv, G, nq, L = wl.B, wl.Hkv, wl.G, wl.Sq, wl.Lk
-    done_bytes, done_s, units = 0, 0.0, 0
-    b = 0
-    while b < B and done_s < target_s and (max_units is None or units < max_units):
-        sub = dict(q=gen["q"][b:b + 1], k=gen["k"][b:b + 1], v=gen["v"][b:b + 1], seqlens=gen["seqlens"][b:b + 1])
-        kc, ks = oracle.quantize_qk(sub["k"])
-        vc, vs = oracle.quantize_v(sub["v"], sub["seqlens"])
+    kc, ks = oracle.quantize_qk(gen["k"])
+    vc, vs = oracle.quantize_v(gen["v"], gen["seqlens"])
+    t = time.perf_counter()
+    qc, qs = oracle.quantize_qk(gen["q"])
+    ref, _ = oracle.attention(qc, qs, kc, ks, vc, vs, gen["seqlens"], causal=True)
+    sec = time.perf_counter() - t
+    del kc, ks, vc, vs
+    kv_bytes = int(gen["seqlens"].astype(np.int64).sum()) * wl.Hkv * KV_BYTES_PER_TOKEN_HEAD
+    res = {"cpu_value": kv_bytes / sec / 1e9, "cpu_unit": "GB/s", "cpu_cores": oracle.num_threads(),
+           "cpu_kind": "oracle", "cpu_seconds": sec,
+           "cpu_sample": f"whole workload ({wl.B} sequences): Q quantize + fp64 attention; cache quantized untimed"}
+    res.update(_errs(out_gpu, ref, "err_vs_oracle"))
+    bs = sorted({0, wl.B // 2, wl.B - 1})
+    got, orc, bf, rot = [], [], [], []
+    for b in bs:
+        one = slice(b, b + 1)
+        r, _ = oracle.attention_ref(gen["q"][one], gen["k"][one], gen["v"][one], gen["seqlens"][one], causal=True)
+        bf.append(r[0])
+        got.append(out_gpu[b])
+        orc.append(ref[b])
+        if rot_gpu is not None:
+            rot.append(rot_gpu[b])
+    bf = np.stack(bf)
+    res.update(_errs(np.stack(got), bf, "err_vs_bf16"))
+    res.update(_errs(np.stack(orc), bf, "oracle_err_vs_bf16"))
+    res["err_bf16_rows"] = f"batch entries {bs}, every head and query token"
+    if rot_gpu is not None:
+        rorc = []
+        for b in bs:
+            one = slice(b, b + 1)
+            rqc, rqs = oracle.quantize_qk_hadamard(gen["q"][one])
+            rkc, rks = oracle.quantize_qk_hadamard(gen["k"][one], gen["seqlens"][one])
+            rvc, rvs = oracle.quantize_v(gen["v"][one], gen["seqlens"][one])
+            o, _ = oracle.attention(rqc, rqs, rkc, rks, rvc, rvs, gen["seqlens"][one], causal=True)
+            rorc.append(o[0])
+        res.update(_errs(np.stack(rot), np.stack(rorc), "hadamard_err_vs_oracle"))
+        res.update(_errs(np.stack(rot), bf, "hadamard_err_vs_bf16"))
+    return res
+
+
+def cpu_prefill_leg(p):
+    """Oracle on a subset of the S=8192 prefill (batch entry 0, one query head per
+    KV head: 8 of the 128 (b, h_q) pairs), extrapolated linearly: the quantize of
+    Q, K, V of entry 0 times B, the attention of the subset times 16."""
+    import oracle
+    wl, gen = p["wl"], p["gen"]
+    one = slice(0, 1)
+    t = time.perf_counter()
+    qc, qs = oracle.quantize_qk(gen["q"][one])
+    kc, ks = oracle.quantize_qk(gen["k"][one])
+    vc, vs = oracle.quantize_v(gen["v"][one], gen["seqlens"][one])
+    t_quant = time.perf_counter() - t
+    S = wl.Sq
+    sel = np.array([(0, h, i) for h in PREFILL_SUBSET_HEADS for i in range(S)], dtype=np.int32)
+    t = time.perf_counter()
+    ref, _ = oracle.attention(qc, qs, kc, ks, vc, vs, gen["seqlens"][one], causal=True, sel=sel)
+    t_attn = time.perf_counter() - t
+    frac = len(PREFILL_SUBSET_HEADS) / (wl.B * wl.Hq)
+    sec = t_quant * wl.B + t_attn / frac
+    res = {"cpu_value": p["flops"] / sec / 1e12, "cpu_unit": "TFLOPS", "cpu_cores": oracle.num_threads(),
+           "cpu_kind": "oracle", "cpu_seconds_measured": t_quant + t_attn, "cpu_seconds_extrapolated": sec,
+           "cpu_sample": f"batch entry 0, query heads {PREFILL_SUBSET_HEADS[0]}..{PREFILL_SUBSET_HEADS[-1]} step "
+                         f"4 (8 of 128 (b, h_q) pairs, all {S} rows): attention x16, quantize of entry 0 x{wl.B}; "
+                         "extrapolated linearly"}
+    got = np.transpose(p["out_sub"], (1, 0, 2)).reshape(-1, 128)     # [h, i] order like sel
+    res.update(_errs(got, ref, "err_vs_oracle"))
+    rng = np.random.default_rng(0)
+    pick = np.sort(rng.choice(sel.shape[0], size=256, replace=False))
+    psel = sel[pick]
+    bf, _ = oracle.attention_ref(gen["q"][one], gen["k"][one], gen["v"][one], gen["seqlens"][one], causal=True,
+                                 sel=psel)
+    res.update(_errs(got[pick], bf, "err_vs_bf16"))
+    res.update(_errs(ref[pick], bf, "oracle_err_vs_bf16"))
+    res["err_bf16_rows"] = "256 random rows of the subset"
+    if p.get("rot_sub") is not None:
+        rqc, rqs = oracle.quantize_qk_hadamard(gen["q"][one])
+        rkc, rks = oracle.quantize_qk_hadamard(gen["k"][one], gen["seqlens"][one])
+        ro, _ = oracle.attention(rqc, rqs, rkc, rks, vc, vs, gen["seqlens"][one], causal=True, sel=psel)
+        rgot = np.transpose(p["rot_sub"], (1, 0, 2)).reshape(-1, 128)[pick]
+        res.update(_errs(rgot, ro, "hadamard_err_vs_oracle"))
+        res.update(_errs(rgot, bf, "hadamard_err_vs_bf16"))
+    return res
+
+
+def cpu_small_prefill_leg(s):
+    import oracle
+    gen, wl = s["gen"], s["wl"]
+    n, sec = 0, 0.0
+    while sec < 1.0:
         t = time.perf_counter()
-        qc, qs = oracle.quantize_qk(sub["q"])
-        oracle.attention(qc, qs, kc, ks, vc, vs, sub["seqlens"], causal=True)
-        done_s += time.perf_counter() - t
-        done_bytes += Hkv * int(sub["seqlens"][0]) * KV_BYTES_PER_TOKEN_HEAD
-        units += Hkv
-        b += 1
-    return done_bytes, done_s, units, oracle.num_threads()
+        oz = oracle.quantize_workload(gen)
+        ref, _ = oracle.attention(oz["qc"], oz["qs"], oz["kc"], oz["ks"], oz["vc"], oz["vs"], gen["seqlens"],
+                                  causal=True)
+        sec += time.perf_counter() - t
+        n += 1
+    res = {"cpu_value": s["flops"] * n / sec / 1e12, "cpu_unit": "TFLOPS", "cpu_cores": oracle.num_threads(),
+           "cpu_kind": "oracle", "cpu_seconds": sec,
+           "cpu_sample": f"whole workload (quantize Q, K, V + attention), {n} repetitions"}
+    res.update(_errs(s["out"], ref, "err_vs_oracle"))
+    bf, _ = oracle.attention_ref(gen["q"], gen["k"], gen["v"], gen["seqlens"], causal=True)
+    res.update(_errs(s["out"], bf, "err_vs_bf16"))
+    res.update(_errs(ref, bf, "oracle_err_vs_bf16"))
+    return res
 
 
 def run_reference(args, world, rank):
-    """--impl reference: the CPU oracle, as it stands, on the decode workload."""
+    """--impl reference: the CPU oracle, as it stands, on the headline decode workload.
+
+    One step is a bounded sample of the workload: one batch entry (its 8 KV
+    heads, 8192 keys, 4 query rows each), MXFP4 query quantize + fp64 attention,
+    the entry's cache quantized outside the timing (as on the GPU); when K + W
+    such steps would take more than about three minutes, a step is one (b, h_kv)
+    unit instead."""
     if rank != 0:
         return 0
     import oracle
     import synth
     wl = synth.WORKLOADS[DECODE_WORKLOAD]
     gen = wl.generate()
-    # One reference step = one batch entry (8 KV heads x 8192 keys) of the workload.
-    b_cycle = list(range(wl.B))
     cache = {}
 
-    def unit(b):
+    def entry(b):
         if b not in cache:
             kc, ks = oracle.quantize_qk(gen["k"][b:b + 1])
             vc, vs = oracle.quantize_v(gen["v"][b:b + 1], gen["seqlens"][b:b + 1])
             cache[b] = (kc, ks, vc, vs)
         return cache[b]
 
+    def sub(arrs, h):
+        kc, ks, vc, vs = arrs
+        s = slice(h, h + 1)
+        return kc[:, s], ks[:, s], vc[:, s], vs[:, s]
+
+    G = wl.G
+    mode = {"unit": False}
+
     def step(i):
-        b = b_cycle[i % len(b_cycle)]
-        kc, ks, vc, vs = unit(b)
-        qc, qs = oracle.quantize_qk(gen["q"][b:b + 1])
+        b = i % wl.B
+        kc, ks, vc, vs = entry(b)
+        if mode["unit"]:
+            h = (i // wl.B) % wl.Hkv
+            kc, ks, vc, vs = sub((kc, ks, vc, vs), h)
+            qc, qs = oracle.quantize_qk(gen["q"][b:b + 1, :, h * G:(h + 1) * G])
+        else:
+            qc, qs = oracle.quantize_qk(gen["q"][b:b + 1])
         oracle.attention(qc, qs, kc, ks, vc, vs, gen["seqlens"][b:b + 1], causal=True)
 
-    steps = max(1, args.steps)
-    # Bound the whole run to a few minutes: time the first step, cap the count.
-    for i in range(min(args.warmup, 2)):
-        step(i)
+    steps, warmup = max(1, args.steps), max(0, args.warmup)
+    entry(0)
     t = time.perf_counter()
     step(0)
     one = time.perf_counter() - t
-    steps_run = max(1, min(steps, int(120.0 / max(one, 1e-3))))
-    for i in range(steps_run):
-        unit(b_cycle[i % len(b_cycle)])   # quantize the cache outside the timing
+    if (steps + warmup) * one > 180.0:
+        mode["unit"] = True
+    step_bytes = (wl.Lk if mode["unit"] else wl.Hkv * wl.Lk) * KV_BYTES_PER_TOKEN_HEAD
+    for i in range(warmup):
+        step(i)
+    for i in range(steps):
+        entry(i % wl.B)   # the cache is quantized outside the timing
     t = time.perf_counter()
-    for i in range(steps_run):
+    for i in range(steps):
         step(i)
     sec = time.perf_counter() - t
-    step_bytes = wl.Hkv * wl.Lk * KV_BYTES_PER_TOKEN_HEAD
-    value = step_bytes * steps_run / sec / 1e9
+    value = step_bytes * steps / sec / 1e9
+    sample = ("one (b, h_kv) unit per step: 8192 keys, 4 query rows" if mode["unit"]
+              else "one batch entry per step (of 32): 8 KV heads x 8192 keys, 4 query rows each")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1, "steps": steps_run,
-        "warmup": min(args.warmup, 2), "ms_per_step": sec / steps_run * 1e3, "higher_is_better": True,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": sec / steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": DECODE_WORKLOAD, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "nq": wl.Sq, "L": wl.Lk,
-                   "d": 128, "reference_step": "one batch entry: 8 KV heads x 8192 keys, 4 query rows each"},
+        "config": headline_config(world),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": f"{steps_run} steps of one batch entry each (of {wl.B})"},
+                         "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
-    if steps_run < steps:
-        line["steps_requested"] = steps
     print(json.dumps(line), flush=True)
     return 0
 
 
 # ------------------------------------------------------------------------------- main
-
-def prefill_object(args, peak_src, bf16_tf):
-    p = run_prefill(args)
-    peaks = run_mma_peaks()
-    fp4_peak = peaks["mxf4_m128n128k64"]      # the QK^T instruction's own measured peak
-    fp8_peak = peaks["mxf8f6f4_m128n144k32"]  # the P.V instruction's own measured peak
-    # Roofline time of the executed MMAs: QK^T in FP4; P.V twice (P_hi and P_lo terms) in FP8 at
-    # N = 144 (128 channels, the ones row that sums P, padding to a multiple of 16).
-    t_roof = p["qk_flops"] / (fp4_peak * 1e12) + 2 * p["qk_flops"] * (144 / 128) / (fp8_peak * 1e12)
-    attn_s = p["attn_ms"] * 1e-3
-    clocks = p["clocks"]
-    sm_hz = (clocks.get("sm_mhz") or 1965.0) * 1e6
-    # MUFU bound: one ex2 per executed score element, 16 per clock per SM.
-    import torch
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    mufu_s = p["tiles"] * 128 * 128 / (16.0 * sms * sm_hz)
-    return {
-        "workload": PREFILL_WORKLOAD, "value": p["flops"] / (p["ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
-        "ms_per_step": p["ms"], "steps": args.prefill_steps, "step": "quantize Q,K,V + causal prefill attention",
-        "attention_ms": p["attn_ms"], "attention_tflops": p["flops"] / attn_s / 1e12,
-        "roofline": {"bound": "tensor", "kernel": "qk4v8_prefill_kernel<false>",
-                     "achieved": p["flops"] / attn_s / 1e12,
-                     "peak": p["flops"] / t_roof / 1e12, "unit": "TFLOPS",
-                     "frac": t_roof / attn_s,
-                     "peak_source": "measured tcgen05 peaks of the kernel's own MMA shapes (mma_peaks)"},
-        "qk_stage": {"kernel": "qk4v8_prefill_kernel<true> (QK^T stage build)", "ms": p["stage_ms"],
-                     "tflops": p["qk_flops"] / (p["stage_ms"] * 1e-3) / 1e12,
-                     "frac_of_measured_fp4": p["qk_flops"] / (p["stage_ms"] * 1e-3) / 1e12 / fp4_peak,
-                     "frac_of_spec_fp4_9pf": p["qk_flops"] / (p["stage_ms"] * 1e-3) / 1e12 / 9000.0},
-        "mma_peaks_tflops": peaks,
-        "mufu_bound_ms": mufu_s * 1e3, "mufu_frac": mufu_s / attn_s,
-        "bf16_x4_fp4_nominal_tflops": bf16_tf * 4.0,
-        "clocks": clocks,
-    }
-
 
 def main():
     args = parse_args()
@@ -578,11 +879,20 @@ def main():
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (B200); the library has no CPU path")
     world, rank, local = dist_setup(args.gpus)
-    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = load_peaks()
+    hbm_gbs, bf16_tf, peak_src = load_peaks()
+    hadamard = not args.no_hadamard
 
+    if args.quantize_only:
+        if rank == 0:
+            import synth
+            gen = synth.WORKLOADS[PREFILL_WORKLOAD].generate()
+            print(json.dumps({"quantize": run_quantize_kernels(hbm_gbs, gen, reps=3)}), flush=True)
+        return 0
     if args.no_decode:
         if rank == 0:
-            print(json.dumps({"prefill": prefill_object(args, peak_src, bf16_tf)}), flush=True)
+            p = run_prefill(args, False)
+            p["steps"] = args.prefill_steps
+            print(json.dumps({"prefill": prefill_object(p, run_mma_peaks())}), flush=True)
         return 0
 
     d = run_decode(args, world, rank)
@@ -592,6 +902,7 @@ def main():
     ms_per_step = d["elapsed_ms"] / steps
     achieved = d["kv_bytes"] / (d["attn_avg_ms"] * 1e-3) / 1e9
     e2e_value = aggregate_gbs(d["kv_bytes"], d["e2e_steps"], world, d["e2e_ms"])
+    traffic = NCU_TRAFFIC.get(args.decode_workload)
 
     line = {
         "metric": METRIC,
@@ -606,16 +917,17 @@ def main():
         "vs_baseline": None,
         "dtype": "e2m1/e4m3 MMA, f32 softmax and accumulate",
         "data": "synthetic",
-        "config": {
-            "workload": args.decode_workload, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "nq": wl.Sq, "L": wl.Lk, "d": 128,
-            "kv_splits": d["splits"], "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": f"no flush: the packed KV cache ({d['kv_bytes'] / 1e6:.0f} MB) is larger than L2 (126 MB)",
-            "tokens_per_s": wl.B * wl.Sq * steps * world / (d["elapsed_ms"] * 1e-3),
-        },
+        "config": headline_config(world) if args.decode_workload == DECODE_WORKLOAD else
+        {"workload": args.decode_workload},
+        "kv_splits": d["splits"],
+        "tokens_per_s": wl.B * wl.Sq * steps * world / (d["elapsed_ms"] * 1e-3),
         "roofline": {
             "bound": "hbm", "kernel": decode_kernel_name(wl.G * wl.Sq),
             "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
-            "peak_source": f"{peak_src} hbm_gbs", "traffic": None,
+            "frac_of_spec_8tbs": achieved / SPEC_HBM_GBS,
+            "peak_source": f"{peak_src} hbm_gbs (burst copy)",
+            "traffic": None if traffic is None else traffic[0],
+            "traffic_source": None if traffic is None else traffic[1],
             "algorithmic_bytes_per_launch": d["kv_bytes"], "avg_launch_ms": d["attn_avg_ms"],
             "launch_timing": d["attn_timing"],
         },
@@ -625,21 +937,40 @@ def main():
         "clocks": d["clocks"],
     }
 
-    if not args.no_extra_decode and world == 1:
-        line["decode_workloads"] = {}
-        for name in ("decode_long_b8_hq64_hkv8_l64k_128k", "verify_b64_nq8_hq64_hkv8_l16384"):
-            w = run_decode_workload(name, args.extra_steps, min(args.warmup, 5), hbm_gbs)
-            line["decode_workloads"][name] = w
-            line["gpu_launches"] += w["launches_per_step"] * args.extra_steps
-    if not args.no_prefill:
-        line["prefill"] = prefill_object(args, peak_src, bf16_tf)
-        line["gpu_launches"] += 4 * args.prefill_steps
+    extra = {}
+    if world == 1 and not args.no_extra_decode:
+        for key, name in (("decode_long", LONG_WORKLOAD), ("verify", VERIFY_WORKLOAD)):
+            extra[key] = run_decode_workload(name, args.extra_steps, min(args.warmup, 5), hbm_gbs,
+                                             hadamard and key == "verify")
+            line[key] = extra[key]["res"]
+    pre = small = None
+    if world == 1 and not args.no_prefill:
+        peaks = run_mma_peaks()
+        line["mma_peaks"] = {**{k: v for k, v in peaks.items()}, "unit": "TFLOPS",
+                             "how": "one CTA per SM issuing one tcgen05.mma shape from shared memory, CUDA events"}
+        pre = run_prefill(args, hadamard)
+        pre["steps"] = args.prefill_steps
+        line["prefill"] = prefill_object(pre, peaks)
+        small = run_prefill_small()
+        line["prefill_small"] = small["res"]
+        line["quantize"] = run_quantize_kernels(hbm_gbs, pre["gen"])
 
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        nbytes, sec, units, threads = oracle_decode_sample(d["gen"], wl, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": nbytes / sec / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                                "sample": f"{units} of {wl.B * wl.Hkv} (b, h_kv) units, whole batch entries, "
-                                          f"{sec:.1f} s"}
+        head = cpu_decode_leg(d["gen"], wl, d["out"], None if d["rot"] is None else d["rot"][0])
+        line["cpu_baseline"] = {"value": head["cpu_value"], "unit": "GB/s", "cores": head["cpu_cores"],
+                                "kind": "oracle", "sample": head["cpu_sample"]}
+        line["context_error"] = {k: v for k, v in head.items() if "err" in k}
+        line["context_error"]["note"] = ("err_vs_oracle: GPU vs the fp64 QK4V8 oracle (bar: max 3e-2, mean 3e-3); "
+                                         "err_vs_bf16: GPU vs fp64 attention over the unquantized bf16 inputs "
+                                         "(context, no bar); hadamard_*: Q and K quantized after rotation")
+        if d["rot"] is not None:
+            line["context_error"]["hadamard_ms_per_step"] = d["rot"][1]
+        for key, x in extra.items():
+            x["res"].update(cpu_decode_leg(x["gen"], x["wl"], x["out"], x["rot"]))
+        if pre is not None:
+            line["prefill"].update(cpu_prefill_leg(pre))
+        if small is not None:
+            line["prefill_small"].update(cpu_small_prefill_leg(small))
 
     if rank == 0:
         print(json.dumps(line), flush=True)
