@@ -176,7 +176,9 @@ def decode_workspace_bytes(B: int, Hq: int, nq: int, num_splits: int) -> int:
     return int(lib().qk4v8_decode_workspace_bytes(B, Hq, nq, num_splits))
 
 
-def decode_default_splits(B: int, Hq: int, Hkv: int, nq: int, max_seqlen: int) -> int:
+def decode_default_splits(B: int, Hq: int, Hkv: int, nq: int, max_seqlen: int, window: int = 0) -> int:
+    if window:
+        return int(lib().qk4v8_decode_default_splits_window(B, Hq, Hkv, nq, max_seqlen, int(window)))
     return int(lib().qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen))
 
 
@@ -184,14 +186,17 @@ def attention_decode(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optio
                      causal_in_block: bool = True, softmax_scale: Optional[float] = None, num_splits: int = 0,
                      workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                      lse: Optional[torch.Tensor] = None, return_lse: bool = False,
-                     dev_status: Optional[torch.Tensor] = None):
-    """Split-KV decode / speculative verify over a packed cache. Returns out bf16 [B, nq, Hq, 128]."""
+                     dev_status: Optional[torch.Tensor] = None, window: int = 0):
+    """Split-KV decode / speculative verify over a packed cache. Returns out bf16 [B, nq, Hq, 128].
+
+    window > 0: draft-block attention, each query row sees only the last `window`
+    keys before the nq-token block and the block (qk4v8_attention_decode_window)."""
     dev = q.codes.device
     B, Hq, nq = q.B, q.H, q.length
     sl = _seqlens(seqlens_k, B, dev)
     if max_seqlen is None:
         max_seqlen = k.cap
-    splits = num_splits if num_splits > 0 else decode_default_splits(B, Hq, k.H, nq, max_seqlen)
+    splits = num_splits if num_splits > 0 else decode_default_splits(B, Hq, k.H, nq, max_seqlen, window)
     need = decode_workspace_bytes(B, Hq, nq, splits)
     if workspace is None:
         workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
@@ -199,13 +204,15 @@ def attention_decode(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optio
         out = torch.empty((B, nq, Hq, D), dtype=torch.bfloat16, device=dev)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, nq), dtype=torch.float32, device=dev)
-    check(lib().qk4v8_attention_decode(q.codes.data_ptr(), q.scales.data_ptr(), B, Hq, nq, q.cap,
-                                       k.codes.data_ptr(), k.scales.data_ptr(), v.codes.data_ptr(),
-                                       v.scales.data_ptr(), k.H, k.cap, _ptr(sl), int(max_seqlen),
-                                       int(bool(causal_in_block)), float(softmax_scale or 0.0), int(splits),
-                                       workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                       out.data_ptr(), _ptr(lse), _ptr(dev_status), _stream(dev)),
-          "qk4v8_attention_decode")
+    head = (q.codes.data_ptr(), q.scales.data_ptr(), B, Hq, nq, q.cap, k.codes.data_ptr(), k.scales.data_ptr(),
+            v.codes.data_ptr(), v.scales.data_ptr(), k.H, k.cap, _ptr(sl), int(max_seqlen),
+            int(bool(causal_in_block)))
+    tail = (float(softmax_scale or 0.0), int(splits), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), out.data_ptr(), _ptr(lse), _ptr(dev_status), _stream(dev))
+    if window:
+        check(lib().qk4v8_attention_decode_window(*head, int(window), *tail), "qk4v8_attention_decode_window")
+    else:
+        check(lib().qk4v8_attention_decode(*head, *tail), "qk4v8_attention_decode")
     return (out, lse) if return_lse else out
 
 
@@ -217,16 +224,16 @@ def attention_decode_bf16(q: torch.Tensor, k: MXFP4, v: MXFP8V, seqlens_k, max_s
                           causal_in_block: bool = True, softmax_scale: Optional[float] = None, num_splits: int = 0,
                           workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                           lse: Optional[torch.Tensor] = None, return_lse: bool = False,
-                          dev_status: Optional[torch.Tensor] = None):
+                          dev_status: Optional[torch.Tensor] = None, window: int = 0):
     """Decode step from bf16 queries q [B, nq, Hq, 128]; the query is MXFP4-quantized inside the call.
-    Returns out bf16 [B, nq, Hq, 128] (and lse [B, Hq, nq])."""
+    Returns out bf16 [B, nq, Hq, 128] (and lse [B, Hq, nq]). window as for attention_decode."""
     _check_bf16(q, "q")
     dev = q.device
     B, nq, Hq, _ = q.shape
     sl = _seqlens(seqlens_k, B, dev)
     if max_seqlen is None:
         max_seqlen = k.cap
-    splits = num_splits if num_splits > 0 else decode_default_splits(B, Hq, k.H, nq, max_seqlen)
+    splits = num_splits if num_splits > 0 else decode_default_splits(B, Hq, k.H, nq, max_seqlen, window)
     need = decode_bf16_workspace_bytes(B, Hq, k.H, nq, splits)
     if workspace is None and need:
         workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
@@ -235,12 +242,15 @@ def attention_decode_bf16(q: torch.Tensor, k: MXFP4, v: MXFP8V, seqlens_k, max_s
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, nq), dtype=torch.float32, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    check(lib().qk4v8_attention_decode_bf16(q.data_ptr(), B, Hq, nq, q.stride(0), q.stride(1), q.stride(2),
-                                            k.codes.data_ptr(), k.scales.data_ptr(), v.codes.data_ptr(),
-                                            v.scales.data_ptr(), k.H, k.cap, _ptr(sl), int(max_seqlen),
-                                            int(bool(causal_in_block)), float(softmax_scale or 0.0), int(splits),
-                                            _ptr(workspace), ws_bytes, out.data_ptr(), _ptr(lse), _ptr(dev_status),
-                                            _stream(dev)), "qk4v8_attention_decode_bf16")
+    head = (q.data_ptr(), B, Hq, nq, q.stride(0), q.stride(1), q.stride(2), k.codes.data_ptr(), k.scales.data_ptr(),
+            v.codes.data_ptr(), v.scales.data_ptr(), k.H, k.cap, _ptr(sl), int(max_seqlen),
+            int(bool(causal_in_block)))
+    tail = (float(softmax_scale or 0.0), int(splits), _ptr(workspace), ws_bytes, out.data_ptr(), _ptr(lse),
+            _ptr(dev_status), _stream(dev))
+    if window:
+        check(lib().qk4v8_attention_decode_bf16_window(*head, int(window), *tail), "qk4v8_attention_decode_bf16_window")
+    else:
+        check(lib().qk4v8_attention_decode_bf16(*head, *tail), "qk4v8_attention_decode_bf16")
     return (out, lse) if return_lse else out
 
 

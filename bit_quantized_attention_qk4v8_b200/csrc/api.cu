@@ -335,6 +335,15 @@ int qk4v8_decode_default_splits(int B, int Hq, int Hkv, int nq, int max_seqlen) 
 
 namespace {
 
+// Largest number of keys one sequence's query block sees: max_seqlen, or with
+// a window the window plus the block, plus up to 127 keys of the tile that
+// holds the window's first key.
+int window_span(int max_seqlen, int nq, int window) {
+    if (window <= 0) return max_seqlen;
+    const int64_t span = static_cast<int64_t>(window) + nq + 127;
+    return span < max_seqlen ? static_cast<int>(span) : max_seqlen;
+}
+
 // Query of a decode call: packed MXFP4 (codes, scales, cap) or bf16 rows
 // [b][t][h][128] with element strides, quantized inside the kernel.
 struct DecodeQuery {
@@ -363,9 +372,9 @@ bool gqa_rows(int Hq, int Hkv, int nq) {
 // partials to the workspace and the caller runs the merge.
 int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k_codes, const uint8_t *k_scales,
                    const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k,
-                   int max_seqlen, int causal_in_block, float softmax_scale, int num_splits, void *workspace,
-                   size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, cudaStream_t stream,
-                   int *splits_used, bool *direct) {
+                   int max_seqlen, int causal_in_block, int window, float softmax_scale, int num_splits,
+                   void *workspace, size_t workspace_bytes, void *out, float *lse, int32_t *dev_status,
+                   cudaStream_t stream, int *splits_used, bool *direct) {
     int st;
     if (q.bf16) {
         if (!aligned16(q.bf16) || q.sb % 8 || q.st % 8 || q.sh % 8 || q.sb < 0 || q.st < 0 || q.sh < 0)
@@ -389,7 +398,13 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
         return set_error(QK4V8_ERR_INVALID_ARG, "bf16 Q in the split kernel needs (Hq/Hkv)*nq < %d",
                          qk4v8::kGqaMinRows);
     if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
-    const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen);
+    if (window < 0) return set_error(QK4V8_ERR_INVALID_ARG, "window must be >= 0 (0: none)");
+    if (window > 0 && (Hq / Hkv) * nq > qk4v8::kDecodeMaxRows)
+        return set_error(QK4V8_ERR_INVALID_ARG, "a window needs (Hq/Hkv)*nq <= %d query rows per KV head",
+                         qk4v8::kDecodeMaxRows);
+    // Keys a sequence's query block can see, for planning the splits.
+    const int span = window_span(max_seqlen, nq, window);
+    const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, span);
     // Direct output: the swap-AB kernel with one split, and the GQA decode kernel
     // always (with splits, its own merge launch finishes the cut sequences).
     const bool direct_out = out && ((splits == 1 && swap_ab_rows(Hq, Hkv, nq)) || gqa_rows(Hq, Hkv, nq));
@@ -401,7 +416,7 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
     CUtensorMap tk, tv;
     if ((st = make_k_map(&tk, k_codes, B * Hkv, kv_cap)) || (st = make_v_map(&tv, v_codes, B * Hkv, kv_cap)))
         return st;
-    const int tiles = (max_seqlen + 127) / 128;
+    const int tiles = (span + 127) / 128;
     qk4v8::AttnParams p{};
     p.q_codes = q.codes;
     p.q_scales = q.scales;
@@ -421,6 +436,7 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
     p.kv_cap = kv_cap;
     p.Lk = max_seqlen;
     p.causal = causal_in_block ? 1 : 0;
+    p.window = window;
     p.scale_log2 = resolve_scale(softmax_scale) * kLog2e;
     p.decode = 1;
     p.n_qtiles = 1;
@@ -468,8 +484,8 @@ int qk4v8_attention_decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scal
     q.scales = q_scales;
     q.cap = q_cap;
     return decode_splitkv(q, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
-                          causal_in_block, softmax_scale, num_splits, workspace, workspace_bytes, nullptr, nullptr,
-                          dev_status, static_cast<cudaStream_t>(stream), &splits, &direct);
+                          causal_in_block, 0, softmax_scale, num_splits, workspace, workspace_bytes, nullptr,
+                          nullptr, dev_status, static_cast<cudaStream_t>(stream), &splits, &direct);
 }
 
 int qk4v8_decode_merge(const void *workspace, size_t workspace_bytes, int B, int Hq, int nq, int num_splits,
@@ -492,11 +508,12 @@ int qk4v8_decode_merge(const void *workspace, size_t workspace_bytes, int B, int
     return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "decode merge launch");
 }
 
-int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
-                           const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
-                           const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
-                           int causal_in_block, float softmax_scale, int num_splits, void *workspace,
-                           size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, void *stream) {
+int qk4v8_attention_decode_window(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq,
+                                  int q_cap, const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
+                                  const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k,
+                                  int max_seqlen, int causal_in_block, int window, float softmax_scale,
+                                  int num_splits, void *workspace, size_t workspace_bytes, void *out, float *lse,
+                                  int32_t *dev_status, void *stream) {
     if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
     int splits = 0;
     bool direct = false;
@@ -505,10 +522,24 @@ int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int 
     q.scales = q_scales;
     q.cap = q_cap;
     int st = decode_splitkv(q, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
-                            causal_in_block, softmax_scale, num_splits, workspace, workspace_bytes, out, lse,
+                            causal_in_block, window, softmax_scale, num_splits, workspace, workspace_bytes, out, lse,
                             dev_status, static_cast<cudaStream_t>(stream), &splits, &direct);
     if (st || direct) return st;
     return qk4v8_decode_merge(workspace, workspace_bytes, B, Hq, nq, splits, out, lse, stream);
+}
+
+int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
+                           const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
+                           const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
+                           int causal_in_block, float softmax_scale, int num_splits, void *workspace,
+                           size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, void *stream) {
+    return qk4v8_attention_decode_window(q_codes, q_scales, B, Hq, nq, q_cap, k_codes, k_scales, v_codes, v_scales,
+                                         Hkv, kv_cap, seqlens_k, max_seqlen, causal_in_block, 0, softmax_scale,
+                                         num_splits, workspace, workspace_bytes, out, lse, dev_status, stream);
+}
+
+int qk4v8_decode_default_splits_window(int B, int Hq, int Hkv, int nq, int max_seqlen, int window) {
+    return qk4v8_decode_default_splits(B, Hq, Hkv, nq, window_span(max_seqlen, nq, window));
 }
 
 size_t qk4v8_decode_bf16_workspace_bytes(int B, int Hq, int Hkv, int nq, int num_splits) {
@@ -533,12 +564,29 @@ int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_
                                 const int32_t *seqlens_k, int max_seqlen, int causal_in_block, float softmax_scale,
                                 int num_splits, void *workspace, size_t workspace_bytes, void *out, float *lse,
                                 int32_t *dev_status, void *stream) {
+    return qk4v8_attention_decode_bf16_window(q, B, Hq, nq, q_stride_b, q_stride_t, q_stride_h, k_codes, k_scales,
+                                              v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen, causal_in_block,
+                                              0, softmax_scale, num_splits, workspace, workspace_bytes, out, lse,
+                                              dev_status, stream);
+}
+
+int qk4v8_attention_decode_bf16_window(const void *q, int B, int Hq, int nq, int64_t q_stride_b,
+                                       int64_t q_stride_t, int64_t q_stride_h, const uint8_t *k_codes,
+                                       const uint8_t *k_scales, const uint8_t *v_codes, const uint8_t *v_scales,
+                                       int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
+                                       int causal_in_block, int window, float softmax_scale, int num_splits,
+                                       void *workspace, size_t workspace_bytes, void *out, float *lse,
+                                       int32_t *dev_status, void *stream) {
     if (!q) return set_error(QK4V8_ERR_INVALID_ARG, "q is null");
     if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq < 1 || nq > 8 || (Hq / Hkv) * nq > 128)
         return set_error(QK4V8_ERR_INVALID_ARG, "bad sizes B=%d Hq=%d Hkv=%d nq=%d", B, Hq, Hkv, nq);
     if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
-    const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen);
+    if (window < 0 || (window > 0 && (Hq / Hkv) * nq > qk4v8::kDecodeMaxRows))
+        return set_error(QK4V8_ERR_INVALID_ARG, "window must be >= 0, and > 0 only with (Hq/Hkv)*nq <= %d",
+                         qk4v8::kDecodeMaxRows);
+    const int splits =
+        num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, window_span(max_seqlen, nq, window));
     const size_t need = qk4v8_decode_bf16_workspace_bytes(B, Hq, Hkv, nq, splits);
     if (need && (!workspace || !aligned16(workspace) || workspace_bytes < need))
         return set_error(QK4V8_ERR_INVALID_ARG, "workspace must be 16-byte aligned and >= %zu bytes", need);
@@ -552,8 +600,8 @@ int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_
         dq.st = q_stride_t;
         dq.sh = q_stride_h;
         int st = decode_splitkv(dq, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k,
-                                max_seqlen, causal_in_block, softmax_scale, splits, workspace, workspace_bytes, out,
-                                lse, dev_status, s, &used, &direct);
+                                max_seqlen, causal_in_block, window, softmax_scale, splits, workspace,
+                                workspace_bytes, out, lse, dev_status, s, &used, &direct);
         if (st || direct) return st;
         return qk4v8_decode_merge(workspace, workspace_bytes, B, Hq, nq, used, out, lse, stream);
     }
@@ -584,7 +632,7 @@ int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_
     dq.scales = qs;
     dq.cap = 128;
     st = decode_splitkv(dq, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
-                        causal_in_block, softmax_scale, splits, rest, rest_bytes, gqa ? out : nullptr,
+                        causal_in_block, window, softmax_scale, splits, rest, rest_bytes, gqa ? out : nullptr,
                         gqa ? lse : nullptr, dev_status, s, &used, &direct);
     if (st || direct) return st;
     return qk4v8_decode_merge(rest, rest_bytes, B, Hq, nq, used, out, lse, stream);

@@ -250,7 +250,10 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
     const int R = p.G * nq;
     const int L = imax(0, imin(p.seqlens[b], p.kv_cap));
     const int n_tiles = (L + 127) / 128;
-    const int tile_begin = split * p.split_tiles;
+    // Keys below lo are outside the window: the splits start at its first tile
+    // (tile indices below are absolute).
+    const int lo = kv_window_lo(p, L);
+    const int tile_begin = lo / 128 + split * p.split_tiles;
     const int tile_end = imin(tile_begin + p.split_tiles, n_tiles);
     const int T = tile_end - tile_begin;
 
@@ -618,7 +621,8 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
                 u[i + 1] = v.y;
             }
             if (!(it > 0 && ok && tok < L - (p.causal ? nq - 1 : 0))) {
-                const bool any_key = ok && tok < L;
+                // (Keys below the window's lo lie in the first tile of the first split.)
+                const bool any_key = ok && tok < L && tok >= lo;
 #pragma unroll
                 for (int i = 0; i < NC; ++i)
                     if (!(any_key && tok < lim_s[c0 + i])) u[i] = -INFINITY;

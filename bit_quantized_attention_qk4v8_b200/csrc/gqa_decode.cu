@@ -121,6 +121,10 @@ __device__ __forceinline__ uint32_t gd_sf_id(uint32_t idesc, uint32_t id) { retu
 
 }  // namespace
 
+// kWindow: the instance for draft-block attention, whose query rows see only
+// keys from the window's first key (kv_window_lo) on; the other instance is
+// the plain decode, with no per-key lower bound in its softmax loop.
+template <bool kWindow>
 __global__ void __launch_bounds__(kGdThreads, 1)
     qk4v8_gqa_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                             const AttnParams p) {
@@ -630,6 +634,10 @@ __global__ void __launch_bounds__(kGdThreads, 1)
             const int NP = (T + 1) / 2;
             float mneg = 0.f;  // -m_w (log2 units)
             int e = 0;         // m_w - m_O
+            // m_O comes from the first half (64 keys) of the unit's first tile that
+            // holds a visible key: the second half when a window starts there.
+            const int u_lo = kWindow ? kv_window_lo(p, u.L) : 0;  // the unit's first visible key
+            const int mo_half = kWindow && u_lo - u.tile_begin * 128 >= 64 ? 1 : 0;
             auto receive_mo = [&]() -> bool {
                 if (!__all_sync(0xffffffffu, wait_bar(&mo_bar[grp], c & 1, abort_flag, p.status))) return false;
                 const float m0 = __uint_as_float(lds32(a_m));
@@ -652,6 +660,7 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const int jv = ti < T ? imax(0, imin(limit - (u.tile_begin + ti) * 128, 128)) : 0;  // keys j < jv
+                const int jlo = kWindow ? u_lo - (u.tile_begin + ti) * 128 : 0;  // and keys j >= jlo (window)
                 int eb[4];  // e + x of each block when it was encoded
                 // The tile in two halves of 64 keys, to bound the registers held at once.
                 // S is released to the tensor core once the second half has been read.
@@ -669,8 +678,15 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&s_free[set]);  // the tensor core may now compute S(gp+2)
                     }
-                    // Keys at or past the row's bound are -inf (raw scores; the scale is positive).
-                    if (jv < 64 * hh + 64) {
+                    // Keys at or past the row's bound, and before the window, are -inf
+                    // (raw scores; the scale is positive).
+                    if (kWindow) {
+                        if (jv < 64 * hh + 64 || jlo > 64 * hh) {
+#pragma unroll
+                            for (int j = 0; j < 64; ++j)
+                                if (64 * hh + j >= jv || 64 * hh + j < jlo) sh[j] = 0xFF800000u;
+                        }
+                    } else if (jv < 64 * hh + 64) {
 #pragma unroll
                         for (int j = 0; j < 64; ++j)
                             if (64 * hh + j >= jv) sh[j] = 0xFF800000u;
@@ -678,10 +694,14 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                     const float bmx0 = max32(*reinterpret_cast<const uint32_t (*)[32]>(&sh[0])) * sc;
                     const float bmx1 = max32(*reinterpret_cast<const uint32_t (*)[32]>(&sh[32])) * sc;
                     const float hm = fmaxf(bmx0, bmx1);
-                    if (k == 0 && hh == 0) {
-                        // The first half of the unit's first tile fixes m_O: the row's largest
-                        // score there. It holds the unit's first key, so a row with no key in
-                        // it has none in the unit. Its owner posts it to the other three.
+                    const bool mo_post = k == 0 && half == 0 && hh == mo_half;
+                    const bool mo_take = k == 0 && half == 1 && hh == 0;
+                    if (kWindow ? (mo_post || mo_take) : (k == 0 && hh == 0)) {
+                        // The first half of the unit's first tile with a visible key fixes
+                        // m_O: the row's largest score there. It holds the unit's first
+                        // visible key, so a row with no key in it has none in the unit. Its
+                        // owner posts it to the other three. (With a window, a half before
+                        // it is all masked: its P is zero, whatever the reference.)
                         if (half == 0) {
                             mneg = hm > -INFINITY ? -hm : 0.f;
                             e = 0;
@@ -944,7 +964,10 @@ cudaError_t launch_gqa_decode(const CUtensorMap &tk, const CUtensorMap &tv, cons
     if (e != cudaSuccess) return e;
     int sms = dev < kMaxDevices ? sm_count[dev] : 0;
     if (dev >= kMaxDevices || !configured[dev]) {
-        e = cudaFuncSetAttribute(qk4v8_gqa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(qk4v8_gqa_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GdSmem::kBytes);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(qk4v8_gqa_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GdSmem::kBytes);
         if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -956,7 +979,10 @@ cudaError_t launch_gqa_decode(const CUtensorMap &tk, const CUtensorMap &tv, cons
     }
     // Persistent: one CTA per SM (shared memory and the 512 TMEM columns allow no
     // more); the kernel schedules the work over the grid itself.
-    qk4v8_gqa_decode_kernel<<<sms, kGdThreads, GdSmem::kBytes, stream>>>(tk, tv, p);
+    if (p.window > 0)
+        qk4v8_gqa_decode_kernel<true><<<sms, kGdThreads, GdSmem::kBytes, stream>>>(tk, tv, p);
+    else
+        qk4v8_gqa_decode_kernel<false><<<sms, kGdThreads, GdSmem::kBytes, stream>>>(tk, tv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess || !p.direct_out || p.num_splits < 2) return e;
     return launch_cut_merge(p, stream);

@@ -12,6 +12,14 @@ namespace qk4v8 {
 __device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
 __device__ __forceinline__ int imax(int a, int b) { return a > b ? a : b; }
 
+// First key a decode query block of a sequence of L keys may see: with a
+// window, the last `window` keys before the block's Sq tokens (MiMo DFlash
+// article, section on block-diffusion speculative decoding: the draft block
+// attends to a sliding window over the most recent context), else key 0.
+__device__ __forceinline__ int kv_window_lo(const AttnParams &p, int L) {
+    return p.window > 0 ? imax(0, L - p.Sq - p.window) : 0;
+}
+
 __device__ __forceinline__ bool aborted(volatile uint32_t *flag, const int32_t *status) {
     if (*flag) return true;
     if (status && *reinterpret_cast<const volatile int32_t *>(status) != 0) {

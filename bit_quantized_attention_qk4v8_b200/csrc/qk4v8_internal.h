@@ -29,6 +29,10 @@ struct AttnParams {
     int q_cap, kv_cap;
     int Lk;                   // KV length when seqlens is null
     int causal;
+    // Decode only: > 0 limits every query row of a sequence of L keys to keys
+    // j >= L - Sq - window (the last `window` keys before the Sq-token block, and
+    // the block); 0: no lower bound.
+    int window;
     float scale_log2;         // softmax_scale * log2(e)
     int decode;               // 0: units (b, h_q, q tile); 1: units (b, h_kv, split)
     int n_qtiles;

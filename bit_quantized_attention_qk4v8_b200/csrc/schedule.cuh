@@ -11,15 +11,19 @@
 namespace qk4v8 {
 
 // One piece of work: key tiles [tile_begin, tile_begin + T) of the sequence
-// (b, h_kv). `whole` when the piece is the whole sequence; otherwise it is
-// piece `slot` of `n_pieces`, written as a partial (O / l, log2-sum-exp).
+// (b, h_kv), absolute tile indices. `whole` when the piece is the whole
+// sequence; otherwise it is piece `slot` of `n_pieces`, written as a partial
+// (O / l, log2-sum-exp).
 struct GdUnit {
     int b, h_kv, L, tile_begin, T, slot, n_pieces;
     bool whole;
 };
 
+// Key tiles of sequence b the schedule covers: from the tile holding its first
+// visible key to its last key.
 __device__ __forceinline__ int gd_tiles(const AttnParams &p, int b) {
-    return (imax(0, imin(p.seqlens[b], p.kv_cap)) + 127) / 128;
+    const int L = imax(0, imin(p.seqlens[b], p.kv_cap));
+    return (L + 127) / 128 - kv_window_lo(p, L) / 128;
 }
 
 // Schedule of one CTA, computed once at the start.
@@ -155,7 +159,7 @@ __device__ __forceinline__ void gd_piece(const AttnParams &p, const GdSched &sc,
     u.b = b;
     u.h_kv = h;
     u.L = imax(0, imin(p.seqlens[b], p.kv_cap));
-    u.tile_begin = static_cast<int>(t0);
+    u.tile_begin = kv_window_lo(p, u.L) / 128 + static_cast<int>(t0);
     u.T = Ts > 0 ? static_cast<int>(t1 - t0) : 0;
     u.whole = t0 == 0 && t1 == Ts;
     if (Ts > 0) {
@@ -179,7 +183,7 @@ __device__ __forceinline__ bool gd_next(const AttnParams &p, const GdSched &sc, 
         u.b = rem / p.Hkv;
         u.L = imax(0, imin(p.seqlens[u.b], p.kv_cap));
         const int n_tiles = (u.L + 127) / 128;
-        u.tile_begin = split * p.split_tiles;
+        u.tile_begin = kv_window_lo(p, u.L) / 128 + split * p.split_tiles;
         u.T = imax(0, imin(u.tile_begin + p.split_tiles, n_tiles) - u.tile_begin);
         u.slot = split;
         u.n_pieces = p.num_splits;

@@ -251,6 +251,44 @@ QK4V8_API int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_sc
                            void *out, float *lse, int32_t *dev_status, void *stream);
 
 /*
+ * Draft-block attention: decode with a sliding window (MiMo DFlash article,
+ * section on block-diffusion speculative decoding: the draft model predicts a
+ * block of 8 tokens in one forward; its attention sees the in-block positions
+ * together with a sliding window over the most recent 1024 context tokens).
+ * Reading taken: for a sequence of L keys whose last nq positions are the
+ * query block, every query row sees keys j >= max(0, L - nq - window) (the
+ * last `window` keys before the block, and the block), and, with
+ * causal_in_block, only up to its own position; with causal_in_block = 0 the
+ * block is non-causal, as in the draft model. window = 0 is plain decode.
+ * Only the keys in the window are streamed: the splits cover the tiles from
+ * the one holding the window's first key.
+ *   window   >= 0; a window needs (Hq / Hkv) * nq <= 64 query rows per KV head
+ *   other arguments, layouts and errors as for qk4v8_attention_decode (packed
+ *   Q) and qk4v8_attention_decode_bf16 (bf16 Q, with its workspace rule);
+ *   num_splits = 0 picks qk4v8_decode_default_splits_window.
+ * qk4v8_decode_default_splits_window: the default split count for such a call
+ * (qk4v8_decode_default_splits over the keys one block can see).
+ */
+QK4V8_API int qk4v8_attention_decode_window(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq,
+                                            int q_cap, const uint8_t *k_codes, const uint8_t *k_scales,
+                                            const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap,
+                                            const int32_t *seqlens_k, int max_seqlen, int causal_in_block,
+                                            int window, float softmax_scale, int num_splits, void *workspace,
+                                            size_t workspace_bytes, void *out, float *lse, int32_t *dev_status,
+                                            void *stream);
+
+QK4V8_API int qk4v8_attention_decode_bf16_window(const void *q, int B, int Hq, int nq, int64_t q_stride_b,
+                                                 int64_t q_stride_t, int64_t q_stride_h, const uint8_t *k_codes,
+                                                 const uint8_t *k_scales, const uint8_t *v_codes,
+                                                 const uint8_t *v_scales, int Hkv, int kv_cap,
+                                                 const int32_t *seqlens_k, int max_seqlen, int causal_in_block,
+                                                 int window, float softmax_scale, int num_splits, void *workspace,
+                                                 size_t workspace_bytes, void *out, float *lse, int32_t *dev_status,
+                                                 void *stream);
+
+QK4V8_API int qk4v8_decode_default_splits_window(int B, int Hq, int Hkv, int nq, int max_seqlen, int window);
+
+/*
  * Decode step from bf16 queries (MpFA QK4V8 article, section 3.2: the query's
  * MXFP4 scales are computed as it is loaded, inside the attention call).
  * Same result, bit for bit, as qk4v8_quantize_qk (capacity 128) followed by
