@@ -22,10 +22,11 @@ import torch
 from ._lib import QK4V8Error, check, lib
 
 __all__ = [
-    "MXFP4", "MXFP8V", "QK4V8Error", "lib", "round_cap",
+    "MXFP4", "MXFP8V", "PagedKV", "QK4V8Error", "lib", "round_cap",
     "quantize_qk", "quantize_v", "quantize", "attention_prefill", "attention_decode",
     "decode_workspace_bytes", "decode_default_splits", "attention_decode_splitkv", "decode_merge",
     "attention_decode_bf16", "decode_bf16_workspace_bytes",
+    "paged_kv", "kv_append", "attention_decode_paged", "attention_decode_bf16_paged",
 ]
 
 D = 128
@@ -314,3 +315,131 @@ def mma_peak_run(kind: int, ctas: int, iters: int, device=None, dev_status: Opti
           "qk4v8_test_mma_peak")
     _, m, n, kk = MMA_PEAK_SHAPES[int(kind)]
     return 2 * m * n * kk * int(ctas) * int(iters)
+
+
+# ----------------------------------------------------------------------------------------------------------
+# Paged KV cache (include/qk4v8.h: qk4v8_kv_append, qk4v8_attention_decode_paged).
+
+@dataclass
+class PagedKV:
+    """Packed KV cache in pools of 128-token pages, and the per-sequence state.
+
+    k_codes uint8 [P, Hkv, 128, 64], k_scales uint8 [P, Hkv, 512],
+    v_codes uint8 [P, Hkv, 128, 128], v_scales uint8 [P, Hkv, 512] (P pages);
+    block_table int32 [B, max_pages]: page of each 128-token block of a sequence;
+    seqlens int32 [B]: tokens held; v_tail bf16 [B, Hkv, 32, 128]: the open V
+    group of each sequence and head, which every append reads and refreshes."""
+    k_codes: torch.Tensor
+    k_scales: torch.Tensor
+    v_codes: torch.Tensor
+    v_scales: torch.Tensor
+    v_tail: torch.Tensor
+    block_table: torch.Tensor
+    seqlens: torch.Tensor
+    hadamard_k: bool = False
+
+    @property
+    def num_pages(self) -> int:
+        return self.k_codes.shape[0]
+
+    @property
+    def Hkv(self) -> int:
+        return self.k_codes.shape[1]
+
+    @property
+    def B(self) -> int:
+        return self.block_table.shape[0]
+
+    @property
+    def max_pages(self) -> int:
+        return self.block_table.shape[1]
+
+
+def paged_kv(B: int, Hkv: int, num_pages: int, block_table: torch.Tensor, device="cuda",
+             hadamard_k: bool = False) -> PagedKV:
+    """An empty paged cache (every sequence of length 0) over a new pool of num_pages pages.
+    block_table: int32 [B, max_pages] page indices, owned by the caller's page allocator."""
+    dev = torch.device(device)
+    bt = block_table.to(device=dev, dtype=torch.int32).contiguous()
+    if bt.dim() != 2 or bt.shape[0] != B:
+        raise ValueError("block_table must be [B, max_pages]")
+    u8 = torch.uint8
+    return PagedKV(k_codes=torch.empty((num_pages, Hkv, 128, 64), dtype=u8, device=dev),
+                   k_scales=torch.empty((num_pages, Hkv, 512), dtype=u8, device=dev),
+                   v_codes=torch.empty((num_pages, Hkv, 128, 128), dtype=u8, device=dev),
+                   v_scales=torch.empty((num_pages, Hkv, 512), dtype=u8, device=dev),
+                   v_tail=torch.empty((B, Hkv, 32, 128), dtype=torch.bfloat16, device=dev),
+                   block_table=bt, seqlens=torch.zeros((B,), dtype=torch.int32, device=dev), hadamard_k=hadamard_k)
+
+
+def kv_append(cache: PagedKV, k_new: torch.Tensor, v_new: torch.Tensor, dev_status: Optional[torch.Tensor] = None):
+    """Append k_new, v_new (bf16 [B, n_new, Hkv, 128], same strides) to every sequence
+    (qk4v8_kv_append); cache.seqlens advances by n_new on the device."""
+    _check_bf16(k_new, "k_new")
+    _check_bf16(v_new, "v_new")
+    if k_new.shape != v_new.shape or k_new.stride() != v_new.stride():
+        raise ValueError("k_new and v_new must have the same shape and strides")
+    B, n_new, Hkv, _ = k_new.shape
+    check(lib().qk4v8_kv_append(k_new.data_ptr(), v_new.data_ptr(), B, n_new, Hkv, D, k_new.stride(0),
+                                k_new.stride(1), k_new.stride(2), cache.seqlens.data_ptr(),
+                                cache.seqlens.data_ptr(), cache.block_table.data_ptr(), cache.max_pages,
+                                cache.num_pages, cache.k_codes.data_ptr(), cache.k_scales.data_ptr(),
+                                cache.v_codes.data_ptr(), cache.v_scales.data_ptr(), cache.v_tail.data_ptr(),
+                                int(cache.hadamard_k), _ptr(dev_status), _stream(k_new.device)), "qk4v8_kv_append")
+    return cache
+
+
+def _paged_call_args(cache: PagedKV):
+    return (cache.k_codes.data_ptr(), cache.k_scales.data_ptr(), cache.v_codes.data_ptr(), cache.v_scales.data_ptr(),
+            cache.Hkv, cache.num_pages, cache.block_table.data_ptr(), cache.max_pages, cache.seqlens.data_ptr())
+
+
+def attention_decode_paged(q: MXFP4, cache: PagedKV, max_seqlen: int, causal_in_block: bool = True,
+                           window: int = 0, softmax_scale: Optional[float] = None, num_splits: int = 0,
+                           workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                           lse: Optional[torch.Tensor] = None, return_lse: bool = False,
+                           dev_status: Optional[torch.Tensor] = None):
+    """Decode / verify / draft-block attention over a paged cache (qk4v8_attention_decode_paged)."""
+    dev = q.codes.device
+    B, Hq, nq = q.B, q.H, q.length
+    splits = num_splits if num_splits > 0 else decode_default_splits(B, Hq, cache.Hkv, nq, max_seqlen, window)
+    if workspace is None:
+        workspace = torch.empty((max(16, decode_workspace_bytes(B, Hq, nq, splits)),), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((B, nq, Hq, D), dtype=torch.bfloat16, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, nq), dtype=torch.float32, device=dev)
+    check(lib().qk4v8_attention_decode_paged(q.codes.data_ptr(), q.scales.data_ptr(), B, Hq, nq, q.cap,
+                                             *_paged_call_args(cache), int(max_seqlen), int(bool(causal_in_block)),
+                                             int(window), float(softmax_scale or 0.0), int(splits),
+                                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                             out.data_ptr(), _ptr(lse), _ptr(dev_status), _stream(dev)),
+          "qk4v8_attention_decode_paged")
+    return (out, lse) if return_lse else out
+
+
+def attention_decode_bf16_paged(q: torch.Tensor, cache: PagedKV, max_seqlen: int, causal_in_block: bool = True,
+                                window: int = 0, softmax_scale: Optional[float] = None, num_splits: int = 0,
+                                workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                                lse: Optional[torch.Tensor] = None, return_lse: bool = False,
+                                dev_status: Optional[torch.Tensor] = None):
+    """Decode step from bf16 queries q [B, nq, Hq, 128] over a paged cache (qk4v8_attention_decode_bf16_paged)."""
+    _check_bf16(q, "q")
+    dev = q.device
+    B, nq, Hq, _ = q.shape
+    splits = num_splits if num_splits > 0 else decode_default_splits(B, Hq, cache.Hkv, nq, max_seqlen, window)
+    need = decode_bf16_workspace_bytes(B, Hq, cache.Hkv, nq, splits)
+    if workspace is None and need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((B, nq, Hq, D), dtype=torch.bfloat16, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, nq), dtype=torch.float32, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib().qk4v8_attention_decode_bf16_paged(q.data_ptr(), B, Hq, nq, q.stride(0), q.stride(1), q.stride(2),
+                                                  *_paged_call_args(cache), int(max_seqlen),
+                                                  int(bool(causal_in_block)), int(window),
+                                                  float(softmax_scale or 0.0), int(splits), _ptr(workspace), ws_bytes,
+                                                  out.data_ptr(), _ptr(lse), _ptr(dev_status), _stream(dev)),
+          "qk4v8_attention_decode_bf16_paged")
+    return (out, lse) if return_lse else out

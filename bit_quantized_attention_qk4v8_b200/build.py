@@ -10,7 +10,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqk4v8.so")
-SOURCES = ["quantize.cu", "attention.cu", "prefill.cu", "decode.cu", "gqa_decode.cu", "mma_peak.cu", "api.cu"]
+SOURCES = ["quantize.cu", "attention.cu", "prefill.cu", "decode.cu", "gqa_decode.cu", "mma_peak.cu", "kv_cache.cu",
+           "api.cu"]
 HEADERS = ["ptx.cuh", "pipeline.cuh", "mx_encode.cuh", "tile_ops.cuh", "schedule.cuh", "qk4v8_internal.h"]
 
 NVCC_FLAGS = [

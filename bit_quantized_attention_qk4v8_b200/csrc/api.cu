@@ -370,11 +370,17 @@ bool gqa_rows(int Hq, int Hkv, int nq) {
 // kernel. With `out` given and a single split on the swap-AB kernel, the kernel
 // writes out (and lse) itself and *direct is set; otherwise it writes the split
 // partials to the workspace and the caller runs the merge.
+// Paged K/V pools of a decode call (block_table null: contiguous caches).
+struct KvPages {
+    const int32_t *block_table = nullptr;
+    int max_pages = 0, num_pages = 0;
+};
+
 int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k_codes, const uint8_t *k_scales,
-                   const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k,
-                   int max_seqlen, int causal_in_block, int window, float softmax_scale, int num_splits,
-                   void *workspace, size_t workspace_bytes, void *out, float *lse, int32_t *dev_status,
-                   cudaStream_t stream, int *splits_used, bool *direct) {
+                   const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap, const KvPages &pages,
+                   const int32_t *seqlens_k, int max_seqlen, int causal_in_block, int window, float softmax_scale,
+                   int num_splits, void *workspace, size_t workspace_bytes, void *out, float *lse,
+                   int32_t *dev_status, cudaStream_t stream, int *splits_used, bool *direct) {
     int st;
     if (q.bf16) {
         if (!aligned16(q.bf16) || q.sb % 8 || q.st % 8 || q.sh % 8 || q.sb < 0 || q.st < 0 || q.sh < 0)
@@ -399,6 +405,16 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
                          qk4v8::kGqaMinRows);
     if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
     if (window < 0) return set_error(QK4V8_ERR_INVALID_ARG, "window must be >= 0 (0: none)");
+    if (pages.block_table) {
+        if (pages.max_pages <= 0 || pages.num_pages <= 0 ||
+            static_cast<int64_t>(pages.num_pages) * Hkv >= (int64_t{1} << 31) ||
+            static_cast<int64_t>(pages.max_pages) * 128 >= (int64_t{1} << 31))
+            return set_error(QK4V8_ERR_INVALID_ARG, "bad page pool: num_pages=%d max_pages=%d", pages.num_pages,
+                             pages.max_pages);
+        if ((Hq / Hkv) * nq > qk4v8::kDecodeMaxRows)
+            return set_error(QK4V8_ERR_INVALID_ARG, "a paged cache needs (Hq/Hkv)*nq <= %d query rows per KV head",
+                             qk4v8::kDecodeMaxRows);
+    }
     if (window > 0 && (Hq / Hkv) * nq > qk4v8::kDecodeMaxRows)
         return set_error(QK4V8_ERR_INVALID_ARG, "a window needs (Hq/Hkv)*nq <= %d query rows per KV head",
                          qk4v8::kDecodeMaxRows);
@@ -414,7 +430,10 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
         return set_error(QK4V8_ERR_INVALID_ARG, "workspace must be 16-byte aligned and >= %zu bytes", need);
     if ((st = check_device())) return st;
     CUtensorMap tk, tv;
-    if ((st = make_k_map(&tk, k_codes, B * Hkv, kv_cap)) || (st = make_v_map(&tv, v_codes, B * Hkv, kv_cap)))
+    // A paged pool is the contiguous layout with num_pages rows of capacity 128.
+    const int map_rows = pages.block_table ? pages.num_pages * Hkv : B * Hkv;
+    const int map_cap = pages.block_table ? 128 : kv_cap;
+    if ((st = make_k_map(&tk, k_codes, map_rows, map_cap)) || (st = make_v_map(&tv, v_codes, map_rows, map_cap)))
         return st;
     const int tiles = (span + 127) / 128;
     qk4v8::AttnParams p{};
@@ -437,6 +456,9 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
     p.Lk = max_seqlen;
     p.causal = causal_in_block ? 1 : 0;
     p.window = window;
+    p.block_table = pages.block_table;
+    p.max_pages = pages.max_pages;
+    p.num_pages = pages.num_pages;
     p.scale_log2 = resolve_scale(softmax_scale) * kLog2e;
     p.decode = 1;
     p.n_qtiles = 1;
@@ -483,9 +505,9 @@ int qk4v8_attention_decode_splitkv(const uint8_t *q_codes, const uint8_t *q_scal
     q.codes = q_codes;
     q.scales = q_scales;
     q.cap = q_cap;
-    return decode_splitkv(q, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
-                          causal_in_block, 0, softmax_scale, num_splits, workspace, workspace_bytes, nullptr,
-                          nullptr, dev_status, static_cast<cudaStream_t>(stream), &splits, &direct);
+    return decode_splitkv(q, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, KvPages{}, seqlens_k,
+                          max_seqlen, causal_in_block, 0, softmax_scale, num_splits, workspace, workspace_bytes,
+                          nullptr, nullptr, dev_status, static_cast<cudaStream_t>(stream), &splits, &direct);
 }
 
 int qk4v8_decode_merge(const void *workspace, size_t workspace_bytes, int B, int Hq, int nq, int num_splits,
@@ -508,12 +530,15 @@ int qk4v8_decode_merge(const void *workspace, size_t workspace_bytes, int B, int
     return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "decode merge launch");
 }
 
-int qk4v8_attention_decode_window(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq,
-                                  int q_cap, const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
-                                  const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k,
-                                  int max_seqlen, int causal_in_block, int window, float softmax_scale,
-                                  int num_splits, void *workspace, size_t workspace_bytes, void *out, float *lse,
-                                  int32_t *dev_status, void *stream) {
+}  // extern "C"
+
+namespace {
+
+int decode_packed(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
+                  const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes, const uint8_t *v_scales,
+                  int Hkv, int kv_cap, const KvPages &pages, const int32_t *seqlens_k, int max_seqlen,
+                  int causal_in_block, int window, float softmax_scale, int num_splits, void *workspace,
+                  size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, void *stream) {
     if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
     int splits = 0;
     bool direct = false;
@@ -521,11 +546,45 @@ int qk4v8_attention_decode_window(const uint8_t *q_codes, const uint8_t *q_scale
     q.codes = q_codes;
     q.scales = q_scales;
     q.cap = q_cap;
-    int st = decode_splitkv(q, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
-                            causal_in_block, window, softmax_scale, num_splits, workspace, workspace_bytes, out, lse,
-                            dev_status, static_cast<cudaStream_t>(stream), &splits, &direct);
+    int st = decode_splitkv(q, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, pages, seqlens_k,
+                            max_seqlen, causal_in_block, window, softmax_scale, num_splits, workspace,
+                            workspace_bytes, out, lse, dev_status, static_cast<cudaStream_t>(stream), &splits,
+                            &direct);
     if (st || direct) return st;
     return qk4v8_decode_merge(workspace, workspace_bytes, B, Hq, nq, splits, out, lse, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int qk4v8_attention_decode_window(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq,
+                                  int q_cap, const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
+                                  const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k,
+                                  int max_seqlen, int causal_in_block, int window, float softmax_scale,
+                                  int num_splits, void *workspace, size_t workspace_bytes, void *out, float *lse,
+                                  int32_t *dev_status, void *stream) {
+    return decode_packed(q_codes, q_scales, B, Hq, nq, q_cap, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap,
+                         KvPages{}, seqlens_k, max_seqlen, causal_in_block, window, softmax_scale, num_splits,
+                         workspace, workspace_bytes, out, lse, dev_status, stream);
+}
+
+int qk4v8_attention_decode_paged(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
+                                 const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
+                                 const uint8_t *v_scales, int Hkv, int num_pages, const int32_t *block_table,
+                                 int max_pages, const int32_t *seqlens_k, int max_seqlen, int causal_in_block,
+                                 int window, float softmax_scale, int num_splits, void *workspace,
+                                 size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, void *stream) {
+    if (!block_table) return set_error(QK4V8_ERR_INVALID_ARG, "block_table is null");
+    if (max_pages <= 0 || max_pages >= (1 << 24))
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad max_pages %d", max_pages);
+    KvPages pages;
+    pages.block_table = block_table;
+    pages.max_pages = max_pages;
+    pages.num_pages = num_pages;
+    return decode_packed(q_codes, q_scales, B, Hq, nq, q_cap, k_codes, k_scales, v_codes, v_scales, Hkv,
+                         max_pages * 128, pages, seqlens_k, max_seqlen, causal_in_block, window, softmax_scale,
+                         num_splits, workspace, workspace_bytes, out, lse, dev_status, stream);
 }
 
 int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
@@ -570,13 +629,15 @@ int qk4v8_attention_decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_
                                               dev_status, stream);
 }
 
-int qk4v8_attention_decode_bf16_window(const void *q, int B, int Hq, int nq, int64_t q_stride_b,
-                                       int64_t q_stride_t, int64_t q_stride_h, const uint8_t *k_codes,
-                                       const uint8_t *k_scales, const uint8_t *v_codes, const uint8_t *v_scales,
-                                       int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
-                                       int causal_in_block, int window, float softmax_scale, int num_splits,
-                                       void *workspace, size_t workspace_bytes, void *out, float *lse,
-                                       int32_t *dev_status, void *stream) {
+}  // extern "C"
+
+namespace {
+
+int decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_stride_b, int64_t q_stride_t, int64_t q_stride_h,
+                const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes, const uint8_t *v_scales,
+                int Hkv, int kv_cap, const KvPages &pages, const int32_t *seqlens_k, int max_seqlen,
+                int causal_in_block, int window, float softmax_scale, int num_splits, void *workspace,
+                size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, void *stream) {
     if (!q) return set_error(QK4V8_ERR_INVALID_ARG, "q is null");
     if (!out || !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq < 1 || nq > 8 || (Hq / Hkv) * nq > 128)
@@ -599,7 +660,7 @@ int qk4v8_attention_decode_bf16_window(const void *q, int B, int Hq, int nq, int
         dq.sb = q_stride_b;
         dq.st = q_stride_t;
         dq.sh = q_stride_h;
-        int st = decode_splitkv(dq, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k,
+        int st = decode_splitkv(dq, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, pages, seqlens_k,
                                 max_seqlen, causal_in_block, window, softmax_scale, splits, workspace,
                                 workspace_bytes, out, lse, dev_status, s, &used, &direct);
         if (st || direct) return st;
@@ -631,11 +692,76 @@ int qk4v8_attention_decode_bf16_window(const void *q, int B, int Hq, int nq, int
     dq.codes = qc;
     dq.scales = qs;
     dq.cap = 128;
-    st = decode_splitkv(dq, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, seqlens_k, max_seqlen,
-                        causal_in_block, window, softmax_scale, splits, rest, rest_bytes, gqa ? out : nullptr,
-                        gqa ? lse : nullptr, dev_status, s, &used, &direct);
+    st = decode_splitkv(dq, B, Hq, nq, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap, pages, seqlens_k,
+                        max_seqlen, causal_in_block, window, softmax_scale, splits, rest, rest_bytes,
+                        gqa ? out : nullptr, gqa ? lse : nullptr, dev_status, s, &used, &direct);
     if (st || direct) return st;
     return qk4v8_decode_merge(rest, rest_bytes, B, Hq, nq, used, out, lse, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int qk4v8_attention_decode_bf16_window(const void *q, int B, int Hq, int nq, int64_t q_stride_b,
+                                       int64_t q_stride_t, int64_t q_stride_h, const uint8_t *k_codes,
+                                       const uint8_t *k_scales, const uint8_t *v_codes, const uint8_t *v_scales,
+                                       int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
+                                       int causal_in_block, int window, float softmax_scale, int num_splits,
+                                       void *workspace, size_t workspace_bytes, void *out, float *lse,
+                                       int32_t *dev_status, void *stream) {
+    return decode_bf16(q, B, Hq, nq, q_stride_b, q_stride_t, q_stride_h, k_codes, k_scales, v_codes, v_scales, Hkv,
+                       kv_cap, KvPages{}, seqlens_k, max_seqlen, causal_in_block, window, softmax_scale, num_splits,
+                       workspace, workspace_bytes, out, lse, dev_status, stream);
+}
+
+int qk4v8_attention_decode_bf16_paged(const void *q, int B, int Hq, int nq, int64_t q_stride_b, int64_t q_stride_t,
+                                      int64_t q_stride_h, const uint8_t *k_codes, const uint8_t *k_scales,
+                                      const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int num_pages,
+                                      const int32_t *block_table, int max_pages, const int32_t *seqlens_k,
+                                      int max_seqlen, int causal_in_block, int window, float softmax_scale,
+                                      int num_splits, void *workspace, size_t workspace_bytes, void *out, float *lse,
+                                      int32_t *dev_status, void *stream) {
+    if (!block_table) return set_error(QK4V8_ERR_INVALID_ARG, "block_table is null");
+    if (max_pages <= 0 || max_pages >= (1 << 24))
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad max_pages %d", max_pages);
+    KvPages pages;
+    pages.block_table = block_table;
+    pages.max_pages = max_pages;
+    pages.num_pages = num_pages;
+    return decode_bf16(q, B, Hq, nq, q_stride_b, q_stride_t, q_stride_h, k_codes, k_scales, v_codes, v_scales, Hkv,
+                       max_pages * 128, pages, seqlens_k, max_seqlen, causal_in_block, window, softmax_scale,
+                       num_splits, workspace, workspace_bytes, out, lse, dev_status, stream);
+}
+
+size_t qk4v8_kv_tail_bytes(int B, int Hkv) {
+    if (B <= 0 || Hkv <= 0) return 0;
+    return static_cast<size_t>(B) * Hkv * 32 * 128 * 2;
+}
+
+int qk4v8_kv_append(const void *k_new, const void *v_new, int B, int n_new, int Hkv, int d, int64_t stride_b,
+                    int64_t stride_t, int64_t stride_h, const int32_t *seqlens, int32_t *seqlens_out,
+                    const int32_t *block_table, int max_pages, int num_pages, uint8_t *k_codes, uint8_t *k_scales,
+                    uint8_t *v_codes, uint8_t *v_scales, void *v_tail, int hadamard_k, int32_t *dev_status,
+                    void *stream) {
+    if (!k_new || !v_new || !seqlens || !block_table || !k_codes || !k_scales || !v_codes || !v_scales || !v_tail)
+        return set_error(QK4V8_ERR_INVALID_ARG, "null pointer");
+    if (d != 128) return set_error(QK4V8_ERR_INVALID_ARG, "head_dim must be 128 (got %d)", d);
+    if (B <= 0 || n_new <= 0 || Hkv <= 0 || max_pages <= 0 || num_pages <= 0 ||
+        static_cast<int64_t>(num_pages) * Hkv >= (int64_t{1} << 31) || max_pages >= (1 << 24))
+        return set_error(QK4V8_ERR_INVALID_ARG, "bad sizes B=%d n_new=%d Hkv=%d max_pages=%d num_pages=%d", B, n_new,
+                         Hkv, max_pages, num_pages);
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(v_tail))
+        return set_error(QK4V8_ERR_INVALID_ARG, "K/V inputs, code pools and v_tail must be 16-byte aligned");
+    if (stride_b % 8 || stride_t % 8 || stride_h % 8 || stride_b < 0 || stride_t < 0 || stride_h < 0)
+        return set_error(QK4V8_ERR_INVALID_ARG, "strides must be non-negative multiples of 8 elements");
+    int st;
+    if ((st = check_device())) return st;
+    cudaError_t e = qk4v8::launch_kv_append(k_new, v_new, B, n_new, Hkv, stride_b, stride_t, stride_h, seqlens,
+                                            block_table, max_pages, num_pages, k_codes, k_scales, v_codes, v_scales,
+                                            v_tail, hadamard_k != 0, seqlens_out, dev_status,
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "kv append launch");
 }
 
 // Test hook (declared in include/qk4v8_test.h): while enabled, attention

@@ -230,7 +230,9 @@ __device__ __noinline__ void rescale_o_cols(uint32_t taddr, int nt, int nc, int 
 
 }  // namespace
 
-template <int NT, int RW, int NC, int ST, int MINB>
+// kExt: the instance for draft-block windows and paged caches; the other is
+// the plain decode over a contiguous cache.
+template <int NT, int RW, int NC, int ST, int MINB, bool kExt>
 __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
     qk4v8_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                         const AttnParams p) {
@@ -252,7 +254,7 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
     const int n_tiles = (L + 127) / 128;
     // Keys below lo are outside the window: the splits start at its first tile
     // (tile indices below are absolute).
-    const int lo = kv_window_lo(p, L);
+    const int lo = kExt ? kv_window_lo(p, L) : 0;
     const int tile_begin = lo / 128 + split * p.split_tiles;
     const int tile_end = imin(tile_begin + p.split_tiles, n_tiles);
     const int T = tile_end - tile_begin;
@@ -340,8 +342,8 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
         }
-        const int kvh = b * p.Hkv + h_kv;
-        const int nblk = p.kv_cap / 128;
+        const int nblk = kv_row_blocks<kExt>(p);
+        PageLookup pl;
         int issued = 0;
         for (int it = 0; it < T; ++it) {
             const int tile = tile_begin + it;
@@ -349,11 +351,13 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
             const uint32_t ph = (it / kStagesD) & 1;
             bool ok = wait_bar(&kv_empty[st], ph ^ 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, ok)) break;
+            int row, blk;
+            kv_tile_row<kExt>(p, b, h_kv, tile, pl, row, blk);
             if (lane == 0) {
                 mbar_arrive_expect_tx(&kv_full[st], Lay::kKBytes + Lay::kVBytes + 1024);
-                tma_load_3d(smem + Lay::kK + st * Lay::kKBytes, &tmap_k, 0, tile * 128, kvh, &kv_full[st]);
-                tma_load_3d(smem + Lay::kV + st * Lay::kVBytes, &tmap_v, tile * 128, 0, kvh, &kv_full[st]);
-                const int64_t atom = (static_cast<int64_t>(kvh) * nblk + tile) * 512;
+                tma_load_3d(smem + Lay::kK + st * Lay::kKBytes, &tmap_k, 0, blk * 128, row, &kv_full[st]);
+                tma_load_3d(smem + Lay::kV + st * Lay::kVBytes, &tmap_v, blk * 128, 0, row, &kv_full[st]);
+                const int64_t atom = (static_cast<int64_t>(row) * nblk + blk) * 512;
                 bulk_load(smem + Lay::kSfK + st * 512, p.k_scales + atom, 512, &kv_full[st]);
                 bulk_load(smem + Lay::kSfV + st * 512, p.v_scales + atom, 512, &kv_full[st]);
             }
@@ -622,7 +626,7 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
             }
             if (!(it > 0 && ok && tok < L - (p.causal ? nq - 1 : 0))) {
                 // (Keys below the window's lo lie in the first tile of the first split.)
-                const bool any_key = ok && tok < L && tok >= lo;
+                const bool any_key = ok && tok < L && (!kExt || tok >= lo);
 #pragma unroll
                 for (int i = 0; i < NC; ++i)
                     if (!(any_key && tok < lim_s[c0 + i])) u[i] = -INFINITY;
@@ -822,12 +826,18 @@ static cudaError_t launch_nt(const CUtensorMap &tk, const CUtensorMap &tv, const
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= kMaxDevices || !configured[dev]) {
-        e = cudaFuncSetAttribute(qk4v8_decode_kernel<NT, RW, NC, ST, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Lay::kBytes);
+        e = cudaFuncSetAttribute(qk4v8_decode_kernel<NT, RW, NC, ST, MINB, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kBytes);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(qk4v8_decode_kernel<NT, RW, NC, ST, MINB, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kBytes);
         if (e != cudaSuccess) return e;
         if (dev < kMaxDevices) configured[dev] = true;
     }
-    qk4v8_decode_kernel<NT, RW, NC, ST, MINB><<<grid, Lay::kThreads, Lay::kBytes, stream>>>(tk, tv, p);
+    if (p.window > 0 || p.block_table)
+        qk4v8_decode_kernel<NT, RW, NC, ST, MINB, true><<<grid, Lay::kThreads, Lay::kBytes, stream>>>(tk, tv, p);
+    else
+        qk4v8_decode_kernel<NT, RW, NC, ST, MINB, false><<<grid, Lay::kThreads, Lay::kBytes, stream>>>(tk, tv, p);
     return cudaGetLastError();
 }
 

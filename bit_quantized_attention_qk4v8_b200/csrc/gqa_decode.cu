@@ -121,10 +121,11 @@ __device__ __forceinline__ uint32_t gd_sf_id(uint32_t idesc, uint32_t id) { retu
 
 }  // namespace
 
-// kWindow: the instance for draft-block attention, whose query rows see only
-// keys from the window's first key (kv_window_lo) on; the other instance is
-// the plain decode, with no per-key lower bound in its softmax loop.
-template <bool kWindow>
+// kExt: the instance for draft-block attention (query rows see only keys from
+// the window's first key, kv_window_lo, on) and paged caches (key tiles looked
+// up in the block table); the other instance is the plain decode over a
+// contiguous cache, with neither in its loops.
+template <bool kExt>
 __global__ void __launch_bounds__(kGdThreads, 1)
     qk4v8_gqa_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                             const AttnParams p) {
@@ -225,7 +226,8 @@ __global__ void __launch_bounds__(kGdThreads, 1)
     if (warp == kGdProducerWarp) {
         // ------------------------------------------------------------- K producer
         if (lane == 0) prefetch_tensormap(&tmap_k);
-        const int nblk = p.kv_cap / 128;
+        const int nblk = kv_row_blocks<kExt>(p);
+        PageLookup pl;
         int g = 0;  // tiles so far
         int gk_issued = 0;
         bool ok = true;
@@ -235,7 +237,6 @@ __global__ void __launch_bounds__(kGdThreads, 1)
         while (ok && gd_next(p, gs, it, u)) {
             const int T = u.T;
             if (T <= 0) continue;
-            const int kvh = u.b * p.Hkv + u.h_kv;
             // K tiles of the unit: the K ring frees as soon as the pair's QK^T
             // completes, so K runs up to kGdKStages tiles ahead of the tensor core.
             for (int it = 0; it < T && ok; ++it) {
@@ -243,11 +244,12 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                 const int st = gk % kGdKStages;
                 ok = __all_sync(0xffffffffu, wait_bar(&k_empty[st], ((gk / kGdKStages) & 1) ^ 1, abort_flag, p.status));
                 if (!ok) break;
+                int row, blk;
+                kv_tile_row<kExt>(p, u.b, u.h_kv, u.tile_begin + it, pl, row, blk);
                 if (lane == 0) {
-                    const int tile = u.tile_begin + it;
                     mbar_arrive_expect_tx(&k_full[st], S::kKBytes + 512);
-                    tma_load_3d(smem + S::kK + st * S::kKBytes, &tmap_k, 0, tile * 128, kvh, &k_full[st]);
-                    bulk_load(smem + S::kSfK + st * 512, p.k_scales + (static_cast<int64_t>(kvh) * nblk + tile) * 512,
+                    tma_load_3d(smem + S::kK + st * S::kKBytes, &tmap_k, 0, blk * 128, row, &k_full[st]);
+                    bulk_load(smem + S::kSfK + st * 512, p.k_scales + (static_cast<int64_t>(row) * nblk + blk) * 512,
                               512, &k_full[st]);
                 }
                 gk_issued = gk + 1;
@@ -332,7 +334,8 @@ __global__ void __launch_bounds__(kGdThreads, 1)
         // V tiles on their own warp, so that a V stage waiting for its P V never
         // holds back the K loads of later pairs.
         if (lane == 0) prefetch_tensormap(&tmap_v);
-        const int nblk = p.kv_cap / 128;
+        const int nblk = kv_row_blocks<kExt>(p);
+        PageLookup pl;
         int g = 0, gv_issued = 0;
         bool ok = true;
         GdIter it;
@@ -341,7 +344,6 @@ __global__ void __launch_bounds__(kGdThreads, 1)
         while (ok && gd_next(p, gs, it, u)) {
             const int T = u.T;
             if (T <= 0) continue;
-            const int kvh = u.b * p.Hkv + u.h_kv;
             const bool last_partial = (u.L & 127) != 0 && u.tile_begin + T == (u.L + 127) / 128;
             for (int jt = 0; jt < T && ok; ++jt) {
                 const int gv = g + jt;
@@ -350,10 +352,12 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                 ok = __all_sync(0xffffffffu, wait_bar(&v_empty[sv], ph ^ 1, abort_flag, p.status));
                 if (!ok) break;
                 const int tile = u.tile_begin + jt;
+                int row, blk;
+                kv_tile_row<kExt>(p, u.b, u.h_kv, tile, pl, row, blk);
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&v_full[sv], S::kVTmaBytes + 512);
-                    tma_load_3d(smem + S::kV + sv * S::kVBytes, &tmap_v, tile * 128, 0, kvh, &v_full[sv]);
-                    bulk_load(smem + S::kSfV + sv * 512, p.v_scales + (static_cast<int64_t>(kvh) * nblk + tile) * 512,
+                    tma_load_3d(smem + S::kV + sv * S::kVBytes, &tmap_v, blk * 128, 0, row, &v_full[sv]);
+                    bulk_load(smem + S::kSfV + sv * 512, p.v_scales + (static_cast<int64_t>(row) * nblk + blk) * 512,
                               512, &v_full[sv]);
                 }
                 gv_issued = gv + 1;
@@ -636,8 +640,8 @@ __global__ void __launch_bounds__(kGdThreads, 1)
             int e = 0;         // m_w - m_O
             // m_O comes from the first half (64 keys) of the unit's first tile that
             // holds a visible key: the second half when a window starts there.
-            const int u_lo = kWindow ? kv_window_lo(p, u.L) : 0;  // the unit's first visible key
-            const int mo_half = kWindow && u_lo - u.tile_begin * 128 >= 64 ? 1 : 0;
+            const int u_lo = kExt ? kv_window_lo(p, u.L) : 0;  // the unit's first visible key
+            const int mo_half = kExt && u_lo - u.tile_begin * 128 >= 64 ? 1 : 0;
             auto receive_mo = [&]() -> bool {
                 if (!__all_sync(0xffffffffu, wait_bar(&mo_bar[grp], c & 1, abort_flag, p.status))) return false;
                 const float m0 = __uint_as_float(lds32(a_m));
@@ -660,7 +664,7 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const int jv = ti < T ? imax(0, imin(limit - (u.tile_begin + ti) * 128, 128)) : 0;  // keys j < jv
-                const int jlo = kWindow ? u_lo - (u.tile_begin + ti) * 128 : 0;  // and keys j >= jlo (window)
+                const int jlo = kExt ? u_lo - (u.tile_begin + ti) * 128 : 0;  // and keys j >= jlo (window)
                 int eb[4];  // e + x of each block when it was encoded
                 // The tile in two halves of 64 keys, to bound the registers held at once.
                 // S is released to the tensor core once the second half has been read.
@@ -680,7 +684,7 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                     }
                     // Keys at or past the row's bound, and before the window, are -inf
                     // (raw scores; the scale is positive).
-                    if (kWindow) {
+                    if (kExt) {
                         if (jv < 64 * hh + 64 || jlo > 64 * hh) {
 #pragma unroll
                             for (int j = 0; j < 64; ++j)
@@ -696,7 +700,7 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                     const float hm = fmaxf(bmx0, bmx1);
                     const bool mo_post = k == 0 && half == 0 && hh == mo_half;
                     const bool mo_take = k == 0 && half == 1 && hh == 0;
-                    if (kWindow ? (mo_post || mo_take) : (k == 0 && hh == 0)) {
+                    if (kExt ? (mo_post || mo_take) : (k == 0 && hh == 0)) {
                         // The first half of the unit's first tile with a visible key fixes
                         // m_O: the row's largest score there. It holds the unit's first
                         // visible key, so a row with no key in it has none in the unit. Its
@@ -979,7 +983,7 @@ cudaError_t launch_gqa_decode(const CUtensorMap &tk, const CUtensorMap &tv, cons
     }
     // Persistent: one CTA per SM (shared memory and the 512 TMEM columns allow no
     // more); the kernel schedules the work over the grid itself.
-    if (p.window > 0)
+    if (p.window > 0 || p.block_table)
         qk4v8_gqa_decode_kernel<true><<<sms, kGdThreads, GdSmem::kBytes, stream>>>(tk, tv, p);
     else
         qk4v8_gqa_decode_kernel<false><<<sms, kGdThreads, GdSmem::kBytes, stream>>>(tk, tv, p);

@@ -20,6 +20,49 @@ __device__ __forceinline__ int kv_window_lo(const AttnParams &p, int L) {
     return p.window > 0 ? imax(0, L - p.Sq - p.window) : 0;
 }
 
+// A warp's copy of 32 consecutive block-table entries of one sequence.
+struct PageLookup {
+    int b = -1, base = 0, entry = 0;
+};
+
+// Where key tile `tile` of (b, h_kv) lives: `row` of the [rows][tokens] K/V
+// tensor maps and scale arrays, and the 128-token block `blk` in that row.
+// Contiguous cache: row b * Hkv + h_kv, block `tile`. Paged cache: page
+// block_table[b][tile], row page * Hkv + h_kv, block 0; the warp loads the
+// entries 32 tiles at a time. An entry outside [0, num_pages) reads page 0
+// instead and records QK4V8_ERR_INVALID_ARG (1) in *status. All 32 lanes of
+// the warp call it with the same arguments. kPaging = false compiles the
+// contiguous case alone (kernel instances that never see a block table).
+template <bool kPaging>
+__device__ __forceinline__ void kv_tile_row(const AttnParams &p, int b, int h_kv, int tile, PageLookup &pl, int &row,
+                                            int &blk) {
+    if (!kPaging || !p.block_table) {
+        row = b * p.Hkv + h_kv;
+        blk = tile;
+        return;
+    }
+    const int base = tile & ~31;
+    if (pl.b != b || pl.base != base) {
+        const int t = base + static_cast<int>(threadIdx.x & 31);
+        pl.entry = t < p.max_pages ? p.block_table[static_cast<int64_t>(b) * p.max_pages + t] : 0;
+        pl.b = b;
+        pl.base = base;
+    }
+    int page = __shfl_sync(0xffffffffu, pl.entry, tile & 31);
+    if (page < 0 || page >= p.num_pages) {
+        if ((threadIdx.x & 31) == 0 && p.status) atomicCAS(p.status, 0, 1);
+        page = 0;
+    }
+    row = page * p.Hkv + h_kv;
+    blk = 0;
+}
+
+// 128-token blocks per row of the K/V scale arrays.
+template <bool kPaging>
+__device__ __forceinline__ int kv_row_blocks(const AttnParams &p) {
+    return kPaging && p.block_table ? 1 : p.kv_cap / 128;
+}
+
 __device__ __forceinline__ bool aborted(volatile uint32_t *flag, const int32_t *status) {
     if (*flag) return true;
     if (status && *reinterpret_cast<const volatile int32_t *>(status) != 0) {

@@ -33,6 +33,11 @@ struct AttnParams {
     // j >= L - Sq - window (the last `window` keys before the Sq-token block, and
     // the block); 0: no lower bound.
     int window;
+    // Decode only: paged K/V when non-null. Key tile t of sequence b is page
+    // block_table[b * max_pages + t] of pools [num_pages][Hkv][128 tokens]
+    // (kv_cap is then max_pages * 128); null: contiguous [B][Hkv][kv_cap].
+    const int32_t *block_table;
+    int max_pages, num_pages;
     float scale_log2;         // softmax_scale * log2(e)
     int decode;               // 0: units (b, h_q, q tile); 1: units (b, h_kv, split)
     int n_qtiles;
@@ -81,6 +86,14 @@ cudaError_t launch_gqa_decode(const CUtensorMap &tmap_k, const CUtensorMap &tmap
 // Merge of the sequences a persistent decode kernel cut (direct output, splits >= 2,
 // <= 64 rows per KV head), from the partials and the recorded piece counts.
 cudaError_t launch_cut_merge(const AttnParams &p, cudaStream_t stream);
+// Paged KV append (K and V of n_new tokens per sequence at positions
+// seqlens[b] ..; V groups re-encoded from the staging buffer `tail`), then
+// seqlens_out[b] = seqlens[b] + n_new (seqlens_out may be seqlens).
+cudaError_t launch_kv_append(const void *k, const void *v, int B, int n_new, int H, int64_t sb, int64_t st,
+                             int64_t sh, const int32_t *seqlens, const int32_t *block_table, int max_pages,
+                             int num_pages, uint8_t *k_codes, uint8_t *k_scales, uint8_t *v_codes,
+                             uint8_t *v_scales, void *tail, bool rotate_k, int32_t *seqlens_out, int32_t *status,
+                             cudaStream_t stream);
 cudaError_t launch_decode_merge(const float *ws_o, const float *ws_lse, int B, int Hq, int nq, int splits,
                                 __nv_bfloat16 *out, float *lse, cudaStream_t stream);
 

@@ -289,6 +289,69 @@ QK4V8_API int qk4v8_attention_decode_bf16_window(const void *q, int B, int Hq, i
 QK4V8_API int qk4v8_decode_default_splits_window(int B, int Hq, int Hkv, int nq, int max_seqlen, int window);
 
 /*
+ * Paged KV cache (MpFA article, section 6.1: the QK4V8 attention combined with
+ * a quantized KV cache; section 3.2: block scales computed online as the data
+ * arrives). The packed cache lives in pools of pages of 128 tokens; page p of
+ * KV head h holds
+ *   K codes  [num_pages][Hkv][128][64],  K scales [num_pages][Hkv][512]
+ *   V codes  [num_pages][Hkv][128][128], V scales [num_pages][Hkv][512]
+ * i.e. the packed layouts above with B = num_pages and cap = 128 (the size
+ * helpers give the pool sizes: qk4v8_mxfp4_codes_bytes(num_pages, Hkv, 128)
+ * and so on). block_table int32 [B][max_pages] (device) maps the n-th 128-token
+ * block of sequence b to its page; sequences hold at most max_pages * 128
+ * tokens. A block-table entry outside [0, num_pages) is not followed: the
+ * kernels read page 0 instead (attention) or skip the token (append) and write
+ * QK4V8_ERR_INVALID_ARG to *dev_status.
+ *
+ * qk4v8_kv_append: appends n_new tokens to every sequence. k_new and v_new are
+ * bf16 [B][n_new][Hkv][128] with the given element strides (shared by both;
+ * multiples of 8). Token t goes to position seqlens[b] + t (seqlens: device
+ * int32 [B], the lengths before the call); seqlens_out (device, nullable, may
+ * be seqlens) receives seqlens[b] + n_new once every kernel of the call has
+ * read seqlens. K rows are quantized on their own (with hadamard_k, after the
+ * rotation of qk4v8_quantize_qk_hadamard). V's 32-token groups change as
+ * tokens arrive: every group the new tokens touch gets its E8M0 scale
+ * recomputed from all of its tokens and all its codes rewritten, which needs
+ * the bf16 values of the open (last, partly filled) group of each sequence and
+ * head: v_tail, bf16 [B][Hkv][32][128] (qk4v8_kv_tail_bytes), owned by the
+ * caller, read and refreshed by every append. So the bytes after any sequence
+ * of appends equal those of qk4v8_quantize_qk / qk4v8_quantize_v over the whole
+ * sequence. Build a sequence's cache by appending its prompt to an empty
+ * sequence (seqlens 0, v_tail contents then unused). Codes of tokens past the
+ * new length within the last V group are written as 0; other padding is left
+ * as it was (the attention kernels ignore it). Four launches on `stream`.
+ *
+ * qk4v8_attention_decode_paged / qk4v8_attention_decode_bf16_paged: the
+ * decode calls (with the draft-block window) over such a pool, for up to 64
+ * query rows per KV head; other arguments as for the non-paged calls.
+ */
+QK4V8_API size_t qk4v8_kv_tail_bytes(int B, int Hkv);
+
+QK4V8_API int qk4v8_kv_append(const void *k_new, const void *v_new, int B, int n_new, int Hkv, int d,
+                              int64_t stride_b, int64_t stride_t, int64_t stride_h, const int32_t *seqlens,
+                              int32_t *seqlens_out, const int32_t *block_table, int max_pages, int num_pages,
+                              uint8_t *k_codes, uint8_t *k_scales, uint8_t *v_codes, uint8_t *v_scales,
+                              void *v_tail, int hadamard_k, int32_t *dev_status, void *stream);
+
+QK4V8_API int qk4v8_attention_decode_paged(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq,
+                                           int q_cap, const uint8_t *k_codes, const uint8_t *k_scales,
+                                           const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int num_pages,
+                                           const int32_t *block_table, int max_pages, const int32_t *seqlens_k,
+                                           int max_seqlen, int causal_in_block, int window, float softmax_scale,
+                                           int num_splits, void *workspace, size_t workspace_bytes, void *out,
+                                           float *lse, int32_t *dev_status, void *stream);
+
+QK4V8_API int qk4v8_attention_decode_bf16_paged(const void *q, int B, int Hq, int nq, int64_t q_stride_b,
+                                                int64_t q_stride_t, int64_t q_stride_h, const uint8_t *k_codes,
+                                                const uint8_t *k_scales, const uint8_t *v_codes,
+                                                const uint8_t *v_scales, int Hkv, int num_pages,
+                                                const int32_t *block_table, int max_pages, const int32_t *seqlens_k,
+                                                int max_seqlen, int causal_in_block, int window,
+                                                float softmax_scale, int num_splits, void *workspace,
+                                                size_t workspace_bytes, void *out, float *lse, int32_t *dev_status,
+                                                void *stream);
+
+/*
  * Decode step from bf16 queries (MpFA QK4V8 article, section 3.2: the query's
  * MXFP4 scales are computed as it is loaded, inside the attention call).
  * Same result, bit for bit, as qk4v8_quantize_qk (capacity 128) followed by

@@ -30,3 +30,21 @@ def unpack_e2m1(packed: np.ndarray) -> np.ndarray:
     out[..., 0::2] = packed & 0xF
     out[..., 1::2] = packed >> 4
     return out
+
+
+def gather_pages(codes, scales, block_table, n_blocks):
+    """Paged pools -> contiguous packed tensors of n_blocks 128-token blocks.
+
+    codes [P, H, R, X] and scales [P, H, 512] (numpy), block_table [B, max_pages].
+    K pools (R = 128 tokens, X = 64 bytes) give codes [B, H, n_blocks * 128, 64];
+    V pools (R = 128 channels, X = 128 tokens) give codes [B, H, 128, n_blocks * 128].
+    Scales come back as [B, H, n_blocks, 512] atoms. Plain indexing."""
+    idx = np.asarray(block_table)[:, :n_blocks]
+    c = codes[idx]                                   # [B, n, H, R, X]
+    s = scales[idx]                                  # [B, n, H, 512]
+    B, n, H, R, X = c.shape
+    if X == 64:      # K: token rows
+        c = np.transpose(c, (0, 2, 1, 3, 4)).reshape(B, H, n * R, X)
+    else:            # V: channel rows, tokens contiguous
+        c = np.transpose(c, (0, 2, 3, 1, 4)).reshape(B, H, R, n * X)
+    return c, np.transpose(s, (0, 2, 1, 3))
