@@ -65,7 +65,7 @@ def _load():
                                          ctypes.c_double, vp, i64, vp, vp]
         lib.oracle_attention.restype = i32
         lib.oracle_attention_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
-                                                ctypes.c_double, vp, i64, vp, vp]
+                                                i32, ctypes.c_double, vp, i64, vp, vp]
         lib.oracle_attention_window.restype = i32
         lib.oracle_hadamard_rows.argtypes = [vp, i64, vp]
         lib.oracle_hadamard_rows.restype = i32
@@ -142,8 +142,9 @@ def quantize_qk(x_bits: np.ndarray):
     return quantize_rows(xt, E2M1)
 
 
-def quantize_v(v_bits: np.ndarray, seqlens=None):
-    """MXFP8-E4M3 quantization of V given as bf16 bits [B, T, Hkv, d].
+def quantize_v(v_bits: np.ndarray, seqlens=None, fmt: int = E4M3):
+    """MXFP8-E4M3 quantization of V given as bf16 bits [B, T, Hkv, d] (fmt=E2M1:
+    MXFP4, the QK4V4 comparison point).
 
     Groups of 32 run along T. Returns codes [B, Hkv, d, T] and scales
     [B, Hkv, d, ceil(T/32)]; tokens at or past seqlens[b] are padding.
@@ -153,10 +154,10 @@ def quantize_v(v_bits: np.ndarray, seqlens=None):
     valid = None
     if seqlens is not None:
         valid = np.broadcast_to(np.asarray(seqlens, dtype=np.int32)[:, None, None], (B, H, d))
-    return quantize_rows(vt, E4M3, valid)
+    return quantize_rows(vt, fmt, valid)
 
 
-def attention(qc, qs, kc, ks, vc, vs, seqlens=None, causal=True, scale=None, sel=None, window=0):
+def attention(qc, qs, kc, ks, vc, vs, seqlens=None, causal=True, scale=None, sel=None, window=0, v_fmt=E4M3):
     """fp64 attention over the dequantized MX tensors.
 
     qc/qs [B,Hq,Sq,d]/[B,Hq,Sq,d/32]; kc/ks [B,Hkv,Lk,d]/[B,Hkv,Lk,d/32];
@@ -164,6 +165,7 @@ def attention(qc, qs, kc, ks, vc, vs, seqlens=None, causal=True, scale=None, sel
     sel: int32 [n,3] rows (b, h_q, i) or None for all rows.
     window > 0: each row sees only the last `window` keys before the query
     block and the block itself (the C function's visible_keys rule).
+    v_fmt: element format of V's codes (E4M3, or E2M1 for QK4V4).
     Returns (out, lse): out [B,Sq,Hq,d] and lse [B,Sq,Hq] when sel is None,
     else out [n,d] and lse [n].
     """
@@ -178,7 +180,8 @@ def attention(qc, qs, kc, ks, vc, vs, seqlens=None, causal=True, scale=None, sel
     out = np.empty((n, d), dtype=np.float64)
     lse = np.empty((n,), dtype=np.float64)
     rc = lib.oracle_attention_window(*[a.ctypes.data for a in arrs], sl.ctypes.data if sl is not None else None,
-                                     B, Hq, Hkv, Sq, Lk, d, int(bool(causal)), int(window), float(scale), selp, n,
+                                     B, Hq, Hkv, Sq, Lk, d, int(bool(causal)), int(window), int(v_fmt),
+                                     float(scale), selp, n,
                                      out.ctypes.data, lse.ctypes.data)
     if rc != 0:
         raise RuntimeError(f"oracle_attention_window failed ({rc})")
@@ -279,9 +282,9 @@ def quantize_qk_hadamard(x_bits: np.ndarray, seqlens=None):
     return quantize_rows_f32(y, E2M1, valid)
 
 
-def quantize_workload(gen: dict):
+def quantize_workload(gen: dict, v_fmt: int = E4M3):
     """Oracle quantization of a generated workload dict (q, k, v, seqlens)."""
     qc, qs = quantize_qk(gen["q"])
     kc, ks = quantize_qk(gen["k"])
-    vc, vs = quantize_v(gen["v"], gen["seqlens"])
+    vc, vs = quantize_v(gen["v"], gen["seqlens"], v_fmt)
     return dict(qc=qc, qs=qs, kc=kc, ks=ks, vc=vc, vs=vs)

@@ -214,7 +214,10 @@ static void visible_keys(int L, int Sq, int i, int causal, int window, int *lo, 
  *
  * qc, qs  [B][Hq][Sq][d] codes, [B][Hq][Sq][d/32] scales   (E2M1)
  * kc, ks  [B][Hkv][Lk][d] codes, [B][Hkv][Lk][d/32] scales (E2M1)
- * vc, vs  [B][Hkv][d][Lk] codes, [B][Hkv][d][ceil(Lk/32)] scales (E4M3)
+ * vc, vs  [B][Hkv][d][Lk] codes, [B][Hkv][d][ceil(Lk/32)] scales, element
+ *         format v_fmt: E4M3 (QK4V8), or E2M1 for the QK4V4 comparison point
+ *         of the MpFA article (section 2.2: V at 4 bits costs about 0.8
+ *         perplexity; section 5.3: a pitfall on long texts)
  * seqlens [B] KV length per sequence (NULL: Lk)
  * causal, window  the visible keys of each row (visible_keys above)
  * sel     [n_sel][3] rows (b, h_q, i) to compute; NULL computes every row in
@@ -223,8 +226,8 @@ static void visible_keys(int L, int Sq, int i, int causal, int window, int *lo, 
  */
 int oracle_attention_window(const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, const uint8_t *ks,
                             const uint8_t *vc, const uint8_t *vs, const int32_t *seqlens,
-                            int B, int Hq, int Hkv, int Sq, int Lk, int d, int causal, int window, double scale,
-                            const int32_t *sel, int64_t n_sel, double *out, double *lse) {
+                            int B, int Hq, int Hkv, int Sq, int Lk, int d, int causal, int window, int v_fmt,
+                            double scale, const int32_t *sel, int64_t n_sel, double *out, double *lse) {
     if (d % 32 || Hkv <= 0 || Hq % Hkv) return -1;
     const int G = Hq / Hkv;
     const int dg = d / 32;
@@ -280,7 +283,7 @@ int oracle_attention_window(const uint8_t *qc, const uint8_t *qs, const uint8_t 
         const uint8_t *vcu = vc + (int64_t)u * d * Lk, *vsu = vs + (int64_t)u * d * lg;
         for (int c = 0; c < d; ++c)
             for (int j = 0; j < L; ++j)
-                vd[(int64_t)j * d + c] = ldexp(oracle_decode(ORACLE_E4M3, vcu[(int64_t)c * Lk + j]),
+                vd[(int64_t)j * d + c] = ldexp(oracle_decode(v_fmt, vcu[(int64_t)c * Lk + j]),
                                                (int)vsu[(int64_t)c * lg + j / 32] - 127);
         for (int64_t oi = cnt[u]; oi < cnt[u + 1]; ++oi) {
             const int64_t r = order[oi];
@@ -329,8 +332,8 @@ int oracle_attention(const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, co
                      const uint8_t *vc, const uint8_t *vs, const int32_t *seqlens,
                      int B, int Hq, int Hkv, int Sq, int Lk, int d, int causal, double scale,
                      const int32_t *sel, int64_t n_sel, double *out, double *lse) {
-    return oracle_attention_window(qc, qs, kc, ks, vc, vs, seqlens, B, Hq, Hkv, Sq, Lk, d, causal, 0, scale, sel,
-                                   n_sel, out, lse);
+    return oracle_attention_window(qc, qs, kc, ks, vc, vs, seqlens, B, Hq, Hkv, Sq, Lk, d, causal, 0, ORACLE_E4M3,
+                                   scale, sel, n_sel, out, lse);
 }
 
 /*

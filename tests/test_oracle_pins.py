@@ -557,3 +557,62 @@ def test_rotation_spreads_an_outlier_channel():
     back = oracle.dequantize_rows(cr, sr, oracle.E2M1) @ H / math.sqrt(128)  # rotate back
     err_rot = np.abs(back - xb)
     assert err_rot[:, 0:32].mean() < 0.7 * err_plain[:, 0:32].mean()
+
+
+# ------------------------------------------------------- QK4V4 (V in MXFP4)
+
+@pytest.mark.parametrize("causal,lens", [(True, [70, 33]), (False, [64, 1])])
+def test_qk4v4_oracle_matches_naive_on_dequantized(causal, lens):
+    """V quantized to E2M1 along tokens (the QK4V4 comparison point): the oracle
+    must equal naive attention over the E2M1-dequantized values."""
+    rng = np.random.default_rng(40 + len(lens))
+    B, Sq, Hq, Hkv, Lk = 2, 3, 4, 2, 70
+    gen = dict(q=f32_to_bf16_bits(rng.standard_normal((B, Sq, Hq, 128)).astype(np.float32) * 2),
+               k=f32_to_bf16_bits(rng.standard_normal((B, Lk, Hkv, 128)).astype(np.float32) * 2),
+               v=f32_to_bf16_bits(rng.standard_normal((B, Lk, Hkv, 128)).astype(np.float32)),
+               seqlens=np.array(lens, dtype=np.int32))
+    qz = oracle.quantize_workload(gen, v_fmt=oracle.E2M1)
+    assert qz["vc"].max() <= 15
+    out, lse = oracle.attention(qz["qc"], qz["qs"], qz["kc"], qz["ks"], qz["vc"], qz["vs"], gen["seqlens"],
+                                causal=causal, v_fmt=oracle.E2M1)
+    qd = np.transpose(deq_e2m1(qz["qc"], qz["qs"]), (0, 2, 1, 3))
+    kd = np.transpose(deq_e2m1(qz["kc"], qz["ks"]), (0, 2, 1, 3))
+    vd = np.transpose(deq_e2m1(qz["vc"], qz["vs"]), (0, 3, 1, 2))
+    ref, rlse = naive_attention(qd, kd, vd, gen["seqlens"], causal, 1 / math.sqrt(128))
+    assert np.allclose(out, ref, rtol=0, atol=1e-12)
+    fin = np.isfinite(rlse)
+    assert np.allclose(lse[fin], rlse[fin], rtol=0, atol=1e-12)
+
+
+def test_qk4v4_grid_inputs_equal_reference():
+    rng = np.random.default_rng(41)
+    B, Sq, Hq, Hkv, Lk = 1, 4, 2, 1, 64
+    q = _grid_tensor(rng, (B, Sq, Hq, 128), oracle.E2M1)
+    k = _grid_tensor(rng, (B, Lk, Hkv, 128), oracle.E2M1)
+    v = np.transpose(_grid_tensor(rng, (B, Hkv, 128, Lk), oracle.E2M1), (0, 3, 1, 2))
+    gen = dict(q=f32_to_bf16_bits(q.astype(np.float32)), k=f32_to_bf16_bits(k.astype(np.float32)),
+               v=f32_to_bf16_bits(v.astype(np.float32)), seqlens=np.array([64], np.int32))
+    qz = oracle.quantize_workload(gen, v_fmt=oracle.E2M1)
+    out, _ = oracle.attention(qz["qc"], qz["qs"], qz["kc"], qz["ks"], qz["vc"], qz["vs"], gen["seqlens"],
+                              causal=True, scale=1 / 64.0, v_fmt=oracle.E2M1)
+    ref, _ = oracle.attention_ref(gen["q"], gen["k"], gen["v"], gen["seqlens"], causal=True, scale=1 / 64.0)
+    assert np.allclose(out, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+
+
+def test_qk4v4_error_exceeds_qk4v8_error():
+    """V at 4 bits loses more than V at 8 bits (the article's section 2.2): with
+    Q and K quantized the same way, the error that V's quantization adds to the
+    output (against the same attention over unquantized V) is several times
+    larger for E2M1 than for E4M3."""
+    wl = synth.Workload("t", "decode", B=2, Hq=8, Hkv=2, Sq=4, Lk=300, seed=5)
+    gen = wl.generate()
+    errs = {}
+    for fmt in (oracle.E4M3, oracle.E2M1):
+        qz = oracle.quantize_workload(gen, v_fmt=fmt)
+        o, _ = oracle.attention(qz["qc"], qz["qs"], qz["kc"], qz["ks"], qz["vc"], qz["vs"], gen["seqlens"],
+                                causal=True, v_fmt=fmt)
+        qd = np.transpose(deq_e2m1(qz["qc"], qz["qs"]), (0, 2, 1, 3))
+        kd = np.transpose(deq_e2m1(qz["kc"], qz["ks"]), (0, 2, 1, 3))
+        ref, _ = naive_attention(qd, kd, bf16_bits_to_f64(gen["v"]), gen["seqlens"], True, 1 / math.sqrt(128))
+        errs[fmt] = np.abs(o - ref).mean()
+    assert errs[oracle.E2M1] > 3 * errs[oracle.E4M3]
