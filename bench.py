@@ -32,7 +32,14 @@ The JSON line also carries one flat object per other workload or measurement:
     or a stated subset (the S=8192 prefill), extrapolated linearly;
   - error keys (err_*): the GPU output against the oracle, and, as context,
     against fp64 attention over the unquantized bf16 inputs; hadamard_* keys
-    give the same for Q and K quantized after their Hadamard rotation.
+    give the same for Q and K quantized after their Hadamard rotation, and
+    qk4v4_* keys for V in MXFP4;
+  - qk4v4: the decode workloads with V in MXFP4 (the article's QK4V4
+    comparison point): time, GB/s of the smaller cache, speedup;
+  - paged: the headline decode over 128-token pages in random order, and the
+    cost of appending a token to every sequence;
+  - draft_block: 8 non-causal rows with a 1024-key sliding window over the
+    verify workload's cache (the DFlash draft-block attention).
 `--impl reference` times the CPU oracle alone on the headline decode workload.
 """
 from __future__ import annotations
@@ -447,6 +454,142 @@ def run_decode_workload(name, steps, warmup, hbm_gbs, hadamard):
     return dict(res=res, gen=gen, out=out_np, rot=None if rot is None else rot[0], wl=wl)
 
 
+KV4_BYTES_PER_TOKEN_HEAD = 64 + 64 + 4 + 4   # QK4V4: E2M1 K and V codes, K and V E8M0 scales
+
+
+def run_decode_v4(name, gen, steps, hbm_gbs):
+    """QK4V4 (V in MXFP4) on a decode workload: the bf16-query decode step over an
+    MXFP4-K / MXFP4-V cache, timed like the QK4V8 step."""
+    import torch
+    import bit_quantized_attention_qk4v8_b200 as qk
+    import synth
+    wl = synth.WORKLOADS[name]
+    lens = gen["seqlens"].astype(np.int64)
+    sl = torch.from_numpy(gen["seqlens"]).cuda()
+    cap = qk.round_cap(wl.Lk)
+    kp = qk.quantize_qk(to_dev(gen["k"]), cap=cap, seqlens=sl)
+    vp = qk.quantize_v4(to_dev(gen["v"]), cap=cap, seqlens=sl)
+    q = to_dev(gen["q"])
+    max_len = int(lens.max())
+    splits = qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, max_len)
+    ws = torch.empty((max(16, qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)),),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=max_len, num_splits=splits, workspace=ws, out=out)
+
+    ms, _ = graph_time_ms(step, steps, 3, torch.cuda.current_stream())
+    kv_bytes = int(lens.sum()) * wl.Hkv * KV4_BYTES_PER_TOKEN_HEAD
+    gbs = kv_bytes / (ms * 1e-3) / 1e9
+    return dict(ms=ms, gbs=gbs, frac=gbs / hbm_gbs, kv_bytes=kv_bytes, out=out.float().cpu().numpy())
+
+
+def run_paged(gen, steps, hbm_gbs):
+    """The headline decode over a paged cache: the packed cache copied into 128-token
+    pages in a random page order, one qk4v8_attention_decode_bf16_paged call per
+    step; plus the cost of appending one token to every sequence."""
+    import torch
+    import bit_quantized_attention_qk4v8_b200 as qk
+    import synth
+    wl = synth.WORKLOADS[DECODE_WORKLOAD]
+    sl = torch.from_numpy(gen["seqlens"]).cuda()
+    max_pages = wl.Lk // 128 + 1
+    k, v, q = to_dev(gen["k"]), to_dev(gen["v"]), to_dev(gen["q"])
+    kp = qk.quantize_qk(k, cap=max_pages * 128, seqlens=sl)
+    vp = qk.quantize_v(v, cap=max_pages * 128, seqlens=sl)
+    num_pages = wl.B * max_pages
+    perm = np.random.default_rng(0).permutation(num_pages).astype(np.int32).reshape(wl.B, max_pages)
+    cache = qk.paged_kv(wl.B, wl.Hkv, num_pages, torch.from_numpy(perm))
+    idx = cache.block_table.long()
+    for i in range(max_pages):
+        pages = idx[:, i]
+        cache.k_codes[pages] = kp.codes[:, :, i * 128:(i + 1) * 128]
+        cache.k_scales[pages] = kp.scales[:, :, i]
+        cache.v_codes[pages] = vp.codes[:, :, :, i * 128:(i + 1) * 128]
+        cache.v_scales[pages] = vp.scales[:, :, i]
+    cache.seqlens.copy_(sl)
+    # The staging buffer holds the open V group (none: 8192 is a multiple of 32).
+    out = torch.empty((wl.B, 1, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
+    ref = qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=wl.Lk)
+
+    def step():
+        qk.attention_decode_bf16_paged(q, cache, max_seqlen=wl.Lk, out=out)
+
+    ms, _ = graph_time_ms(step, steps, 3, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    equal = bool(torch.equal(out, ref))
+    kv_bytes = wl.B * wl.Hkv * wl.Lk * KV_BYTES_PER_TOKEN_HEAD
+    # Append: one new token per sequence, 64 steps (the last page has room).
+    knew = k[:, :1].contiguous()
+    vnew = v[:, :1].contiguous()
+    n_app = 64
+    stream = torch.cuda.current_stream()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(n_app):
+        qk.kv_append(cache, knew, vnew)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    app_us = a0.elapsed_time(a1) / n_app * 1e3
+    gbs = kv_bytes / (ms * 1e-3) / 1e9
+    return {"workload": DECODE_WORKLOAD + " (paged, 128-token pages in random order)", "ms_per_step": ms,
+            "value": gbs, "unit": "GB/s", "roofline_frac": gbs / hbm_gbs, "steps": steps,
+            "kernel": "qk4v8_decode_kernel<16,4,4,3,2,true> (paged instance)",
+            "output_equals_contiguous": equal, "append_us_per_call": app_us,
+            "append_call": "qk4v8_kv_append of 1 token to 32 sequences x 8 KV heads (4 launches, not in a graph)"}
+
+
+def run_draft_block(gen, hbm_gbs, window=1024, reps=20):
+    """Draft-block attention on the verify workload's cache: the 8 block rows see
+    the last `window` keys before the block and the block, non-causal. Its
+    working set (the window's tiles, about 110 MB) fits in L2, so L2 is flushed
+    before every timed step and each step is timed alone."""
+    import torch
+    import bit_quantized_attention_qk4v8_b200 as qk
+    import synth
+    wl = synth.WORKLOADS[VERIFY_WORKLOAD]
+    sl = torch.from_numpy(gen["seqlens"]).cuda()
+    cap = qk.round_cap(wl.Lk)
+    kp = qk.quantize_qk(to_dev(gen["k"]), cap=cap, seqlens=sl)
+    vp = qk.quantize_v(to_dev(gen["v"]), cap=cap, seqlens=sl)
+    q = to_dev(gen["q"])
+    out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
+    splits = qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, wl.Lk, window)
+    ws = torch.empty((max(16, qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)),),
+                     dtype=torch.uint8, device="cuda")
+    flush = torch.empty((256 * 2 ** 20,), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=wl.Lk, causal_in_block=False, window=window,
+                                 num_splits=splits, workspace=ws, out=out)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    lens = gen["seqlens"].astype(np.int64)
+    lo = np.maximum(0, lens - wl.Sq - window)
+    vis_bytes = int((lens - lo).sum()) * wl.Hkv * KV_BYTES_PER_TOKEN_HEAD
+    gbs = vis_bytes / (ms * 1e-3) / 1e9
+    return dict(res={"workload": f"draft block on {VERIFY_WORKLOAD}: 8 non-causal rows, window {window}",
+                     "ms_per_step": ms, "value": gbs, "unit": "GB/s", "roofline_frac": gbs / hbm_gbs,
+                     "visible_kv_bytes": vis_bytes, "kv_splits": splits, "steps": reps,
+                     "l2": "flushed (256 MB write) before each timed step",
+                     "tokens_per_s": wl.B * wl.Sq / (ms * 1e-3)},
+                out=out.float().cpu().numpy(), window=window)
+
+
 # ---------------------------------------------------------------------------- prefill
 
 PREFILL_SUBSET_HEADS = list(range(0, 32, 4))   # (b = 0, one query head per KV head): the CPU subset
@@ -682,7 +825,7 @@ def _errs(got, ref, prefix):
     return {f"{prefix}_max_abs": float(d.max()), f"{prefix}_mean_abs": float(d.mean())}
 
 
-def cpu_decode_leg(gen, wl, out_gpu, rot_gpu):
+def cpu_decode_leg(gen, wl, out_gpu, rot_gpu, v4_gpu=None):
     """Oracle on the whole decode workload (cache pre-quantized untimed, as on the
     GPU; Q quantize + attention timed), the GPU output's error against it, and
     the context errors against unquantized attention on three batch entries."""
@@ -724,6 +867,40 @@ def cpu_decode_leg(gen, wl, out_gpu, rot_gpu):
             rorc.append(o[0])
         res.update(_errs(np.stack(rot), np.stack(rorc), "hadamard_err_vs_oracle"))
         res.update(_errs(np.stack(rot), bf, "hadamard_err_vs_bf16"))
+    if v4_gpu is not None:
+        vorc = []
+        for b in bs:
+            one = slice(b, b + 1)
+            sub = dict(q=gen["q"][one], k=gen["k"][one], v=gen["v"][one], seqlens=gen["seqlens"][one])
+            oz = oracle.quantize_workload(sub, v_fmt=oracle.E2M1)
+            o, _ = oracle.attention(oz["qc"], oz["qs"], oz["kc"], oz["ks"], oz["vc"], oz["vs"], sub["seqlens"],
+                                    causal=True, v_fmt=oracle.E2M1)
+            vorc.append(o[0])
+        got4 = np.stack([v4_gpu[b] for b in bs])
+        res.update(_errs(got4, np.stack(vorc), "qk4v4_err_vs_oracle"))
+        res.update(_errs(got4, bf, "qk4v4_err_vs_bf16"))
+    return res
+
+
+def cpu_draft_block_leg(gen, wl, out_gpu, window):
+    """Error of the draft-block (window) output against the windowed oracle and the
+    windowed unquantized reference, on three batch entries."""
+    import oracle
+    bs = sorted({0, wl.B // 2, wl.B - 1})
+    got, orc, bf = [], [], []
+    for b in bs:
+        one = slice(b, b + 1)
+        sub = dict(q=gen["q"][one], k=gen["k"][one], v=gen["v"][one], seqlens=gen["seqlens"][one])
+        oz = oracle.quantize_workload(sub)
+        o, _ = oracle.attention(oz["qc"], oz["qs"], oz["kc"], oz["ks"], oz["vc"], oz["vs"], sub["seqlens"],
+                                causal=False, window=window)
+        r, _ = oracle.attention_ref(sub["q"], sub["k"], sub["v"], sub["seqlens"], causal=False, window=window)
+        got.append(out_gpu[b])
+        orc.append(o[0])
+        bf.append(r[0])
+    res = _errs(np.stack(got), np.stack(orc), "err_vs_oracle")
+    res.update(_errs(np.stack(got), np.stack(bf), "err_vs_bf16"))
+    res["err_rows"] = f"batch entries {bs}, every head and block row"
     return res
 
 
@@ -938,11 +1115,30 @@ def main():
     }
 
     extra = {}
+    v4 = {}
+    draft = None
     if world == 1 and not args.no_extra_decode:
         for key, name in (("decode_long", LONG_WORKLOAD), ("verify", VERIFY_WORKLOAD)):
             extra[key] = run_decode_workload(name, args.extra_steps, min(args.warmup, 5), hbm_gbs,
                                              hadamard and key == "verify")
             line[key] = extra[key]["res"]
+        # QK4V4, the article's comparison point, on the three decode workloads.
+        for key, name, g in (("decode", DECODE_WORKLOAD, d["gen"]), ("decode_long", LONG_WORKLOAD,
+                                                                        extra["decode_long"]["gen"]),
+                             ("verify", VERIFY_WORKLOAD, extra["verify"]["gen"])):
+            v4[key] = run_decode_v4(name, g, args.extra_steps, hbm_gbs)
+        line["qk4v4"] = {"what": "V in MXFP4 (QK4V4) instead of MXFP8, same step, swap-AB kernel",
+                         "decode_ms": v4["decode"]["ms"], "decode_gbs": v4["decode"]["gbs"],
+                         "decode_speedup_vs_qk4v8": ms_per_step / v4["decode"]["ms"],
+                         "decode_long_ms": v4["decode_long"]["ms"], "decode_long_gbs": v4["decode_long"]["gbs"],
+                         "decode_long_speedup_vs_qk4v8": extra["decode_long"]["res"]["ms_per_step"] /
+                         v4["decode_long"]["ms"],
+                         "verify_ms": v4["verify"]["ms"], "verify_gbs": v4["verify"]["gbs"],
+                         "verify_speedup_vs_qk4v8": extra["verify"]["res"]["ms_per_step"] / v4["verify"]["ms"],
+                         "bytes_per_token_head": KV4_BYTES_PER_TOKEN_HEAD}
+        line["paged"] = run_paged(d["gen"], args.extra_steps, hbm_gbs)
+        draft = run_draft_block(extra["verify"]["gen"], hbm_gbs)
+        line["draft_block"] = draft["res"]
     pre = small = None
     if world == 1 and not args.no_prefill:
         peaks = run_mma_peaks()
@@ -956,17 +1152,23 @@ def main():
         line["quantize"] = run_quantize_kernels(hbm_gbs, pre["gen"])
 
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        head = cpu_decode_leg(d["gen"], wl, d["out"], None if d["rot"] is None else d["rot"][0])
+        head = cpu_decode_leg(d["gen"], wl, d["out"], None if d["rot"] is None else d["rot"][0],
+                              v4["decode"]["out"] if "decode" in v4 else None)
         line["cpu_baseline"] = {"value": head["cpu_value"], "unit": "GB/s", "cores": head["cpu_cores"],
                                 "kind": "oracle", "sample": head["cpu_sample"]}
         line["context_error"] = {k: v for k, v in head.items() if "err" in k}
         line["context_error"]["note"] = ("err_vs_oracle: GPU vs the fp64 QK4V8 oracle (bar: max 3e-2, mean 3e-3); "
                                          "err_vs_bf16: GPU vs fp64 attention over the unquantized bf16 inputs "
-                                         "(context, no bar); hadamard_*: Q and K quantized after rotation")
+                                         "(context, no bar); hadamard_*: Q and K quantized after rotation; "
+                                         "qk4v4_*: V in MXFP4 (against the QK4V4 oracle)")
         if d["rot"] is not None:
             line["context_error"]["hadamard_ms_per_step"] = d["rot"][1]
         for key, x in extra.items():
-            x["res"].update(cpu_decode_leg(x["gen"], x["wl"], x["out"], x["rot"]))
+            x["res"].update(cpu_decode_leg(x["gen"], x["wl"], x["out"], x["rot"],
+                                           v4[key]["out"] if key in v4 else None))
+        if draft is not None:
+            line["draft_block"].update(cpu_draft_block_leg(extra["verify"]["gen"], extra["verify"]["wl"],
+                                                           draft["out"], draft["window"]))
         if pre is not None:
             line["prefill"].update(cpu_prefill_leg(pre))
         if small is not None:

@@ -22,11 +22,11 @@ import torch
 from ._lib import QK4V8Error, check, lib
 
 __all__ = [
-    "MXFP4", "MXFP8V", "PagedKV", "QK4V8Error", "lib", "round_cap",
+    "MXFP4", "MXFP4V", "MXFP8V", "PagedKV", "QK4V8Error", "lib", "round_cap",
     "quantize_qk", "quantize_v", "quantize", "attention_prefill", "attention_decode",
     "decode_workspace_bytes", "decode_default_splits", "attention_decode_splitkv", "decode_merge",
     "attention_decode_bf16", "decode_bf16_workspace_bytes",
-    "paged_kv", "kv_append", "attention_decode_paged", "attention_decode_bf16_paged",
+    "paged_kv", "kv_append", "attention_decode_paged", "attention_decode_bf16_paged", "quantize_v4",
 ]
 
 D = 128
@@ -40,6 +40,18 @@ def round_cap(n: int) -> int:
 @dataclass
 class MXFP4:
     """Packed MXFP4 tensor (Q or K): codes uint8 [B][H][cap][64], scales uint8 [B][H][cap/128][512]."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    B: int
+    H: int
+    cap: int
+    length: int
+
+
+@dataclass
+class MXFP4V:
+    """Packed MXFP4 V (the QK4V4 comparison point): codes uint8 [B][H][128][cap/2]
+    (two tokens per byte), scales uint8 [B][H][cap/128][512]."""
     codes: torch.Tensor
     scales: torch.Tensor
     B: int
@@ -119,6 +131,21 @@ def quantize_v(v: torch.Tensor, cap: Optional[int] = None, seqlens=None, out: Op
     return out
 
 
+def quantize_v4(v: torch.Tensor, cap: Optional[int] = None, seqlens=None, out: Optional[MXFP4V] = None) -> MXFP4V:
+    """MXFP4-quantize V ([B, T, H, 128] bf16), groups of 32 along T (qk4v8_quantize_v4, QK4V4)."""
+    _check_bf16(v, "v")
+    B, T, H, _ = v.shape
+    cap = round_cap(T) if cap is None else int(cap)
+    sl = _seqlens(seqlens, B, v.device)
+    if out is None:
+        out = MXFP4V(torch.empty((B, H, D, cap // 2), dtype=torch.uint8, device=v.device),
+                     torch.empty((B, H, cap // 128, 512), dtype=torch.uint8, device=v.device), B, H, cap, T)
+    check(lib().qk4v8_quantize_v4(v.data_ptr(), B, T, H, D, v.stride(0), v.stride(1), v.stride(2), _ptr(sl), cap,
+                                  out.codes.data_ptr(), out.scales.data_ptr(), _stream(v.device)), "qk4v8_quantize_v4")
+    out.length = T
+    return out
+
+
 def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seqlens_k=None, q_cap=None, kv_cap=None,
              hadamard: bool = False):
     """Quantize contiguous Q [B,Sq,Hq,128], K and V [B,Sk,Hkv,128] in one library call.
@@ -183,7 +210,7 @@ def decode_default_splits(B: int, Hq: int, Hkv: int, nq: int, max_seqlen: int, w
     return int(lib().qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen))
 
 
-def attention_decode(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optional[int] = None,
+def attention_decode(q: MXFP4, k: MXFP4, v, seqlens_k, max_seqlen: Optional[int] = None,
                      causal_in_block: bool = True, softmax_scale: Optional[float] = None, num_splits: int = 0,
                      workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                      lse: Optional[torch.Tensor] = None, return_lse: bool = False,
@@ -210,7 +237,9 @@ def attention_decode(q: MXFP4, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optio
             int(bool(causal_in_block)))
     tail = (float(softmax_scale or 0.0), int(splits), workspace.data_ptr(),
             workspace.numel() * workspace.element_size(), out.data_ptr(), _ptr(lse), _ptr(dev_status), _stream(dev))
-    if window:
+    if isinstance(v, MXFP4V):
+        check(lib().qk4v8_attention_decode_v4(*head, int(window), *tail), "qk4v8_attention_decode_v4")
+    elif window:
         check(lib().qk4v8_attention_decode_window(*head, int(window), *tail), "qk4v8_attention_decode_window")
     else:
         check(lib().qk4v8_attention_decode(*head, *tail), "qk4v8_attention_decode")
@@ -221,7 +250,7 @@ def decode_bf16_workspace_bytes(B: int, Hq: int, Hkv: int, nq: int, num_splits: 
     return int(lib().qk4v8_decode_bf16_workspace_bytes(B, Hq, Hkv, nq, num_splits))
 
 
-def attention_decode_bf16(q: torch.Tensor, k: MXFP4, v: MXFP8V, seqlens_k, max_seqlen: Optional[int] = None,
+def attention_decode_bf16(q: torch.Tensor, k: MXFP4, v, seqlens_k, max_seqlen: Optional[int] = None,
                           causal_in_block: bool = True, softmax_scale: Optional[float] = None, num_splits: int = 0,
                           workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                           lse: Optional[torch.Tensor] = None, return_lse: bool = False,
@@ -248,7 +277,9 @@ def attention_decode_bf16(q: torch.Tensor, k: MXFP4, v: MXFP8V, seqlens_k, max_s
             int(bool(causal_in_block)))
     tail = (float(softmax_scale or 0.0), int(splits), _ptr(workspace), ws_bytes, out.data_ptr(), _ptr(lse),
             _ptr(dev_status), _stream(dev))
-    if window:
+    if isinstance(v, MXFP4V):
+        check(lib().qk4v8_attention_decode_bf16_v4(*head, int(window), *tail), "qk4v8_attention_decode_bf16_v4")
+    elif window:
         check(lib().qk4v8_attention_decode_bf16_window(*head, int(window), *tail), "qk4v8_attention_decode_bf16_window")
     else:
         check(lib().qk4v8_attention_decode_bf16(*head, *tail), "qk4v8_attention_decode_bf16")

@@ -89,6 +89,25 @@ int make_v_map(CUtensorMap *map, const uint8_t *codes, int BH, int cap) {
     return QK4V8_OK;
 }
 
+// MXFP4 V codes [B*Hkv][128][cap / 2] (the QK4V4 comparison point): loaded with
+// the 16U4_ALIGN16B element type, which lands each 16 packed codes (8 bytes)
+// in a 16-byte slot of shared memory, the layout the block-scaled f8f6f4 MMA
+// reads for an E2M1 operand. A 128-token x 128-channel box then fills the same
+// 128 x 128-byte, 128-byte-swizzled tile as an MXFP8 V box.
+int make_v4_map(CUtensorMap *map, const uint8_t *codes, int BH, int cap) {
+    auto enc = get_encode_fn();
+    if (!enc) return set_error(QK4V8_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cap), 128, static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(cap) / 2, static_cast<cuuint64_t>(cap) / 2 * 128};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<uint8_t *>(codes), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(QK4V8_ERR_CUDA, "cuTensorMapEncodeTiled(V, MXFP4) failed (%d)", int(r));
+    return QK4V8_OK;
+}
+
 int validate_quant_args(const void *x, int B, int S, int H, int d, int64_t sb, int64_t ss, int64_t sh, int cap,
                         const uint8_t *codes, const uint8_t *scales) {
     if (!x || !codes || !scales) return set_error(QK4V8_ERR_INVALID_ARG, "null pointer");
@@ -186,6 +205,21 @@ int qk4v8_quantize_v(const void *v, int B, int S, int H, int d, int64_t stride_b
     cudaError_t e = qk4v8::launch_quantize_v(v, B, S, H, stride_b, stride_s, stride_h, seqlens, cap, codes, scales,
                                              static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "quantize_v launch");
+}
+
+size_t qk4v8_mxfp4v_codes_bytes(int B, int H, int cap) {
+    return static_cast<size_t>(B) * H * 128 * (cap / 2);
+}
+
+int qk4v8_quantize_v4(const void *v, int B, int S, int H, int d, int64_t stride_b, int64_t stride_s,
+                      int64_t stride_h, const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
+                      void *stream) {
+    int st = validate_quant_args(v, B, S, H, d, stride_b, stride_s, stride_h, cap, codes, scales);
+    if (st) return st;
+    if ((st = check_device())) return st;
+    cudaError_t e = qk4v8::launch_quantize_v4(v, B, S, H, stride_b, stride_s, stride_h, seqlens, cap, codes, scales,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "quantize_v4 launch");
 }
 
 int qk4v8_quantize(const void *q, const void *k, const void *v, int B, int Sq, int Sk, int Hq, int Hkv, int d,
@@ -370,10 +404,13 @@ bool gqa_rows(int Hq, int Hkv, int nq) {
 // kernel. With `out` given and a single split on the swap-AB kernel, the kernel
 // writes out (and lse) itself and *direct is set; otherwise it writes the split
 // partials to the workspace and the caller runs the merge.
-// Paged K/V pools of a decode call (block_table null: contiguous caches).
+// How a decode call's cache is laid out: paged K/V pools (block_table null:
+// contiguous caches), and the V element format (v_fp4: MXFP4, the QK4V4
+// comparison point, contiguous caches only).
 struct KvPages {
     const int32_t *block_table = nullptr;
     int max_pages = 0, num_pages = 0;
+    bool v_fp4 = false;
 };
 
 int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k_codes, const uint8_t *k_scales,
@@ -400,9 +437,16 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
         max_seqlen > kv_cap)
         return set_error(QK4V8_ERR_INVALID_ARG, "bad lengths q_cap=%d kv_cap=%d max_seqlen=%d", q.cap, kv_cap,
                          max_seqlen);
-    if (q.bf16 && !swap_ab_rows(Hq, Hkv, nq))
+    // MXFP4 V runs on the swap-AB kernel, up to 64 query rows per KV head.
+    const bool use_swap = swap_ab_rows(Hq, Hkv, nq) || pages.v_fp4;
+    const bool use_gqa = !use_swap && gqa_rows(Hq, Hkv, nq);
+    if (q.bf16 && !use_swap)
         return set_error(QK4V8_ERR_INVALID_ARG, "bf16 Q in the split kernel needs (Hq/Hkv)*nq < %d",
                          qk4v8::kGqaMinRows);
+    if (pages.v_fp4 && ((Hq / Hkv) * nq > qk4v8::kDecodeMaxRows || pages.block_table ||
+                        (reinterpret_cast<uintptr_t>(v_codes) & 31)))
+        return set_error(QK4V8_ERR_INVALID_ARG, "MXFP4 V needs (Hq/Hkv)*nq <= %d, a contiguous cache and 32-byte "
+                                                "aligned V codes", qk4v8::kDecodeMaxRows);
     if (num_splits < 0) return set_error(QK4V8_ERR_INVALID_ARG, "num_splits must be >= 0");
     if (window < 0) return set_error(QK4V8_ERR_INVALID_ARG, "window must be >= 0 (0: none)");
     if (pages.block_table) {
@@ -423,7 +467,7 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
     const int splits = num_splits > 0 ? num_splits : qk4v8_decode_default_splits(B, Hq, Hkv, nq, span);
     // Direct output: the swap-AB kernel with one split, and the GQA decode kernel
     // always (with splits, its own merge launch finishes the cut sequences).
-    const bool direct_out = out && ((splits == 1 && swap_ab_rows(Hq, Hkv, nq)) || gqa_rows(Hq, Hkv, nq));
+    const bool direct_out = out && ((splits == 1 && use_swap) || use_gqa);
     if (out && !aligned16(out)) return set_error(QK4V8_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
     const size_t need = (direct_out && splits == 1) ? 0 : qk4v8_decode_workspace_bytes(B, Hq, nq, splits);
     if (need && (!workspace || !aligned16(workspace) || workspace_bytes < need))
@@ -433,7 +477,8 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
     // A paged pool is the contiguous layout with num_pages rows of capacity 128.
     const int map_rows = pages.block_table ? pages.num_pages * Hkv : B * Hkv;
     const int map_cap = pages.block_table ? 128 : kv_cap;
-    if ((st = make_k_map(&tk, k_codes, map_rows, map_cap)) || (st = make_v_map(&tv, v_codes, map_rows, map_cap)))
+    if ((st = make_k_map(&tk, k_codes, map_rows, map_cap)) ||
+        (st = pages.v_fp4 ? make_v4_map(&tv, v_codes, map_rows, map_cap) : make_v_map(&tv, v_codes, map_rows, map_cap)))
         return st;
     const int tiles = (span + 127) / 128;
     qk4v8::AttnParams p{};
@@ -459,6 +504,7 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
     p.block_table = pages.block_table;
     p.max_pages = pages.max_pages;
     p.num_pages = pages.num_pages;
+    p.v_fp4 = pages.v_fp4 ? 1 : 0;
     p.scale_log2 = resolve_scale(softmax_scale) * kLog2e;
     p.decode = 1;
     p.n_qtiles = 1;
@@ -481,9 +527,9 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
     // G*nq <= 32 query rows: the swap-AB decode kernel; 33..64: the GQA decode
     // kernel; larger groups use the 128-row attention kernel in its decode
     // instantiation.
-    cudaError_t e = swap_ab_rows(Hq, Hkv, nq) ? qk4v8::launch_decode(tk, tv, p, B * Hkv * splits, stream)
-                    : gqa_rows(Hq, Hkv, nq)   ? qk4v8::launch_gqa_decode(tk, tv, p, stream)
-                                              : qk4v8::launch_attention(tk, tv, p, B * Hkv * splits, stream);
+    cudaError_t e = use_swap  ? qk4v8::launch_decode(tk, tv, p, B * Hkv * splits, stream)
+                    : use_gqa ? qk4v8::launch_gqa_decode(tk, tv, p, stream)
+                              : qk4v8::launch_attention(tk, tv, p, B * Hkv * splits, stream);
     if (e != cudaSuccess) return cuda_error(e, "attention (decode) launch");
     *splits_used = splits;
     *direct = direct_out;
@@ -587,6 +633,18 @@ int qk4v8_attention_decode_paged(const uint8_t *q_codes, const uint8_t *q_scales
                          num_splits, workspace, workspace_bytes, out, lse, dev_status, stream);
 }
 
+int qk4v8_attention_decode_v4(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
+                              const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
+                              const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
+                              int causal_in_block, int window, float softmax_scale, int num_splits, void *workspace,
+                              size_t workspace_bytes, void *out, float *lse, int32_t *dev_status, void *stream) {
+    KvPages layout;
+    layout.v_fp4 = true;
+    return decode_packed(q_codes, q_scales, B, Hq, nq, q_cap, k_codes, k_scales, v_codes, v_scales, Hkv, kv_cap,
+                         layout, seqlens_k, max_seqlen, causal_in_block, window, softmax_scale, num_splits, workspace,
+                         workspace_bytes, out, lse, dev_status, stream);
+}
+
 int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq, int q_cap,
                            const uint8_t *k_codes, const uint8_t *k_scales, const uint8_t *v_codes,
                            const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k, int max_seqlen,
@@ -655,7 +713,7 @@ int decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_stride_b, int64_
     int used = 0;
     bool direct = false;
     DecodeQuery dq;
-    if (swap_ab_rows(Hq, Hkv, nq)) {
+    if (swap_ab_rows(Hq, Hkv, nq) || (pages.v_fp4 && (Hq / Hkv) * nq <= qk4v8::kDecodeMaxRows)) {
         dq.bf16 = static_cast<const __nv_bfloat16 *>(q);
         dq.sb = q_stride_b;
         dq.st = q_stride_t;
@@ -732,6 +790,19 @@ int qk4v8_attention_decode_bf16_paged(const void *q, int B, int Hq, int nq, int6
     return decode_bf16(q, B, Hq, nq, q_stride_b, q_stride_t, q_stride_h, k_codes, k_scales, v_codes, v_scales, Hkv,
                        max_pages * 128, pages, seqlens_k, max_seqlen, causal_in_block, window, softmax_scale,
                        num_splits, workspace, workspace_bytes, out, lse, dev_status, stream);
+}
+
+int qk4v8_attention_decode_bf16_v4(const void *q, int B, int Hq, int nq, int64_t q_stride_b, int64_t q_stride_t,
+                                   int64_t q_stride_h, const uint8_t *k_codes, const uint8_t *k_scales,
+                                   const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap,
+                                   const int32_t *seqlens_k, int max_seqlen, int causal_in_block, int window,
+                                   float softmax_scale, int num_splits, void *workspace, size_t workspace_bytes,
+                                   void *out, float *lse, int32_t *dev_status, void *stream) {
+    KvPages layout;
+    layout.v_fp4 = true;
+    return decode_bf16(q, B, Hq, nq, q_stride_b, q_stride_t, q_stride_h, k_codes, k_scales, v_codes, v_scales, Hkv,
+                       kv_cap, layout, seqlens_k, max_seqlen, causal_in_block, window, softmax_scale, num_splits,
+                       workspace, workspace_bytes, out, lse, dev_status, stream);
 }
 
 size_t qk4v8_kv_tail_bytes(int B, int Hkv) {

@@ -230,8 +230,9 @@ __device__ __noinline__ void rescale_o_cols(uint32_t taddr, int nt, int nc, int 
 
 }  // namespace
 
-// kExt: the instance for draft-block windows and paged caches; the other is
-// the plain decode over a contiguous cache.
+// kExt: the instance for draft-block windows, paged caches and MXFP4 V (the
+// QK4V4 comparison point); the other is the plain decode over a contiguous
+// MXFP8-V cache.
 template <int NT, int RW, int NC, int ST, int MINB, bool kExt>
 __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
     qk4v8_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
@@ -354,7 +355,10 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
             int row, blk;
             kv_tile_row<kExt>(p, b, h_kv, tile, pl, row, blk);
             if (lane == 0) {
-                mbar_arrive_expect_tx(&kv_full[st], Lay::kKBytes + Lay::kVBytes + 1024);
+                // An MXFP4 V tile lands unpacked (one byte per code in shared memory),
+                // but the copy moves its packed bytes, half of the MXFP8 tile's.
+                const int v_bytes = kExt && p.v_fp4 ? Lay::kVBytes / 2 : Lay::kVBytes;
+                mbar_arrive_expect_tx(&kv_full[st], Lay::kKBytes + v_bytes + 1024);
                 tma_load_3d(smem + Lay::kK + st * Lay::kKBytes, &tmap_k, 0, blk * 128, row, &kv_full[st]);
                 tma_load_3d(smem + Lay::kV + st * Lay::kVBytes, &tmap_v, blk * 128, 0, row, &kv_full[st]);
                 const int64_t atom = (static_cast<int64_t>(row) * nblk + blk) * 512;
@@ -369,7 +373,8 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
                 if (!__all_sync(0xffffffffu, ok)) break;
                 const int jv = L - tile * 128;
                 uint8_t *vt = smem + Lay::kV + st * Lay::kVBytes;
-                for (int c = lane; c < 128 * 8; c += 32) {
+                // (E2M1 has no NaN or infinity: MXFP4 V codes need no zeroing.)
+                for (int c = lane; c < 128 * 8 && !(kExt && p.v_fp4); c += 32) {
                     const int row = c >> 3, q = c & 7;
                     if (16 * q + 16 <= jv) continue;
                     uint8_t *chunk = vt + row * 128 + ((q ^ (row & 7)) << 4);
@@ -401,7 +406,8 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
             tc_fence_after();
             const uint32_t sb = smem_u32(smem);
             constexpr uint32_t kIdQK = idesc_d(1u, NT);      // E2M1 x E2M1, N = NT
-            constexpr uint32_t kIdPV = idesc_d(0u, 2 * NT);  // E4M3 x E4M3, N = 2 NT
+            // E4M3 V x E4M3 P, N = 2 NT; with MXFP4 V the A type field is E2M1 (5).
+            const uint32_t kIdPV = idesc_d(0u, 2 * NT) | (kExt && p.v_fp4 ? (5u << 7) : 0u);
             // Descriptors for stage 0 / buffer 0; other stages are fixed
             // offsets of the 14-bit start-address field (in 16-byte units).
             const uint64_t dQ = smem_desc(sb + Lay::kQ, 16, 512, 4);
@@ -834,7 +840,7 @@ static cudaError_t launch_nt(const CUtensorMap &tk, const CUtensorMap &tv, const
         if (e != cudaSuccess) return e;
         if (dev < kMaxDevices) configured[dev] = true;
     }
-    if (p.window > 0 || p.block_table)
+    if (p.window > 0 || p.block_table || p.v_fp4)
         qk4v8_decode_kernel<NT, RW, NC, ST, MINB, true><<<grid, Lay::kThreads, Lay::kBytes, stream>>>(tk, tv, p);
     else
         qk4v8_decode_kernel<NT, RW, NC, ST, MINB, false><<<grid, Lay::kThreads, Lay::kBytes, stream>>>(tk, tv, p);

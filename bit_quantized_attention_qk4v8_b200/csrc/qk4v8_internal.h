@@ -38,6 +38,9 @@ struct AttnParams {
     // (kv_cap is then max_pages * 128); null: contiguous [B][Hkv][kv_cap].
     const int32_t *block_table;
     int max_pages, num_pages;
+    // Decode only: V is MXFP4 (E2M1 codes [B][Hkv][128][kv_cap / 2], the QK4V4
+    // comparison point) instead of MXFP8.
+    int v_fp4;
     float scale_log2;         // softmax_scale * log2(e)
     int decode;               // 0: units (b, h_q, q tile); 1: units (b, h_kv, split)
     int n_qtiles;
@@ -62,6 +65,9 @@ cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, i
 cudaError_t launch_quantize_v(const void *v, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                               const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
                               cudaStream_t stream);
+cudaError_t launch_quantize_v4(const void *v, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
+                               const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
+                               cudaStream_t stream);
 cudaError_t launch_attention(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v, const AttnParams &p,
                              int grid, cudaStream_t stream);
 // Prefill kernel (persistent: one CTA per SM over the (sequence, query head,

@@ -197,6 +197,97 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__
             reinterpret_cast<const uint4 *>(atom)[threadIdx.x];
 }
 
+// ------------------------------------------------------------------ MXFP4 V
+
+// The QK4V4 comparison point (MpFA article, sections 2.2 and 5.3): V in MXFP4,
+// groups of 32 along the token axis like the MXFP8 V. Same staging as
+// quantize_v_kernel; each thread encodes one channel's 32-token group to 16
+// bytes of packed E2M1 (even token in the low nibble), and the 128-token tile of
+// a channel row is 64 bytes of codes [B][H][128][cap / 2].
+constexpr int kC4Pitch = 80;  // bytes per staged code row (64 + 16 padding)
+
+__global__ void __launch_bounds__(256) quantize_v4_kernel(const __nv_bfloat16 *__restrict__ v, int B, int S, int H,
+                                                          int64_t sb, int64_t ss, int64_t sh,
+                                                          const int32_t *__restrict__ seqlens, int cap,
+                                                          uint8_t *__restrict__ codes,
+                                                          uint8_t *__restrict__ scales) {
+    __shared__ __align__(16) uint16_t tile[128 * kVPitch];
+    __shared__ __align__(16) uint8_t atom[512];
+    uint8_t *ctile = reinterpret_cast<uint8_t *>(tile);  // [128 channels][kC4Pitch] after the barrier
+    const int nblk = cap / 128;
+    const int blk = blockIdx.x % nblk;
+    const int h = (blockIdx.x / nblk) % H;
+    const int b = blockIdx.x / (nblk * H);
+    const int t0 = blk * 128;
+    int valid_len = S;
+    if (seqlens) {
+        int L = seqlens[b];
+        valid_len = L < valid_len ? L : valid_len;
+    }
+    for (int i = threadIdx.x; i < 128 * 16; i += 256) {
+        const int tk = i >> 4, ch = i & 15;
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (t0 + tk < valid_len)
+            raw = *reinterpret_cast<const uint4 *>(v + b * sb + static_cast<int64_t>(t0 + tk) * ss + h * sh + ch * 8);
+        *reinterpret_cast<uint4 *>(&tile[tk * kVPitch + ch * 8]) = raw;
+    }
+    __syncthreads();
+    const int c = threadIdx.x & 127;
+    const int g0 = threadIdx.x >> 7;
+    uint32_t words[2][4];
+    int Xs[2];
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+        const int g = g0 + 2 * gi;
+        float amax = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j)
+            amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(tile[(g * 32 + j) * kVPitch + c]) << 16)));
+        const int X = shared_exponent(amax, 2);
+        Xs[gi] = X;
+        const float f = pow2_neg(X);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float y[8];
+            uint32_t sign = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t bits = tile[(g * 32 + 8 * q + e) * kVPitch + c];
+                y[e] = fabsf(__uint_as_float(bits << 16)) * f;
+                sign |= ((bits >> 15) & 1u) << (4 * e + 3);
+            }
+            words[gi][q] = cvt_e2m1x8(y) | sign;
+        }
+    }
+    __syncthreads();  // every read of the bf16 staging is done before it is overwritten
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+        const int g = g0 + 2 * gi;
+        *reinterpret_cast<uint4 *>(&ctile[c * kC4Pitch + g * 16]) =
+            make_uint4(words[gi][0], words[gi][1], words[gi][2], words[gi][3]);
+        atom[(c & 31) * 16 + (c >> 5) * 4 + g] = static_cast<uint8_t>(Xs[gi] + 127);
+    }
+    __syncthreads();
+    const int64_t head = static_cast<int64_t>(b) * H + h;
+    for (int i = threadIdx.x; i < 128 * 4; i += 256) {
+        const int row = i >> 2, ch = i & 3;
+        *reinterpret_cast<uint4 *>(codes + (head * 128 + row) * (cap / 2) + t0 / 2 + ch * 16) =
+            *reinterpret_cast<const uint4 *>(&ctile[row * kC4Pitch + ch * 16]);
+    }
+    if (threadIdx.x < 32)
+        reinterpret_cast<uint4 *>(scales + (head * nblk + blk) * 512)[threadIdx.x] =
+            reinterpret_cast<const uint4 *>(atom)[threadIdx.x];
+}
+
+cudaError_t launch_quantize_v4(const void *v, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
+                               const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
+                               cudaStream_t stream) {
+    const int64_t grid = static_cast<int64_t>(B) * H * (cap / 128);
+    quantize_v4_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(v), B, S, H, sb, ss, sh, seqlens, cap, codes, scales);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                                const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
                                cudaStream_t stream, bool pad_to_cap, bool rotate) {

@@ -251,6 +251,45 @@ QK4V8_API int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_sc
                            void *out, float *lse, int32_t *dev_status, void *stream);
 
 /*
+ * QK4V4: the comparison point of the MpFA article (section 2.2: V at 4 bits
+ * costs about 0.8 perplexity against QK4V8; section 5.3: on long texts it
+ * degrades further). V is quantized to MXFP4 (E2M1 codes, one E8M0 scale per
+ * 32 tokens along the sequence, the same OCP MX rule with emax 2), halving
+ * V's cache bytes (136 instead of 200 bytes per token and KV head with K).
+ *   MXFP4 V tensor, capacity cap (a multiple of 128):
+ *     codes  uint8 [B][H][128][cap/2]   two E2M1 codes per byte along the
+ *                                        token axis, even token in the low nibble
+ *                                        (qk4v8_mxfp4v_codes_bytes)
+ *     scales uint8 [B][H][cap/128][512] as for MXFP8 V
+ * qk4v8_quantize_v4: arguments as for qk4v8_quantize_v.
+ * qk4v8_attention_decode_v4 / qk4v8_attention_decode_bf16_v4: the decode calls
+ * (window included) over packed MXFP4 K and MXFP4 V, on the swap-AB kernel for
+ * up to 64 query rows per KV head; V codes 32-byte aligned, contiguous caches.
+ * P stays two E4M3 terms; the block-scaled MMA takes V as its E2M1 operand.
+ */
+QK4V8_API size_t qk4v8_mxfp4v_codes_bytes(int B, int H, int cap);
+
+QK4V8_API int qk4v8_quantize_v4(const void *v, int B, int S, int H, int d, int64_t stride_b, int64_t stride_s,
+                                int64_t stride_h, const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
+                                void *stream);
+
+QK4V8_API int qk4v8_attention_decode_v4(const uint8_t *q_codes, const uint8_t *q_scales, int B, int Hq, int nq,
+                                        int q_cap, const uint8_t *k_codes, const uint8_t *k_scales,
+                                        const uint8_t *v_codes, const uint8_t *v_scales, int Hkv, int kv_cap,
+                                        const int32_t *seqlens_k, int max_seqlen, int causal_in_block, int window,
+                                        float softmax_scale, int num_splits, void *workspace,
+                                        size_t workspace_bytes, void *out, float *lse, int32_t *dev_status,
+                                        void *stream);
+
+QK4V8_API int qk4v8_attention_decode_bf16_v4(const void *q, int B, int Hq, int nq, int64_t q_stride_b,
+                                             int64_t q_stride_t, int64_t q_stride_h, const uint8_t *k_codes,
+                                             const uint8_t *k_scales, const uint8_t *v_codes,
+                                             const uint8_t *v_scales, int Hkv, int kv_cap, const int32_t *seqlens_k,
+                                             int max_seqlen, int causal_in_block, int window, float softmax_scale,
+                                             int num_splits, void *workspace, size_t workspace_bytes, void *out,
+                                             float *lse, int32_t *dev_status, void *stream);
+
+/*
  * Draft-block attention: decode with a sliding window (MiMo DFlash article,
  * section on block-diffusion speculative decoding: the draft model predicts a
  * block of 8 tokens in one forward; its attention sees the in-block positions
