@@ -437,8 +437,8 @@ int decode_splitkv(const DecodeQuery &q, int B, int Hq, int nq, const uint8_t *k
         max_seqlen > kv_cap)
         return set_error(QK4V8_ERR_INVALID_ARG, "bad lengths q_cap=%d kv_cap=%d max_seqlen=%d", q.cap, kv_cap,
                          max_seqlen);
-    // MXFP4 V runs on the swap-AB kernel, up to 64 query rows per KV head.
-    const bool use_swap = swap_ab_rows(Hq, Hkv, nq) || pages.v_fp4;
+    // MXFP4 V runs on the swap-AB and GQA decode kernels, up to 64 query rows per KV head.
+    const bool use_swap = swap_ab_rows(Hq, Hkv, nq);
     const bool use_gqa = !use_swap && gqa_rows(Hq, Hkv, nq);
     if (q.bf16 && !use_swap)
         return set_error(QK4V8_ERR_INVALID_ARG, "bf16 Q in the split kernel needs (Hq/Hkv)*nq < %d",
@@ -713,7 +713,7 @@ int decode_bf16(const void *q, int B, int Hq, int nq, int64_t q_stride_b, int64_
     int used = 0;
     bool direct = false;
     DecodeQuery dq;
-    if (swap_ab_rows(Hq, Hkv, nq) || (pages.v_fp4 && (Hq / Hkv) * nq <= qk4v8::kDecodeMaxRows)) {
+    if (swap_ab_rows(Hq, Hkv, nq)) {
         dq.bf16 = static_cast<const __nv_bfloat16 *>(q);
         dq.sb = q_stride_b;
         dq.st = q_stride_t;

@@ -122,9 +122,10 @@ __device__ __forceinline__ uint32_t gd_sf_id(uint32_t idesc, uint32_t id) { retu
 }  // namespace
 
 // kExt: the instance for draft-block attention (query rows see only keys from
-// the window's first key, kv_window_lo, on) and paged caches (key tiles looked
-// up in the block table); the other instance is the plain decode over a
-// contiguous cache, with neither in its loops.
+// the window's first key, kv_window_lo, on), paged caches (key tiles looked up
+// in the block table) and MXFP4 V (the QK4V4 comparison point); the other
+// instance is the plain decode over a contiguous MXFP8-V cache, with none of
+// these in its loops.
 template <bool kExt>
 __global__ void __launch_bounds__(kGdThreads, 1)
     qk4v8_gqa_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
@@ -210,7 +211,11 @@ __global__ void __launch_bounds__(kGdThreads, 1)
         for (int s = 0; s < kGdVStages; ++s)
             for (int cc = lane; cc < 16 * 8; cc += 32) {
                 const int r = 128 + (cc >> 3);
-                const uint32_t fillv = r == 128 ? 0x38383838u : 0u;
+                // 1.0 is E4M3 0x38; with MXFP4 V (extended instance) it is E2M1 0x2,
+                // and 0x22 in every byte gives two 1.0 codes whichever 8 bytes of each
+                // 16-byte slot the padded FP4 layout reads.
+                const uint32_t one = kExt && p.v_fp4 ? 0x22222222u : 0x38383838u;
+                const uint32_t fillv = r == 128 ? one : 0u;
                 *reinterpret_cast<uint4 *>(smem + S::kV + s * S::kVBytes + r * 128 + (cc & 7) * 16) =
                     make_uint4(fillv, fillv, fillv, fillv);
             }
@@ -355,7 +360,8 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                 int row, blk;
                 kv_tile_row<kExt>(p, u.b, u.h_kv, tile, pl, row, blk);
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&v_full[sv], S::kVTmaBytes + 512);
+                    // An MXFP4 tile lands unpacked; the copy moves half the bytes.
+                    mbar_arrive_expect_tx(&v_full[sv], (kExt && p.v_fp4 ? S::kVTmaBytes / 2 : S::kVTmaBytes) + 512);
                     tma_load_3d(smem + S::kV + sv * S::kVBytes, &tmap_v, blk * 128, 0, row, &v_full[sv]);
                     bulk_load(smem + S::kSfV + sv * 512, p.v_scales + (static_cast<int64_t>(row) * nblk + blk) * 512,
                               512, &v_full[sv]);
@@ -369,7 +375,8 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                     if (!ok) break;
                     const int jv = u.L - tile * 128;  // valid keys in this tile, 1..127
                     uint8_t *vt = smem + S::kV + sv * S::kVBytes;
-                    for (int cc = lane; cc < 128 * 8; cc += 32) {
+                    // (E2M1 has no NaN or infinity: MXFP4 V codes need no zeroing.)
+                    for (int cc = lane; cc < 128 * 8 && !(kExt && p.v_fp4); cc += 32) {
                         const int r = cc >> 3, q = cc & 7;
                         if (16 * q + 16 <= jv) continue;
                         uint8_t *chunk = vt + r * 128 + ((q ^ (r & 7)) << 4);
@@ -479,6 +486,8 @@ __global__ void __launch_bounds__(kGdThreads, 1)
             // O += P(2k) V(2k) + P(2k+1) V(2k+1), once both V tiles have landed and
             // the set has written its P tiles; the unit's first one overwrites O,
             // once the previous unit's epilogue has read it.
+            // E4M3 P x E4M3 V, N = 144; with MXFP4 V the B format field says E2M1 (5).
+            const uint32_t id_pv = kGdIdPV | (kExt && p.v_fp4 ? (5u << 10) : 0u);
             auto issue_pv = [&](int k) -> bool {
                 const int gp = gp0 + k, set = gp & 1;
                 const bool has1 = 2 * k + 1 < T;
@@ -505,7 +514,7 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                         tc_cp_32x128b_warpx4(tSfP, dSfP0 + static_cast<uint64_t>((2 * set + h) * 32));
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            tc_mma_mxf8(tO, dP + 2 * kk, dV + 2 * kk, gd_sf_id(kGdIdPV, kk), tSfP | (kk << 30),
+                            tc_mma_mxf8(tO, dP + 2 * kk, dV + 2 * kk, gd_sf_id(id_pv, kk), tSfP | (kk << 30),
                                         tSfV | (kk << 30), (k > 0 || h > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(&pv_done[set]);
@@ -983,7 +992,7 @@ cudaError_t launch_gqa_decode(const CUtensorMap &tk, const CUtensorMap &tv, cons
     }
     // Persistent: one CTA per SM (shared memory and the 512 TMEM columns allow no
     // more); the kernel schedules the work over the grid itself.
-    if (p.window > 0 || p.block_table)
+    if (p.window > 0 || p.block_table || p.v_fp4)
         qk4v8_gqa_decode_kernel<true><<<sms, kGdThreads, GdSmem::kBytes, stream>>>(tk, tv, p);
     else
         qk4v8_gqa_decode_kernel<false><<<sms, kGdThreads, GdSmem::kBytes, stream>>>(tk, tv, p);

@@ -263,8 +263,9 @@ QK4V8_API int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_sc
  *     scales uint8 [B][H][cap/128][512] as for MXFP8 V
  * qk4v8_quantize_v4: arguments as for qk4v8_quantize_v.
  * qk4v8_attention_decode_v4 / qk4v8_attention_decode_bf16_v4: the decode calls
- * (window included) over packed MXFP4 K and MXFP4 V, on the swap-AB kernel for
- * up to 64 query rows per KV head; V codes 32-byte aligned, contiguous caches.
+ * (window included) over packed MXFP4 K and MXFP4 V, for up to 64 query rows
+ * per KV head (the swap-AB and GQA decode kernels); V codes 32-byte aligned,
+ * contiguous caches.
  * P stays two E4M3 terms; the block-scaled MMA takes V as its E2M1 operand.
  */
 QK4V8_API size_t qk4v8_mxfp4v_codes_bytes(int B, int H, int cap);
