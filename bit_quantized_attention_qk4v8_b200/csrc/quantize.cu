@@ -20,48 +20,44 @@ namespace qk4v8 {
 
 // ------------------------------------------------------------------ MXFP4
 
-// 16 lanes per token row (128 channels), 8 channels per lane, 4 lanes per group
-// of 32; a warp takes two rows per step, each half-warp one. blockIdx.y is the
-// batch entry; its rows (t, h) are visited in input order (t major), so loads
-// are contiguous. Tokens 0 .. row_len-1 of each sequence are visited: row_len =
-// cap writes the whole capacity (zero codes and scales past the valid length),
-// row_len = S only the rows of the input. Each half-warp steps its (t, h)
-// position by a fixed amount and keeps two rows in flight: the kernel is meant
-// to be bound by memory, and an integer division per row would make it bound by
-// instruction issue instead.
-__device__ __forceinline__ void qk_store_row(uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int64_t head,
-                                             int cap, int t, int sub, uint32_t packed, int X, bool valid) {
-    reinterpret_cast<uint32_t *>(codes + (head * cap + t) * 64)[sub] = packed;
-    if ((sub & 3) == 0) {
-        const int g = sub >> 2;
-        uint8_t *blk = scales + (head * (cap / 128) + t / 128) * 512;
-        blk[(t & 31) * 16 + ((t & 127) >> 5) * 4 + g] = valid ? static_cast<uint8_t>(X + 127) : 0;
-    }
-}
+// One lane per MX group: 4 lanes per 128-channel (token, head) row, 32
+// channels (64 bytes of bf16) per lane, so the group amax needs no shuffle and
+// a warp takes 8 rows per step. blockIdx.y is the batch entry; its rows (t, h)
+// are visited in input order (t major), so a warp's loads are contiguous.
+// Tokens 0 .. row_len-1 of each sequence are visited: row_len = cap writes the
+// whole capacity (zero codes and scales past the valid length), row_len = S
+// only the rows of the input. Each lane steps its (t, h) position by a fixed
+// amount: an integer division per row would make the kernel bound by
+// instruction issue instead of memory.
+//
+// With kRotate the row is first rotated by H / sqrt(128), H the Sylvester
+// Hadamard matrix (MpFA article, sections 2.1 and 3.1), in fp32 as the fast
+// Walsh-Hadamard transform: butterfly stages of stride 1..16 inside the lane,
+// 32 and 64 across the row's lanes (lane xor 1, 2), each mapping the pair
+// (a, b) at channels (i, i + stride) to (a + b, a - b); then one multiply by
+// the fp32 value nearest 2^-3.5. Packed f32x2 adds give the same bits as
+// scalar ones.
 
-// With kRotate, each row is first rotated by H / sqrt(128) (hadamard128_rows)
-// and the rotated fp32 values are quantized.
-__device__ __forceinline__ uint32_t qk_encode_row(uint4 raw, bool valid, int sub, bool rotate, int &X) {
-    if (!rotate) return mxfp4_encode8(raw, valid, X);
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    float v[8];
+// Butterfly stage of stride s (s >= 2) over a lane's 32 values held as 16 pairs.
+template <int S>
+__device__ __forceinline__ void fwht_stage_pairs(float2 (&w)[16]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float(w[i] << 16);
-        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    for (int i = 0; i < 16; ++i) {
+        if ((2 * i) & S) continue;
+        const float2 a = w[i], b = w[i + S / 2];
+        w[i] = fadd2(a, b);
+        w[i + S / 2] = fsub2(a, b);
     }
-    hadamard128_rows(v, sub);
-    return mxfp4_encode8_f32(v, valid, X);
 }
 
 template <bool kRotate>
-__global__ void __launch_bounds__(256) quantize_qk_kernel(const __nv_bfloat16 *__restrict__ x, int B, int S, int H,
+__global__ void __launch_bounds__(256, kRotate ? 3 : 4) quantize_qk_kernel(const __nv_bfloat16 *__restrict__ x, int B, int S, int H,
                                                           int64_t sb, int64_t ss, int64_t sh,
                                                           const int32_t *__restrict__ seqlens, int cap,
                                                           int row_len, uint8_t *__restrict__ codes,
                                                           uint8_t *__restrict__ scales) {
-    const int sub = threadIdx.x & 15;  // lane within the row
-    const int hw = (threadIdx.x >> 4) & 1;
+    const int lane = threadIdx.x & 31;
+    const int g = lane & 3;   // MX group (channels 32g .. 32g+31) of this lane
     const int b = blockIdx.y;
     const int rows = row_len * H;  // rows of this batch entry (the launcher keeps this below 2^30)
     int valid_len = S;
@@ -69,43 +65,89 @@ __global__ void __launch_bounds__(256) quantize_qk_kernel(const __nv_bfloat16 *_
         const int L = seqlens[b];
         valid_len = L < valid_len ? L : valid_len;
     }
-    const int step = static_cast<int>(gridDim.x) * (blockDim.x >> 5) * 2;  // rows per grid step
+    const int step = static_cast<int>(gridDim.x) * (blockDim.x >> 5) * 8;  // rows per grid step
     const int step_t = step / H, step_h = step - step_t * H;
-    // The loop bound is taken per warp (two rows) so every lane reaches the shuffles.
-    int base = (static_cast<int>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 2;
-    int t = (base + hw) / H;
-    int h = (base + hw) - t * H;
+    // The loop bound is taken per warp (8 rows) so every lane reaches the shuffles.
+    int base = (static_cast<int>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 8;
+    int t = (base + (lane >> 2)) / H;
+    int h = (base + (lane >> 2)) - t * H;
     const __nv_bfloat16 *xb = x + b * sb;
     const int64_t head_b = static_cast<int64_t>(b) * H;
-    auto advance = [&](int &tt, int &hh) {
-        tt += step_t;
-        hh += step_h;
-        if (hh >= H) {
-            hh -= H;
-            ++tt;
+    const int nblk = cap / 128;
+    for (; base < rows; base += step) {
+        const bool in = base + (lane >> 2) < rows;
+        const bool valid = in && t < valid_len;
+        uint4 raw[4] = {};
+        if (valid) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(xb + t * ss + h * sh + g * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) raw[i] = src[i];
         }
-    };
-    for (; base < rows; base += 2 * step) {
-        // Two rows of this half-warp: base + hw and base + hw + step.
-        int t1 = t, h1 = h;
-        advance(t1, h1);
-        const bool in0 = base + hw < rows, in1 = base + step + hw < rows;
-        const bool v0 = in0 && t < valid_len, v1 = in1 && t1 < valid_len;
-        uint4 raw0 = make_uint4(0, 0, 0, 0), raw1 = make_uint4(0, 0, 0, 0);
-        if (v0) raw0 = *reinterpret_cast<const uint4 *>(xb + t * ss + h * sh + sub * 8);
-        if (v1) raw1 = *reinterpret_cast<const uint4 *>(xb + t1 * ss + h1 * sh + sub * 8);
-        int X0, X1;
-        const uint32_t p0 = qk_encode_row(raw0, v0, sub, kRotate, X0);
-        if (in0) qk_store_row(codes, scales, head_b + h, cap, t, sub, p0, X0, v0);
-        // The second pair of rows is encoded by the whole warp too (shuffles),
-        // when the warp's first row of it exists.
-        if (base + step < rows) {
-            const uint32_t p1 = qk_encode_row(raw1, v1, sub, kRotate, X1);
-            if (in1) qk_store_row(codes, scales, head_b + h1, cap, t1, sub, p1, X1, v1);
+        // bf16 -> f32, exact: channel 2k in the low half of word k.
+        float2 w[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t ws[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                w[4 * i + k] = make_float2(__uint_as_float(ws[k] << 16), __uint_as_float(ws[k] & 0xFFFF0000u));
         }
-        t = t1;
-        h = h1;
-        advance(t, h);
+        if (kRotate) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {  // stride 1: the two halves of each pair
+                const float a = w[i].x, c = w[i].y;
+                w[i] = make_float2(a + c, a - c);
+            }
+            fwht_stage_pairs<2>(w);
+            fwht_stage_pairs<4>(w);
+            fwht_stage_pairs<8>(w);
+            fwht_stage_pairs<16>(w);
+#pragma unroll
+            for (int m = 1; m <= 2; m <<= 1) {  // strides 32 and 64: the row's other lanes
+                const bool upper = (g & m) != 0;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, w[i].x, m),
+                                                 __shfl_xor_sync(0xffffffffu, w[i].y, m));
+                    w[i] = upper ? fsub2(o, w[i]) : fadd2(w[i], o);
+                }
+            }
+            constexpr float kRsqrt128 = 0x1.6a09e6p-4f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = fmul2(w[i], make_float2(kRsqrt128, kRsqrt128));
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fmaxf(fabsf(w[i].x), fabsf(w[i].y)));
+        const int X = shared_exponent(amax, 2);
+        const float f = pow2_neg(X);
+        uint32_t packed[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float y[8];
+            uint32_t sign = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 a = w[4 * q + e];
+                y[2 * e] = fabsf(a.x) * f;  // exact: power-of-two scaling
+                y[2 * e + 1] = fabsf(a.y) * f;
+                sign |= (__float_as_uint(a.x) >> 31) << (8 * e + 3);
+                sign |= (__float_as_uint(a.y) >> 31) << (8 * e + 7);
+            }
+            packed[q] = valid ? (cvt_e2m1x8(y) | sign) : 0u;
+        }
+        if (in) {
+            *reinterpret_cast<uint4 *>(codes + ((head_b + h) * cap + t) * 64 + g * 16) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            scales[((head_b + h) * nblk + t / 128) * 512 + (t & 31) * 16 + ((t & 127) >> 5) * 4 + g] =
+                valid ? static_cast<uint8_t>(X + 127) : 0;
+        }
+        t += step_t;
+        h += step_h;
+        if (h >= H) {
+            h -= H;
+            ++t;
+        }
     }
 }
 
@@ -294,11 +336,11 @@ cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, i
     const int row_len = pad_to_cap ? cap : S;
     const int64_t rows = static_cast<int64_t>(row_len) * H;  // per batch entry
     if (rows >= (int64_t{1} << 30)) return cudaErrorInvalidValue;
-    // About one wave over all batch entries: 6 CTAs (48 warps, 40 registers a
-    // thread) per SM, each warp with two pairs of rows in flight.
-    const int64_t rows_per_cta = 256 / 16;
+    // About one wave over all batch entries (4 CTAs per SM, 3 with the rotation),
+    // 64 rows per CTA per step.
+    const int64_t rows_per_cta = 64;
     int64_t gx = (rows + rows_per_cta - 1) / rows_per_cta;
-    const int64_t wave = (148 * 6 + B - 1) / B;
+    const int64_t wave = (148 * (rotate ? 3 : 4) + B - 1) / B;
     if (gx > wave) gx = wave;
     if (gx < 1) gx = 1;
     // The grid's y extent is at most 65535: larger batches go in chunks.
