@@ -159,6 +159,31 @@ __global__ void __launch_bounds__(256, kRotate ? 3 : 4) quantize_qk_kernel(const
 constexpr int kVPitch = 136;  // bf16 elements per staged token row (16-byte padding)
 constexpr int kCPitch = 144;  // bytes per staged code row
 
+// Loads the bf16 tile of 128 tokens x 128 channels of (b, h) from token t0 into
+// shared memory (row pitch kVPitch): all eight 16-byte loads of a thread are
+// issued before the first store, so a CTA keeps its whole 32 KiB in flight.
+// Tokens at or past valid_len read as zeros. Ends with a CTA barrier.
+__device__ __forceinline__ void stage_v_tile(const __nv_bfloat16 *__restrict__ v, int b, int h, int t0,
+                                             int valid_len, int64_t sb, int64_t ss, int64_t sh,
+                                             uint16_t *tile) {
+    uint4 raw[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int i = threadIdx.x + 256 * k;
+        const int tk = i >> 4, ch = i & 15;
+        raw[k] = make_uint4(0, 0, 0, 0);
+        if (t0 + tk < valid_len)
+            raw[k] = *reinterpret_cast<const uint4 *>(v + b * sb + static_cast<int64_t>(t0 + tk) * ss + h * sh +
+                                                      ch * 8);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int i = threadIdx.x + 256 * k;
+        *reinterpret_cast<uint4 *>(&tile[(i >> 4) * kVPitch + (i & 15) * 8]) = raw[k];
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__restrict__ v, int B, int S, int H,
                                                          int64_t sb, int64_t ss, int64_t sh,
                                                          const int32_t *__restrict__ seqlens, int cap,
@@ -179,14 +204,7 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__
     }
     // Stage: invalid tokens read as zeros, which leaves them out of every amax
     // and gives them code 0; a group with no valid token gets scale byte 0.
-    for (int i = threadIdx.x; i < 128 * 16; i += 256) {
-        const int tk = i >> 4, ch = i & 15;
-        uint4 raw = make_uint4(0, 0, 0, 0);
-        if (t0 + tk < valid_len)
-            raw = *reinterpret_cast<const uint4 *>(v + b * sb + static_cast<int64_t>(t0 + tk) * ss + h * sh + ch * 8);
-        *reinterpret_cast<uint4 *>(&tile[tk * kVPitch + ch * 8]) = raw;
-    }
-    __syncthreads();
+    stage_v_tile(v, b, h, t0, valid_len, sb, ss, sh, tile);
     const int c = threadIdx.x & 127;
     const int g0 = threadIdx.x >> 7;
     uint32_t words[2][8];
@@ -266,14 +284,7 @@ __global__ void __launch_bounds__(256) quantize_v4_kernel(const __nv_bfloat16 *_
         int L = seqlens[b];
         valid_len = L < valid_len ? L : valid_len;
     }
-    for (int i = threadIdx.x; i < 128 * 16; i += 256) {
-        const int tk = i >> 4, ch = i & 15;
-        uint4 raw = make_uint4(0, 0, 0, 0);
-        if (t0 + tk < valid_len)
-            raw = *reinterpret_cast<const uint4 *>(v + b * sb + static_cast<int64_t>(t0 + tk) * ss + h * sh + ch * 8);
-        *reinterpret_cast<uint4 *>(&tile[tk * kVPitch + ch * 8]) = raw;
-    }
-    __syncthreads();
+    stage_v_tile(v, b, h, t0, valid_len, sb, ss, sh, tile);
     const int c = threadIdx.x & 127;
     const int g0 = threadIdx.x >> 7;
     uint32_t words[2][4];
