@@ -310,7 +310,9 @@ def run_decode(args, world, rank):
     kp = qk.quantize_qk(k, cap=cap, seqlens=sl)      # the cache: quantized once, outside the timing
     vp = qk.quantize_v(to_dev(gen["v"]), cap=cap, seqlens=sl)
     max_len = int(gen["seqlens"].max())
-    splits = args.splits if args.splits > 0 else qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, max_len)
+    # The split count from the host-side lengths (qk4v8_decode_plan_splits), as a
+    # serving scheduler that knows its batch would ask for it.
+    splits = args.splits if args.splits > 0 else qk.decode_plan_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, gen["seqlens"])
     ws_bytes = qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)
     ws = torch.empty((ws_bytes,), dtype=torch.uint8, device="cuda") if ws_bytes else None
     out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
@@ -458,7 +460,7 @@ def run_decode_workload(name, steps, warmup, hbm_gbs, hadamard):
     vp = qk.quantize_v(v, cap=cap, seqlens=sl)
     del v
     max_len = int(lens.max())
-    splits = qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, max_len)
+    splits = qk.decode_plan_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, gen["seqlens"])
     ws_bytes = qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)
     ws = torch.empty((ws_bytes,), dtype=torch.uint8, device="cuda") if ws_bytes else None
     out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")
@@ -509,7 +511,7 @@ def run_decode_v4(name, gen, steps, hbm_gbs):
     vp = qk.quantize_v4(to_dev(gen["v"]), cap=cap, seqlens=sl)
     q = to_dev(gen["q"])
     max_len = int(lens.max())
-    splits = qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, max_len)
+    splits = qk.decode_plan_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, gen["seqlens"])
     ws = torch.empty((max(16, qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)),),
                      dtype=torch.uint8, device="cuda")
     out = torch.empty((wl.B, wl.Sq, wl.Hq, 128), dtype=torch.bfloat16, device="cuda")

@@ -24,7 +24,8 @@ from ._lib import QK4V8Error, check, lib
 __all__ = [
     "MXFP4", "MXFP4V", "MXFP8V", "PagedKV", "QK4V8Error", "lib", "round_cap",
     "quantize_qk", "quantize_v", "quantize", "attention_prefill", "attention_decode",
-    "decode_workspace_bytes", "decode_default_splits", "attention_decode_splitkv", "decode_merge",
+    "decode_workspace_bytes", "decode_default_splits", "decode_plan_splits", "attention_decode_splitkv",
+    "decode_merge",
     "attention_decode_bf16", "decode_bf16_workspace_bytes",
     "paged_kv", "kv_append", "attention_decode_paged", "attention_decode_bf16_paged", "quantize_v4",
 ]
@@ -208,6 +209,16 @@ def decode_default_splits(B: int, Hq: int, Hkv: int, nq: int, max_seqlen: int, w
     if window:
         return int(lib().qk4v8_decode_default_splits_window(B, Hq, Hkv, nq, max_seqlen, int(window)))
     return int(lib().qk4v8_decode_default_splits(B, Hq, Hkv, nq, max_seqlen))
+
+
+def decode_plan_splits(B: int, Hq: int, Hkv: int, nq: int, seqlens, window: int = 0) -> int:
+    """Split count from the host-side sequence lengths (qk4v8_decode_plan_splits)."""
+    import numpy as np
+    lens = np.ascontiguousarray(np.asarray(seqlens if not torch.is_tensor(seqlens) else seqlens.cpu().numpy()),
+                                dtype=np.int32)
+    if lens.size != B:
+        raise ValueError("seqlens must have B entries")
+    return int(lib().qk4v8_decode_plan_splits(B, Hq, Hkv, nq, lens.ctypes.data, int(window)))
 
 
 def attention_decode(q: MXFP4, k: MXFP4, v, seqlens_k, max_seqlen: Optional[int] = None,

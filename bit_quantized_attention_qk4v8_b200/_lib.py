@@ -43,6 +43,7 @@ SIGNATURES = {
     "qk4v8_attention_decode_bf16_window": ([_vp, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i32,
                                             _vp, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp, _vp, _vp, _vp], _i32),
     "qk4v8_decode_default_splits_window": ([_i32, _i32, _i32, _i32, _i32, _i32], _i32),
+    "qk4v8_decode_plan_splits": ([_i32, _i32, _i32, _i32, _vp, _i32], _i32),
     "qk4v8_mxfp4v_codes_bytes": ([_i32, _i32, _i32], _sz),
     "qk4v8_quantize_v4": ([_vp, _i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp], _i32),
     "qk4v8_attention_decode_v4": ([_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _vp,

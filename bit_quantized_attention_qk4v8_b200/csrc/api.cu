@@ -9,7 +9,10 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 #include <mutex>
+#include <queue>
+#include <vector>
 
 #include "../../include/qk4v8.h"
 #include "../../include/qk4v8_test.h"
@@ -657,6 +660,83 @@ int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_scales, int 
 
 int qk4v8_decode_default_splits_window(int B, int Hq, int Hkv, int nq, int max_seqlen, int window) {
     return qk4v8_decode_default_splits(B, Hq, Hkv, nq, window_span(max_seqlen, nq, window));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Modelled time of a split-KV launch over sequences of `tiles` key tiles each
+// (times Hkv heads), `s` splits of `st` tiles: the CTAs start in launch order
+// (sequence, head, split) on `slots` resident slots, empty splits cost nothing,
+// and the active CTAs share the memory bandwidth: each streams min(kBoost,
+// slots / active) tiles per unit of time (1 when every slot is busy). Plus a
+// fixed cost per launch and the merge launch when s > 1. The constants were
+// fitted to measured split sweeps of the long-context decode workload (one
+// time unit is one tile at full occupancy).
+double model_split_time(const std::vector<int> &tiles, int Hkv, int s, int st, int slots) {
+    constexpr double kBoost = 1.5, kLaunch = 17.0, kMerge = 4.0;
+    std::priority_queue<double, std::vector<double>, std::greater<double>> fin;  // virtual finish times
+    double v = 0.0, t = 0.0;
+    auto advance = [&]() {
+        const double vf = fin.top();
+        const double n = static_cast<double>(fin.size());
+        const double rate = std::min(kBoost, static_cast<double>(slots) / n);
+        t += (vf - v) / rate;
+        v = vf;
+        fin.pop();
+    };
+    for (int tb : tiles)
+        for (int h = 0; h < Hkv; ++h)
+            for (int j = 0; j < s; ++j) {
+                const int w = std::min(st, tb - j * st);
+                if (w <= 0) break;
+                if (static_cast<int>(fin.size()) == slots) advance();
+                fin.push(v + w);
+            }
+    while (!fin.empty()) advance();
+    return t + kLaunch + (s > 1 ? kMerge : 0.0);
+}
+
+}  // namespace
+
+extern "C" {
+
+int qk4v8_decode_plan_splits(int B, int Hq, int Hkv, int nq, const int32_t *seqlens_host, int window) {
+    if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv || nq <= 0 || !seqlens_host || window < 0) return 1;
+    int max_len = 0;
+    for (int b = 0; b < B; ++b) max_len = std::max(max_len, seqlens_host[b]);
+    const int rows = (Hq / Hkv) * nq;
+    // Groups of 33..64 rows: the GQA decode kernel balances the key tiles itself.
+    if (rows >= qk4v8::kGqaMinRows || static_cast<int64_t>(B) * Hkv > 4096)
+        return qk4v8_decode_default_splits_window(B, Hq, Hkv, nq, max_len, window);
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+        sms = 148;
+        (void)cudaGetLastError();
+    }
+    const int slots = sms * (rows <= 16 ? 2 : 1);
+    std::vector<int> tiles(static_cast<size_t>(B));
+    int tmax = 1;
+    for (int b = 0; b < B; ++b) {
+        const int L = std::max(0, seqlens_host[b]);
+        const int lo = window > 0 ? std::max(0, L - nq - window) : 0;
+        tiles[b] = (L + 127) / 128 - lo / 128;
+        tmax = std::max(tmax, tiles[b]);
+    }
+    int best = 1;
+    double best_t = 0.0;
+    for (int s = 1; s <= 64 && s <= tmax; ++s) {
+        const int st = (tmax + s - 1) / s;
+        if (s > 1 && (tmax + st - 1) / st < s) continue;  // the same plan as a smaller s
+        const double t = model_split_time(tiles, Hkv, s, st, slots);
+        if (s == 1 || t < best_t) {
+            best_t = t;
+            best = s;
+        }
+    }
+    return best;
 }
 
 size_t qk4v8_decode_bf16_workspace_bytes(int B, int Hq, int Hkv, int nq, int num_splits) {

@@ -329,6 +329,21 @@ QK4V8_API int qk4v8_attention_decode_bf16_window(const void *q, int B, int Hq, i
 QK4V8_API int qk4v8_decode_default_splits_window(int B, int Hq, int Hkv, int nq, int max_seqlen, int window);
 
 /*
+ * Split count for a decode call when the caller knows the sequence lengths on
+ * the host (seqlens_host, int32 [B]; window as for the _window calls). For up
+ * to 32 query rows per KV head it models each candidate split count with the
+ * lengths as they are: CTAs start in launch order on the resident slots,
+ * splits past a sequence's end cost nothing, and the running CTAs share the
+ * memory bandwidth, so a last partial wave runs faster per CTA. It returns the
+ * count with the least modelled time (a fixed split count assumes every
+ * sequence has the longest length, and over-splits batches of mixed lengths).
+ * For 33..64 rows it returns qk4v8_decode_default_splits_window (that kernel
+ * balances its key tiles itself). Returns 1 for invalid sizes. Host only; no
+ * device work.
+ */
+QK4V8_API int qk4v8_decode_plan_splits(int B, int Hq, int Hkv, int nq, const int32_t *seqlens_host, int window);
+
+/*
  * Paged KV cache (MpFA article, section 6.1: the QK4V8 attention combined with
  * a quantized KV cache; section 3.2: block scales computed online as the data
  * arrives). The packed cache lives in pools of pages of 128 tokens; page p of

@@ -83,6 +83,28 @@ def test_default_splits(lib):
         assert f(*bad) == 1
 
 
+def test_plan_splits(lib):
+    """The length-aware plan (148 SMs without a device; two CTAs per SM up to 16
+    rows: 296 slots). Worked by hand for two sequences of 10 and 1 tiles, 4 rows,
+    one KV head: every CTA runs at the 1.5x single-CTA rate (2..11 CTAs on 296
+    slots). s=1: the 1-tile CTA ends at 1/1.5, the 10-tile one at 10/1.5 = 6.67,
+    plus the launch (17): 23.67. s=10 (1 tile per split): 11 CTAs all end at
+    0.67, plus launch and merge (17 + 4): 21.67, the least (s=5: 1.33 + 21).
+    For 33..64 rows it is the default plan; invalid sizes give 1."""
+    import ctypes
+    import numpy as np
+
+    def plan(B, Hq, Hkv, nq, lens, window=0):
+        a = np.ascontiguousarray(lens, dtype=np.int32)
+        return lib.qk4v8_decode_plan_splits(B, Hq, Hkv, nq, a.ctypes.data_as(ctypes.c_void_p), window)
+
+    assert plan(2, 4, 1, 1, [1280, 128]) == 10
+    assert plan(32, 32, 8, 1, [8192] * 32) == 1
+    assert plan(64, 64, 8, 8, [16384] * 64) == lib.qk4v8_decode_default_splits(64, 64, 8, 8, 16384)
+    assert plan(0, 4, 1, 1, [1]) == 1
+    assert lib.qk4v8_decode_plan_splits(2, 4, 1, 1, None, 0) == 1
+
+
 FAKE = 0x10000  # never dereferenced: validation rejects these calls first
 
 
