@@ -104,12 +104,15 @@ __global__ void __launch_bounds__(256, kRotate ? 3 : 4) quantize_qk_kernel(const
             fwht_stage_pairs<16>(w);
 #pragma unroll
             for (int m = 1; m <= 2; m <<= 1) {  // strides 32 and 64: the row's other lanes
-                const bool upper = (g & m) != 0;
+                // The upper lane keeps o - w, the lower one w + o: one fused
+                // s * w + o with s = -1 or +1, which rounds exactly as the
+                // subtraction or the addition does.
+                const float s = (g & m) != 0 ? -1.f : 1.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, w[i].x, m),
                                                  __shfl_xor_sync(0xffffffffu, w[i].y, m));
-                    w[i] = upper ? fsub2(o, w[i]) : fadd2(w[i], o);
+                    w[i] = ffma2(make_float2(s, s), w[i], o);
                 }
             }
             constexpr float kRsqrt128 = 0x1.6a09e6p-4f;
@@ -121,20 +124,19 @@ __global__ void __launch_bounds__(256, kRotate ? 3 : 4) quantize_qk_kernel(const
         for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fmaxf(fabsf(w[i].x), fabsf(w[i].y)));
         const int X = shared_exponent(amax, 2);
         const float f = pow2_neg(X);
+        // x / 2^X is exact (power-of-two scaling); the conversion rounds the
+        // magnitude and keeps the sign bit, also of a value that rounds to zero.
         uint32_t packed[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             float y[8];
-            uint32_t sign = 0;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 a = w[4 * q + e];
-                y[2 * e] = fabsf(a.x) * f;  // exact: power-of-two scaling
-                y[2 * e + 1] = fabsf(a.y) * f;
-                sign |= (__float_as_uint(a.x) >> 31) << (8 * e + 3);
-                sign |= (__float_as_uint(a.y) >> 31) << (8 * e + 7);
+                const float2 a = fmul2(w[4 * q + e], make_float2(f, f));
+                y[2 * e] = a.x;
+                y[2 * e + 1] = a.y;
             }
-            packed[q] = valid ? (cvt_e2m1x8(y) | sign) : 0u;
+            packed[q] = valid ? cvt_e2m1x8(y) : 0u;
         }
         if (in) {
             *reinterpret_cast<uint4 *>(codes + ((head_b + h) * cap + t) * 64 + g * 16) =
@@ -184,6 +186,35 @@ __device__ __forceinline__ void stage_v_tile(const __nv_bfloat16 *__restrict__ v
     __syncthreads();
 }
 
+// Encoder thread layout of both V kernels: thread (cp, g) = (threadIdx.x & 63,
+// threadIdx.x >> 6) takes channels 2cp and 2cp + 1 over the 32 tokens of group
+// g. One 32-bit shared load per token gives both channels (a warp reads 128
+// contiguous bytes of a staged row), and the registers then serve the amax and
+// the encode. The amax of both channels is one bf16x2 max chain: max is exact
+// in bf16, so it equals the fp32 amax.
+__device__ __forceinline__ void load_v_pair(const uint16_t *tile, int cp, int g, int emax, uint32_t (&w)[32],
+                                            int (&X)[2]) {
+    const uint32_t *t32 = reinterpret_cast<const uint32_t *>(tile);
+    __nv_bfloat162 m = __floats2bfloat162_rn(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        w[j] = t32[(g * 32 + j) * (kVPitch / 2) + cp];
+        m = __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j])));
+    }
+    const uint32_t mb = *reinterpret_cast<const uint32_t *>(&m);
+    X[0] = shared_exponent(__uint_as_float(mb << 16), emax);
+    X[1] = shared_exponent(__uint_as_float(mb & 0xFFFF0000u), emax);
+}
+
+// bf16 channel k (0: low half, 1: high half) of a staged word as fp32, exact.
+__device__ __forceinline__ float v_chan(uint32_t w, int k) {
+    return __uint_as_float(k ? (w & 0xFFFF0000u) : (w << 16));
+}
+
+// Staged code rows: channel 2cp at row cp, channel 2cp + 1 at row 64 + cp, so
+// the 32 threads of a warp store to consecutive rows.
+__device__ __forceinline__ int v_code_row(int channel) { return (channel >> 1) + (channel & 1) * 64; }
+
 __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__restrict__ v, int B, int S, int H,
                                                          int64_t sb, int64_t ss, int64_t sh,
                                                          const int32_t *__restrict__ seqlens, int cap,
@@ -191,7 +222,7 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__
                                                          uint8_t *__restrict__ scales) {
     __shared__ __align__(16) uint16_t tile[128 * kVPitch];  // bf16 staging, later the code tile
     __shared__ __align__(16) uint8_t atom[512];
-    uint8_t *ctile = reinterpret_cast<uint8_t *>(tile);     // [128 channels][kCPitch] after the barrier
+    uint8_t *ctile = reinterpret_cast<uint8_t *>(tile);     // [128 code rows][kCPitch] after the barrier
     const int nblk = cap / 128;
     const int blk = blockIdx.x % nblk;
     const int h = (blockIdx.x / nblk) % H;
@@ -205,52 +236,39 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__
     // Stage: invalid tokens read as zeros, which leaves them out of every amax
     // and gives them code 0; a group with no valid token gets scale byte 0.
     stage_v_tile(v, b, h, t0, valid_len, sb, ss, sh, tile);
-    const int c = threadIdx.x & 127;
-    const int g0 = threadIdx.x >> 7;
+    const int cp = threadIdx.x & 63;
+    const int g = threadIdx.x >> 6;
+    uint32_t w[32];
+    int X[2];
+    load_v_pair(tile, cp, g, 8, w, X);
+    // x / 2^X is exact (power-of-two scaling); the conversion rounds the
+    // magnitude and keeps the sign bit, also of a value that rounds to zero.
     uint32_t words[2][8];
-    int Xs[2];
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi) {
-        const int g = g0 + 2 * gi;
-        float amax = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < 32; ++j)
-            amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(tile[(g * 32 + j) * kVPitch + c]) << 16)));
-        const int X = shared_exponent(amax, 8);
-        Xs[gi] = X;
-        const float f = pow2_neg(X);
+    for (int k = 0; k < 2; ++k) {
+        const float f = pow2_neg(X[k]);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int e = 0; e < 4; e += 2) {
-                const uint32_t b0 = tile[(g * 32 + 4 * q + e) * kVPitch + c];
-                const uint32_t b1 = tile[(g * 32 + 4 * q + e + 1) * kVPitch + c];
-                const float y0 = fabsf(__uint_as_float(b0 << 16)) * f;
-                const float y1 = fabsf(__uint_as_float(b1 << 16)) * f;
-                uint32_t pair = cvt_e4m3x2(y0, y1);
-                pair |= ((b0 >> 15) & 1u) << 7;
-                pair |= ((b1 >> 15) & 1u) << 15;
-                word |= pair << (8 * e);
-            }
-            words[gi][q] = word;
+            const uint32_t a = cvt_e4m3x2(v_chan(w[4 * q], k) * f, v_chan(w[4 * q + 1], k) * f);
+            const uint32_t c = cvt_e4m3x2(v_chan(w[4 * q + 2], k) * f, v_chan(w[4 * q + 3], k) * f);
+            words[k][q] = a | (c << 16);
         }
     }
     __syncthreads();  // every read of the bf16 staging is done before it is overwritten
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi) {
-        const int g = g0 + 2 * gi;
-        uint4 *dst = reinterpret_cast<uint4 *>(&ctile[c * kCPitch + g * 32]);
-        dst[0] = make_uint4(words[gi][0], words[gi][1], words[gi][2], words[gi][3]);
-        dst[1] = make_uint4(words[gi][4], words[gi][5], words[gi][6], words[gi][7]);
-        atom[(c & 31) * 16 + (c >> 5) * 4 + g] = static_cast<uint8_t>(Xs[gi] + 127);
+    for (int k = 0; k < 2; ++k) {
+        const int c = 2 * cp + k;
+        uint4 *dst = reinterpret_cast<uint4 *>(&ctile[v_code_row(c) * kCPitch + g * 32]);
+        dst[0] = make_uint4(words[k][0], words[k][1], words[k][2], words[k][3]);
+        dst[1] = make_uint4(words[k][4], words[k][5], words[k][6], words[k][7]);
+        atom[(c & 31) * 16 + (c >> 5) * 4 + g] = static_cast<uint8_t>(X[k] + 127);
     }
     __syncthreads();
     const int64_t head = static_cast<int64_t>(b) * H + h;
     for (int i = threadIdx.x; i < 128 * 8; i += 256) {
         const int row = i >> 3, ch = i & 7;
         *reinterpret_cast<uint4 *>(codes + (head * 128 + row) * cap + t0 + ch * 16) =
-            *reinterpret_cast<const uint4 *>(&ctile[row * kCPitch + ch * 16]);
+            *reinterpret_cast<const uint4 *>(&ctile[v_code_row(row) * kCPitch + ch * 16]);
     }
     if (threadIdx.x < 32)
         reinterpret_cast<uint4 *>(scales + (head * nblk + blk) * 512)[threadIdx.x] =
@@ -261,9 +279,9 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__
 
 // The QK4V4 comparison point (MpFA article, sections 2.2 and 5.3): V in MXFP4,
 // groups of 32 along the token axis like the MXFP8 V. Same staging as
-// quantize_v_kernel; each thread encodes one channel's 32-token group to 16
-// bytes of packed E2M1 (even token in the low nibble), and the 128-token tile of
-// a channel row is 64 bytes of codes [B][H][128][cap / 2].
+// quantize_v_kernel; each thread encodes the 32-token group of two channels to
+// 16 bytes of packed E2M1 each (even token in the low nibble), and the
+// 128-token tile of a channel row is 64 bytes of codes [B][H][128][cap / 2].
 constexpr int kC4Pitch = 80;  // bytes per staged code row (64 + 16 padding)
 
 __global__ void __launch_bounds__(256) quantize_v4_kernel(const __nv_bfloat16 *__restrict__ v, int B, int S, int H,
@@ -273,7 +291,7 @@ __global__ void __launch_bounds__(256) quantize_v4_kernel(const __nv_bfloat16 *_
                                                           uint8_t *__restrict__ scales) {
     __shared__ __align__(16) uint16_t tile[128 * kVPitch];
     __shared__ __align__(16) uint8_t atom[512];
-    uint8_t *ctile = reinterpret_cast<uint8_t *>(tile);  // [128 channels][kC4Pitch] after the barrier
+    uint8_t *ctile = reinterpret_cast<uint8_t *>(tile);  // [128 code rows][kC4Pitch] after the barrier
     const int nblk = cap / 128;
     const int blk = blockIdx.x % nblk;
     const int h = (blockIdx.x / nblk) % H;
@@ -285,47 +303,37 @@ __global__ void __launch_bounds__(256) quantize_v4_kernel(const __nv_bfloat16 *_
         valid_len = L < valid_len ? L : valid_len;
     }
     stage_v_tile(v, b, h, t0, valid_len, sb, ss, sh, tile);
-    const int c = threadIdx.x & 127;
-    const int g0 = threadIdx.x >> 7;
+    const int cp = threadIdx.x & 63;
+    const int g = threadIdx.x >> 6;
+    uint32_t w[32];
+    int X[2];
+    load_v_pair(tile, cp, g, 2, w, X);
     uint32_t words[2][4];
-    int Xs[2];
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi) {
-        const int g = g0 + 2 * gi;
-        float amax = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < 32; ++j)
-            amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(tile[(g * 32 + j) * kVPitch + c]) << 16)));
-        const int X = shared_exponent(amax, 2);
-        Xs[gi] = X;
-        const float f = pow2_neg(X);
+    for (int k = 0; k < 2; ++k) {
+        const float f = pow2_neg(X[k]);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             float y[8];
-            uint32_t sign = 0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const uint32_t bits = tile[(g * 32 + 8 * q + e) * kVPitch + c];
-                y[e] = fabsf(__uint_as_float(bits << 16)) * f;
-                sign |= ((bits >> 15) & 1u) << (4 * e + 3);
-            }
-            words[gi][q] = cvt_e2m1x8(y) | sign;
+            for (int e = 0; e < 8; ++e) y[e] = v_chan(w[8 * q + e], k) * f;
+            words[k][q] = cvt_e2m1x8(y);
         }
     }
     __syncthreads();  // every read of the bf16 staging is done before it is overwritten
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi) {
-        const int g = g0 + 2 * gi;
-        *reinterpret_cast<uint4 *>(&ctile[c * kC4Pitch + g * 16]) =
-            make_uint4(words[gi][0], words[gi][1], words[gi][2], words[gi][3]);
-        atom[(c & 31) * 16 + (c >> 5) * 4 + g] = static_cast<uint8_t>(Xs[gi] + 127);
+    for (int k = 0; k < 2; ++k) {
+        const int c = 2 * cp + k;
+        *reinterpret_cast<uint4 *>(&ctile[v_code_row(c) * kC4Pitch + g * 16]) =
+            make_uint4(words[k][0], words[k][1], words[k][2], words[k][3]);
+        atom[(c & 31) * 16 + (c >> 5) * 4 + g] = static_cast<uint8_t>(X[k] + 127);
     }
     __syncthreads();
     const int64_t head = static_cast<int64_t>(b) * H + h;
     for (int i = threadIdx.x; i < 128 * 4; i += 256) {
         const int row = i >> 2, ch = i & 3;
         *reinterpret_cast<uint4 *>(codes + (head * 128 + row) * (cap / 2) + t0 / 2 + ch * 16) =
-            *reinterpret_cast<const uint4 *>(&ctile[row * kC4Pitch + ch * 16]);
+            *reinterpret_cast<const uint4 *>(&ctile[v_code_row(row) * kC4Pitch + ch * 16]);
     }
     if (threadIdx.x < 32)
         reinterpret_cast<uint4 *>(scales + (head * nblk + blk) * 512)[threadIdx.x] =
