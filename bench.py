@@ -560,10 +560,11 @@ def run_paged(gen, steps, hbm_gbs):
     torch.cuda.synchronize()
     equal = bool(torch.equal(out, ref))
     kv_bytes = wl.B * wl.Hkv * wl.Lk * KV_BYTES_PER_TOKEN_HEAD
-    # Append: one new token per sequence, 64 steps (the last page has room).
+    # Append: one new token per sequence, 32 calls from Python, then 32 more as
+    # one CUDA graph (the last page has room for 128 tokens).
     knew = k[:, :1].contiguous()
     vnew = v[:, :1].contiguous()
-    n_app = 64
+    n_app = 32
     stream = torch.cuda.current_stream()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a0.record(stream)
@@ -572,12 +573,24 @@ def run_paged(gen, steps, hbm_gbs):
     a1.record(stream)
     torch.cuda.synchronize()
     app_us = a0.elapsed_time(a1) / n_app * 1e3
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(n_app):
+            qk.kv_append(cache, knew, vnew)
+    torch.cuda.synchronize()
+    a0.record(stream)
+    g.replay()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    app_graph_us = a0.elapsed_time(a1) / n_app * 1e3
+    del g
     gbs = kv_bytes / (ms * 1e-3) / 1e9
     return {"workload": DECODE_WORKLOAD + " (paged, 128-token pages in random order)", "ms_per_step": ms,
             "value": gbs, "unit": "GB/s", "roofline_frac": gbs / hbm_gbs, "steps": steps,
             "kernel": "qk4v8_decode_kernel<16,4,4,3,2,true> (paged instance)",
-            "output_equals_contiguous": equal, "append_us_per_call": app_us,
-            "append_call": "qk4v8_kv_append of 1 token to 32 sequences x 8 KV heads (4 launches, not in a graph)"}
+            "output_equals_contiguous": equal, "append_us_per_call": app_us, "append_us_per_call_graph": app_graph_us,
+            "append_call": "qk4v8_kv_append of 1 token to 32 sequences x 8 KV heads: the fused append kernel and "
+                           "the in-place length update (2 launches); per call from Python, and inside a CUDA graph"}
 
 
 def run_draft_block(gen, hbm_gbs, window=1024, reps=20):

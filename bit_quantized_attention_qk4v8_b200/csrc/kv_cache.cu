@@ -52,29 +52,52 @@ __device__ __forceinline__ int page_of(const int32_t *__restrict__ block_table, 
 
 }  // namespace
 
-// K rows: 16 lanes per (sequence, new token, head) row, two rows per warp step,
-// the encoder of the quantization kernels (identical bytes), optionally after
-// the Hadamard rotation of the row.
+// One kernel does the whole append. CTA (b, h, chunk), 128 threads:
+//  - K: the chunk's share of the n_new rows of head h, 16 lanes per row (two
+//    rows per warp step), with the quantization kernels' encoder (identical
+//    bytes), optionally after the Hadamard rotation of the row;
+//  - V: thread c = channel c; the chunk's share of the 32-token groups the new
+//    tokens touch. A group's tokens come from the staging buffer (those before
+//    the append, only in the first touched group) and from the new rows; the
+//    channel's amax over them fixes the E8M0 scale, all of the group's codes
+//    are (re)written, and codes past the new length are zero;
+//  - chunk 0 then refreshes the staging buffer with the open group after the
+//    append. It is also the only reader of the old staging (the first touched
+//    group is its own), and thread c reads and writes only column c, so the
+//    refresh needs no barrier;
+//  - with a separate seqlens_out, CTA (b, 0, 0) writes the new length (no CTA
+//    reads seqlens_out). When the two are the same array, a second launch
+//    advances the lengths after every reader.
 template <bool kRotate>
-__global__ void __launch_bounds__(256) kv_append_k_kernel(const __nv_bfloat16 *__restrict__ k, int B, int n_new,
-                                                          int H, int64_t sb, int64_t st, int64_t sh,
-                                                          const int32_t *__restrict__ seqlens,
-                                                          const int32_t *__restrict__ block_table, int max_pages,
-                                                          int num_pages, uint8_t *__restrict__ codes,
-                                                          uint8_t *__restrict__ scales, int32_t *status) {
-    const int sub = threadIdx.x & 15;
-    const int64_t rows = static_cast<int64_t>(B) * n_new * H;
-    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-    for (int64_t base = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 2;
-         base < rows; base += 2 * warps) {
-        const int64_t r = base + ((threadIdx.x >> 4) & 1);
-        const bool in = r < rows;
-        int b = 0, t = 0, h = 0, page = -1, pos = 0;
+__global__ void __launch_bounds__(128) kv_append_kernel(const __nv_bfloat16 *__restrict__ k,
+                                                        const __nv_bfloat16 *__restrict__ v, int n_new, int H,
+                                                        int64_t sb, int64_t st, int64_t sh,
+                                                        const int32_t *__restrict__ seqlens,
+                                                        const int32_t *__restrict__ block_table, int max_pages,
+                                                        int num_pages, uint8_t *__restrict__ k_codes,
+                                                        uint8_t *__restrict__ k_scales, uint8_t *__restrict__ v_codes,
+                                                        uint8_t *__restrict__ v_scales, __nv_bfloat16 *__restrict__ tail,
+                                                        int chunks, int32_t *seqlens_out, int32_t *status) {
+    const int ci = static_cast<int>(blockIdx.x % chunks);
+    const int h = static_cast<int>((blockIdx.x / chunks) % H);
+    const int b = static_cast<int>(blockIdx.x / (static_cast<int64_t>(chunks) * H));
+    const int L0 = seqlens[b];
+    const int L1 = L0 + n_new;
+    const int c = threadIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    // ---- K rows [r_begin, r_end) of this chunk
+    const int rows_per_chunk = (n_new + chunks - 1) / chunks;
+    const int r_begin = ci * rows_per_chunk;
+    const int r_end = r_begin + rows_per_chunk < n_new ? r_begin + rows_per_chunk : n_new;
+    const int sub = lane & 15;
+    // The loop bound is per warp, so all 32 lanes reach the encoder's shuffles.
+    for (int r0 = r_begin + 2 * warp; r0 < r_end; r0 += 8) {
+        const int t = r0 + (lane >> 4);
+        const bool in = t < r_end;
+        const int pos = L0 + t;
+        int page = -1;
         if (in) {
-            h = static_cast<int>(r % H);
-            t = static_cast<int>((r / H) % n_new);
-            b = static_cast<int>(r / (static_cast<int64_t>(H) * n_new));
-            pos = seqlens[b] + t;
             page = page_of(block_table, max_pages, num_pages, b, pos);
             if (page < 0 && sub == 0) flag_bad_page(status);
         }
@@ -84,121 +107,82 @@ __global__ void __launch_bounds__(256) kv_append_k_kernel(const __nv_bfloat16 *_
         uint32_t packed;
         if (kRotate) {
             const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-            float v[8];
+            float x[8];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                v[2 * i] = __uint_as_float(w[i] << 16);
-                v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+                x[2 * i] = __uint_as_float(w[i] << 16);
+                x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
             }
-            hadamard128_rows(v, sub);
-            packed = mxfp4_encode8_f32(v, true, X);
+            hadamard128_rows(x, sub);
+            packed = mxfp4_encode8_f32(x, true, X);
         } else {
             packed = mxfp4_encode8(raw, true, X);
         }
         if (page >= 0) {
             const int64_t row = static_cast<int64_t>(page) * H + h;
             const int rr = pos & 127;
-            reinterpret_cast<uint32_t *>(codes + (row * 128 + rr) * 64)[sub] = packed;
+            reinterpret_cast<uint32_t *>(k_codes + (row * 128 + rr) * 64)[sub] = packed;
             if ((sub & 3) == 0)
-                scales[row * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (sub >> 2)] = static_cast<uint8_t>(X + 127);
+                k_scales[row * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (sub >> 2)] = static_cast<uint8_t>(X + 127);
         }
     }
-}
 
-// V: one CTA of 128 threads (one per channel) per (sequence, head, touched
-// 32-token group). The group's tokens come from the staging buffer (those
-// before the append) and from the new rows; the channel's amax over them
-// fixes the E8M0 scale, all of the group's codes are (re)written, and codes
-// past the new length are zero. The staging buffer is refreshed afterwards by
-// kv_tail_update_kernel (a separate launch: the CTA of the first group reads
-// slots that the last group's new tokens take).
-__global__ void __launch_bounds__(128) kv_append_v_kernel(const __nv_bfloat16 *__restrict__ v, int B, int n_new,
-                                                          int H, int64_t sb, int64_t st, int64_t sh,
-                                                          const int32_t *__restrict__ seqlens,
-                                                          const int32_t *__restrict__ block_table, int max_pages,
-                                                          int num_pages, uint8_t *__restrict__ codes,
-                                                          uint8_t *__restrict__ scales,
-                                                          const __nv_bfloat16 *__restrict__ tail, int groups_per_seq,
-                                                          int32_t *status) {
-    const int c = threadIdx.x;
-    const int gi = static_cast<int>(blockIdx.x % groups_per_seq);
-    const int h = static_cast<int>((blockIdx.x / groups_per_seq) % H);
-    const int b = static_cast<int>(blockIdx.x / (static_cast<int64_t>(groups_per_seq) * H));
-    const int L0 = seqlens[b];
-    const int L1 = L0 + n_new;
-    const int G = L0 / 32 + gi;       // the group this CTA writes
-    if (G * 32 >= L1) return;         // fewer groups touched than the grid allows for
-    const int t0 = G * 32;
-    const int page = page_of(block_table, max_pages, num_pages, b, t0);
-    if (page < 0) {
-        if (c == 0) flag_bad_page(status);
-        return;
-    }
-    const __nv_bfloat16 *tail_bh = tail + ((static_cast<int64_t>(b) * H + h) * 32) * 128;
-    const uint16_t *vin = reinterpret_cast<const uint16_t *>(v) + b * sb + h * sh + c;
-    uint16_t x[32];
-    float amax = 0.f;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const int t = t0 + j;
-        uint16_t bits = 0;
-        if (t < L0)
-            bits = reinterpret_cast<const uint16_t *>(tail_bh)[j * 128 + c];   // staged before this append
-        else if (t < L1)
-            bits = vin[(t - L0) * st];
-        x[j] = bits;
-        amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(bits) << 16)));
-    }
-    const int X = shared_exponent(amax, 8);
-    const float f = pow2_neg(X);
-    uint32_t words[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < 4; e += 2) {
-            const uint32_t b0 = x[4 * q + e], b1 = x[4 * q + e + 1];
-            uint32_t pair = cvt_e4m3x2(fabsf(__uint_as_float(b0 << 16)) * f, fabsf(__uint_as_float(b1 << 16)) * f);
-            pair |= ((b0 >> 15) & 1u) << 7;
-            pair |= ((b1 >> 15) & 1u) << 15;
-            word |= pair << (8 * e);
-        }
-        words[q] = word;
-    }
-    // Tokens past L1 encode as zero (their inputs were zero, and a zero keeps
-    // code 0 whatever the scale).
-    const int64_t row = static_cast<int64_t>(page) * H + h;
-    uint4 *dst = reinterpret_cast<uint4 *>(codes + (row * 128 + c) * 128 + (t0 & 127));
-    dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-    dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
-    scales[row * 512 + (c & 31) * 16 + (c >> 5) * 4 + ((t0 >> 5) & 3)] = static_cast<uint8_t>(X + 127);
-}
-
-// The open group after the append (tokens 32 * (L1 / 32) .. L1 - 1), staged in
-// slots t % 32: its tokens from before the append are in place already; the
-// new ones are copied in. One CTA of 128 threads (channels) per (sequence,
-// head).
-__global__ void __launch_bounds__(128) kv_tail_update_kernel(const __nv_bfloat16 *__restrict__ v, int n_new, int H,
-                                                             int64_t sb, int64_t st, int64_t sh,
-                                                             const int32_t *__restrict__ seqlens,
-                                                             __nv_bfloat16 *__restrict__ tail) {
-    const int c = threadIdx.x;
-    const int h = static_cast<int>(blockIdx.x % H);
-    const int b = static_cast<int>(blockIdx.x / H);
-    const int L0 = seqlens[b];
-    const int L1 = L0 + n_new;
-    if ((L1 & 31) == 0) return;  // no open group
-    const int t0 = L1 & ~31;
+    // ---- V groups L0 / 32 + ci, + chunks, ... touched by the new tokens
     uint16_t *tail_bh = reinterpret_cast<uint16_t *>(tail) + ((static_cast<int64_t>(b) * H + h) * 32) * 128;
     const uint16_t *vin = reinterpret_cast<const uint16_t *>(v) + b * sb + h * sh + c;
-    for (int t = t0 > L0 ? t0 : L0; t < L1; ++t) tail_bh[(t - t0) * 128 + c] = vin[(t - L0) * st];
+    for (int G = L0 / 32 + ci; G * 32 < L1; G += chunks) {
+        const int t0 = G * 32;
+        const int page = page_of(block_table, max_pages, num_pages, b, t0);
+        if (page < 0) {
+            if (c == 0) flag_bad_page(status);
+            continue;
+        }
+        uint16_t x[32];
+        float amax = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int t = t0 + j;
+            uint16_t bits = 0;
+            if (t < L0)
+                bits = tail_bh[j * 128 + c];  // staged before this append
+            else if (t < L1)
+                bits = vin[(t - L0) * st];
+            x[j] = bits;
+            amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(bits) << 16)));
+        }
+        const int X = shared_exponent(amax, 8);
+        const float f = pow2_neg(X);
+        // x / 2^X is exact; the conversion keeps the sign bit, also of a value
+        // that rounds to zero. Tokens past L1 encode as zero.
+        uint32_t words[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const uint32_t lo = cvt_e4m3x2(__uint_as_float(static_cast<uint32_t>(x[4 * q]) << 16) * f,
+                                           __uint_as_float(static_cast<uint32_t>(x[4 * q + 1]) << 16) * f);
+            const uint32_t hi = cvt_e4m3x2(__uint_as_float(static_cast<uint32_t>(x[4 * q + 2]) << 16) * f,
+                                           __uint_as_float(static_cast<uint32_t>(x[4 * q + 3]) << 16) * f);
+            words[q] = lo | (hi << 16);
+        }
+        const int64_t row = static_cast<int64_t>(page) * H + h;
+        uint4 *dst = reinterpret_cast<uint4 *>(v_codes + (row * 128 + c) * 128 + (t0 & 127));
+        dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+        dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+        v_scales[row * 512 + (c & 31) * 16 + (c >> 5) * 4 + ((t0 >> 5) & 3)] = static_cast<uint8_t>(X + 127);
+    }
+
+    // ---- the open group after the append, staged in slots t % 32 (its tokens
+    // from before the append are in place already)
+    if (ci == 0 && (L1 & 31) != 0) {
+        const int t0 = L1 & ~31;
+        for (int t = t0 > L0 ? t0 : L0; t < L1; ++t) tail_bh[(t - t0) * 128 + c] = vin[(t - L0) * st];
+    }
+    if (seqlens_out && ci == 0 && h == 0 && c == 0) seqlens_out[b] = L1;
 }
 
-// seqlens_out[b] = seqlens[b] + n_new, after every reader of seqlens ran (the
-// two may be the same array).
-__global__ void kv_advance_lengths_kernel(const int32_t *seqlens, int B, int n_new, int32_t *seqlens_out) {
+// seqlens[b] += n_new in place, after every reader of seqlens ran.
+__global__ void kv_advance_lengths_kernel(int32_t *seqlens, int B, int n_new) {
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b < B) seqlens_out[b] = seqlens[b] + n_new;
+    if (b < B) seqlens[b] += n_new;
 }
 
 cudaError_t launch_kv_append(const void *k, const void *v, int B, int n_new, int H, int64_t sb, int64_t st,
@@ -206,32 +190,30 @@ cudaError_t launch_kv_append(const void *k, const void *v, int B, int n_new, int
                              int num_pages, uint8_t *k_codes, uint8_t *k_scales, uint8_t *v_codes,
                              uint8_t *v_scales, void *tail, bool rotate_k, int32_t *seqlens_out, int32_t *status,
                              cudaStream_t stream) {
-    const int64_t rows = static_cast<int64_t>(B) * n_new * H;
-    int64_t grid_k = (rows + 15) / 16;  // 16 rows per CTA (8 warps, two rows each)
-    if (grid_k > 148 * 8) grid_k = 148 * 8;
-    if (grid_k < 1) grid_k = 1;
+    // Chunks per (sequence, head): at most 8 touched V groups and 256 K rows
+    // per CTA (one chunk for a decode step of up to 32 tokens).
+    const int groups = (n_new + 31) / 32 + 1;  // the open group and those the new tokens fill
+    int chunks = (groups + 7) / 8;
+    const int chunks_k = (n_new + 255) / 256;
+    if (chunks_k > chunks) chunks = chunks_k;
+    const int64_t grid = static_cast<int64_t>(B) * H * chunks;
+    if (grid >= (int64_t{1} << 31)) return cudaErrorInvalidValue;
+    const bool in_place = seqlens_out && seqlens_out == seqlens;
+    int32_t *direct_out = in_place ? nullptr : seqlens_out;
     const __nv_bfloat16 *kk = static_cast<const __nv_bfloat16 *>(k);
+    const __nv_bfloat16 *vv = static_cast<const __nv_bfloat16 *>(v);
+    __nv_bfloat16 *tl = static_cast<__nv_bfloat16 *>(tail);
     if (rotate_k)
-        kv_append_k_kernel<true><<<static_cast<unsigned>(grid_k), 256, 0, stream>>>(
-            kk, B, n_new, H, sb, st, sh, seqlens, block_table, max_pages, num_pages, k_codes, k_scales, status);
+        kv_append_kernel<true><<<static_cast<unsigned>(grid), 128, 0, stream>>>(
+            kk, vv, n_new, H, sb, st, sh, seqlens, block_table, max_pages, num_pages, k_codes, k_scales, v_codes,
+            v_scales, tl, chunks, direct_out, status);
     else
-        kv_append_k_kernel<false><<<static_cast<unsigned>(grid_k), 256, 0, stream>>>(
-            kk, B, n_new, H, sb, st, sh, seqlens, block_table, max_pages, num_pages, k_codes, k_scales, status);
+        kv_append_kernel<false><<<static_cast<unsigned>(grid), 128, 0, stream>>>(
+            kk, vv, n_new, H, sb, st, sh, seqlens, block_table, max_pages, num_pages, k_codes, k_scales, v_codes,
+            v_scales, tl, chunks, direct_out, status);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    // Groups one append can touch: the open one and those the new tokens fill.
-    const int groups = (n_new + 31) / 32 + 1;
-    const int64_t grid_v = static_cast<int64_t>(B) * H * groups;
-    kv_append_v_kernel<<<static_cast<unsigned>(grid_v), 128, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(v), B, n_new, H, sb, st, sh, seqlens, block_table, max_pages, num_pages,
-        v_codes, v_scales, static_cast<const __nv_bfloat16 *>(tail), groups, status);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    kv_tail_update_kernel<<<static_cast<unsigned>(static_cast<int64_t>(B) * H), 128, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(v), n_new, H, sb, st, sh, seqlens, static_cast<__nv_bfloat16 *>(tail));
-    e = cudaGetLastError();
-    if (e != cudaSuccess || !seqlens_out) return e;
-    kv_advance_lengths_kernel<<<(B + 255) / 256, 256, 0, stream>>>(seqlens, B, n_new, seqlens_out);
+    if (e != cudaSuccess || !in_place) return e;
+    kv_advance_lengths_kernel<<<(B + 255) / 256, 256, 0, stream>>>(seqlens_out, B, n_new);
     return cudaGetLastError();
 }
 

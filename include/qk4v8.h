@@ -374,7 +374,8 @@ QK4V8_API int qk4v8_decode_plan_splits(int B, int Hq, int Hkv, int nq, const int
  * sequence. Build a sequence's cache by appending its prompt to an empty
  * sequence (seqlens 0, v_tail contents then unused). Codes of tokens past the
  * new length within the last V group are written as 0; other padding is left
- * as it was (the attention kernels ignore it). Four launches on `stream`.
+ * as it was (the attention kernels ignore it). One launch on `stream`, two when
+ * seqlens_out is seqlens (the in-place length update runs after every reader).
  *
  * qk4v8_attention_decode_paged / qk4v8_attention_decode_bf16_paged: the
  * decode calls (with the draft-block window) over such a pool, for up to 64

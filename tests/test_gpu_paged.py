@@ -87,6 +87,31 @@ def test_append_whole_prompt_then_tokens():
     _check_cache(cache, gen["k"], gen["v"], T)
 
 
+def test_append_with_separate_length_output():
+    """seqlens_out distinct from seqlens: the append kernel writes the new lengths
+    itself and leaves the input lengths as they were."""
+    from bit_quantized_attention_qk4v8_b200._lib import lib
+    B, Hkv, T = 3, 4, 70
+    gen = _inputs(B, T, Hkv, seed=23)
+    k, v = to_dev(gen["k"]), to_dev(gen["v"])
+    cache = qk.paged_kv(B, Hkv, 8, _block_table(B, 2, 8, 5))
+    qk.kv_append(cache, k[:, :45].contiguous(), v[:, :45].contiguous())
+    lens_out = torch.full((B,), -1, dtype=torch.int32, device="cuda")
+    kn, vn = k[:, 45:].contiguous(), v[:, 45:].contiguous()
+    st = lib().qk4v8_kv_append(kn.data_ptr(), vn.data_ptr(), B, T - 45, Hkv, 128, kn.stride(0), kn.stride(1),
+                               kn.stride(2), cache.seqlens.data_ptr(), lens_out.data_ptr(),
+                               cache.block_table.data_ptr(), cache.max_pages, cache.num_pages,
+                               cache.k_codes.data_ptr(), cache.k_scales.data_ptr(), cache.v_codes.data_ptr(),
+                               cache.v_scales.data_ptr(), cache.v_tail.data_ptr(), 0, None,
+                               torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    torch.cuda.synchronize()
+    assert cache.seqlens.cpu().tolist() == [45] * B
+    assert lens_out.cpu().tolist() == [T] * B
+    cache.seqlens.copy_(lens_out)
+    _check_cache(cache, gen["k"], gen["v"], T)
+
+
 def _paged_from_contiguous(kp, vp, max_pages, num_pages, seed):
     """A page pool holding the contiguous cache's blocks in a random page order."""
     B, H = kp.B, kp.H
