@@ -76,8 +76,7 @@ L2_BYTES = 126 * 2 ** 20
 # kernel, from its committed ncu capture; None until a capture of the kernel as
 # it stands exists.
 NCU_TRAFFIC = {
-    DECODE_WORKLOAD: (423657984, "profiles/decode_attention_b32_hq32_hkv8_l8192.md (dram read 419.77 MB + write "
-                                 "3.89 MB, qk4v8_decode_kernel<16,4,4,3,2,false>)"),
+    DECODE_WORKLOAD: None,
 }
 
 
@@ -255,9 +254,9 @@ def graph_time_ms(step, steps, warmup, stream):
 def decode_kernel_name(rows: int) -> str:
     """The split-KV kernel the library launches for `rows` = (Hq / Hkv) * nq query rows per KV head."""
     if rows <= 4:
-        return "qk4v8_decode_kernel<16,4,4,3,2> (swap-AB split-KV decode)"
+        return "qk4v8_decode_kernel<16,4,4,4,2> (swap-AB split-KV decode)"
     if rows <= 8:
-        return "qk4v8_decode_kernel<16,8,8,3,2> (swap-AB split-KV decode)"
+        return "qk4v8_decode_kernel<16,8,8,4,2> (swap-AB split-KV decode)"
     if rows <= 16:
         return "qk4v8_decode_kernel<16,16,16,3,2> (swap-AB split-KV decode)"
     if rows <= 32:
@@ -587,7 +586,7 @@ def run_paged(gen, steps, hbm_gbs):
     gbs = kv_bytes / (ms * 1e-3) / 1e9
     return {"workload": DECODE_WORKLOAD + " (paged, 128-token pages in random order)", "ms_per_step": ms,
             "value": gbs, "unit": "GB/s", "roofline_frac": gbs / hbm_gbs, "steps": steps,
-            "kernel": "qk4v8_decode_kernel<16,4,4,3,2,true> (paged instance)",
+            "kernel": "qk4v8_decode_kernel<16,4,4,4,2,true> (paged instance)",
             "output_equals_contiguous": equal, "append_us_per_call": app_us, "append_us_per_call_graph": app_graph_us,
             "append_call": "qk4v8_kv_append of 1 token to 32 sequences x 8 KV heads: the fused append kernel and "
                            "the in-place length update (2 launches); per call from Python, and inside a CUDA graph"}

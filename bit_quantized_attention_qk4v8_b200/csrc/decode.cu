@@ -46,7 +46,12 @@ constexpr float kTauD = 8.0f;      // a warp moves m once a score passes it by 2
 constexpr int kEMaxD = 64;         // largest offset e = m - m_O before O itself is rescaled
 constexpr float kMaxMoveD = 16777216.0f;  // cap on one move of m (binades), keeps it an exact integer
 // Stages of the G*nq <= 16 instantiation, small enough for two CTAs per SM.
-constexpr int kDecodeSmallStages = 3;
+// K/V stages of the instances for up to 8 and up to 16 query rows per KV head:
+// two CTAs per SM share its 228 KB (each CTA's dynamic shared memory plus the
+// 1 KB the hardware keeps per CTA), which leaves room for four stages up to 8
+// rows and three for 16.
+constexpr int kDecodeStages8 = 4, kDecodeStages16 = 3;
+constexpr int kSmemPerSm = 228 * 1024, kSmemReservedPerCta = 1024;
 constexpr uint32_t kPhiScaleWord = 0x7F7F7F7Fu;  // E8M0 2^0 for P_hi rows
 constexpr uint32_t kPloScaleWord = 0x7A7A7A7Au;  // E8M0 2^-5 for P_lo rows
 // Named barriers: one per column group (ids 1..4), and one over all softmax warps.
@@ -78,15 +83,18 @@ struct DecodeLayout {
     static constexpr int kSfK = kSfQ + 512;
     static constexpr int kSfV = kSfK + ST * 512;
     static constexpr int kSfP = kSfV + ST * 512;  // one P scale atom per P buffer
-    // Exchange buffers, each [column group][quarter][NC] 32-bit words.
-    static constexpr int kXmax = kSfP + 1024;  // first-tile row maxima
-    static constexpr int kXe = kXmax + 1024;    // offsets e, when O is rescaled
-    static constexpr int kLsum = kXe + 1024;    // epilogue row sums
-    static constexpr int kEsum = kLsum + 1024;  // epilogue offsets e
-    static constexpr int kLim = kEsum + 1024;   // [NT] int: exclusive key bound per query row
-    static constexpr int kVote = kLim + 256;    // [column group][tile parity][quarter] u32 vote words
-    static constexpr int kMneg = kVote + 128;   // [softmax warp][NC] float: -m of each row
-    static constexpr int kBar = kMneg + 1024;
+    // Exchange buffers, each [column group][quarter][NC] 32-bit words, and the
+    // row references [softmax warp][NC]: kSoftmaxWarps * NC words, in 128-byte
+    // units (the small instances fit four K/V stages beside a second CTA).
+    static constexpr int kRowBytes = (kSoftmaxWarps * NC * 4 + 127) / 128 * 128;
+    static constexpr int kXmax = kSfP + 1024;       // first-tile row maxima
+    static constexpr int kXe = kXmax + kRowBytes;   // offsets e, when O is rescaled
+    static constexpr int kLsum = kXe + kRowBytes;   // epilogue row sums
+    static constexpr int kEsum = kLsum + kRowBytes;  // epilogue offsets e
+    static constexpr int kLim = kEsum + kRowBytes;  // [NT] int: exclusive key bound per query row
+    static constexpr int kVote = kLim + (NT * 4 < 128 ? 128 : NT * 4);  // [column group][tile parity][quarter] u32 votes
+    static constexpr int kMneg = kVote + 128;       // [softmax warp][NC] float: -m of each row
+    static constexpr int kBar = kMneg + kRowBytes;
     // kv_full/empty per stage, q_full, patch, s_full x2, p_full x2, pv_done x2,
     // s_free x2,
     // o_final, vote x2 and e exchange per column group.
@@ -98,8 +106,8 @@ struct DecodeLayout {
     static constexpr uint32_t kColO = 2 * NT;
     static constexpr uint32_t kColSfQ = 4 * NT;
     static constexpr uint32_t kTmemCols = 4 * NT + 28 <= 128 ? 128 : (4 * NT + 28 <= 256 ? 256 : 512);
-    static_assert(kCG * 4 * NC * 4 <= 1024, "exchange buffers");
-    static_assert(kSoftmaxWarps * NC * 4 <= 1024 && kMneg % 16 == 0, "row references");
+    static_assert(kCG * 4 * NC * 4 <= kRowBytes, "exchange buffers");
+    static_assert(kSoftmaxWarps * NC * 4 <= kRowBytes && kMneg % 16 == 0, "row references");
     static_assert(NC <= 32 && NT <= 64, "one lane per row of a warp");
     static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
@@ -826,6 +834,7 @@ template <int NT, int RW, int NC, int ST, int MINB>
 static cudaError_t launch_nt(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, int grid,
                              cudaStream_t stream) {
     using Lay = DecodeLayout<NT, RW, NC, ST>;
+    static_assert(MINB * (Lay::kBytes + kSmemReservedPerCta) <= kSmemPerSm, "MINB CTAs per SM must fit");
     constexpr int kMaxDevices = 64;
     static bool configured[kMaxDevices] = {};
     int dev = 0;
@@ -850,9 +859,9 @@ static cudaError_t launch_nt(const CUtensorMap &tk, const CUtensorMap &tv, const
 cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, int grid,
                           cudaStream_t stream) {
     const int R = p.G * p.Sq;
-    if (R <= 4) return launch_nt<16, 4, 4, kDecodeSmallStages, 2>(tk, tv, p, grid, stream);
-    if (R <= 8) return launch_nt<16, 8, 8, kDecodeSmallStages, 2>(tk, tv, p, grid, stream);
-    if (R <= 16) return launch_nt<16, 16, 16, kDecodeSmallStages, 2>(tk, tv, p, grid, stream);
+    if (R <= 4) return launch_nt<16, 4, 4, kDecodeStages8, 2>(tk, tv, p, grid, stream);
+    if (R <= 8) return launch_nt<16, 8, 8, kDecodeStages8, 2>(tk, tv, p, grid, stream);
+    if (R <= 16) return launch_nt<16, 16, 16, kDecodeStages16, 2>(tk, tv, p, grid, stream);
     if (R <= 32) return launch_nt<32, 32, 16, 6, 1>(tk, tv, p, grid, stream);
     return launch_nt<64, 64, 16, 6, 1>(tk, tv, p, grid, stream);
 }
