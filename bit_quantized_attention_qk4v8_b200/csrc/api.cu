@@ -229,11 +229,15 @@ int qk4v8_quantize(const void *q, const void *k, const void *v, int B, int Sq, i
                    const int32_t *seqlens_k, int q_cap, int kv_cap, uint8_t *q_codes, uint8_t *q_scales,
                    uint8_t *k_codes, uint8_t *k_scales, uint8_t *v_codes, uint8_t *v_scales, void *stream) {
     const int64_t qs = static_cast<int64_t>(Hq) * 128, ks = static_cast<int64_t>(Hkv) * 128;
-    int st = qk4v8_quantize_qk(q, B, Sq, Hq, d, qs * Sq, qs, 128, nullptr, q_cap, q_codes, q_scales, stream);
+    int st = validate_quant_args(q, B, Sq, Hq, d, qs * Sq, qs, 128, q_cap, q_codes, q_scales);
+    if (!st) st = validate_quant_args(k, B, Sk, Hkv, d, ks * Sk, ks, 128, kv_cap, k_codes, k_scales);
+    if (!st) st = validate_quant_args(v, B, Sk, Hkv, d, ks * Sk, ks, 128, kv_cap, v_codes, v_scales);
     if (st) return st;
-    st = qk4v8_quantize_qk(k, B, Sk, Hkv, d, ks * Sk, ks, 128, seqlens_k, kv_cap, k_codes, k_scales, stream);
-    if (st) return st;
-    return qk4v8_quantize_v(v, B, Sk, Hkv, d, ks * Sk, ks, 128, seqlens_k, kv_cap, v_codes, v_scales, stream);
+    if ((st = check_device())) return st;
+    cudaError_t e = qk4v8::launch_quantize_qkv(q, k, v, B, Sq, Sk, Hq, Hkv, seqlens_k, q_cap, kv_cap, q_codes,
+                                               q_scales, k_codes, k_scales, v_codes, v_scales,
+                                               static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QK4V8_OK : cuda_error(e, "quantize (Q, K, V) launch");
 }
 
 }  // extern "C"

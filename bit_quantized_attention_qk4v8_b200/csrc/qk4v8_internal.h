@@ -65,6 +65,10 @@ cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, i
 cudaError_t launch_quantize_v(const void *v, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                               const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
                               cudaStream_t stream);
+cudaError_t launch_quantize_qkv(const void *q, const void *k, const void *v, int B, int Sq, int Sk, int Hq, int Hkv,
+                                const int32_t *seqlens_k, int q_cap, int kv_cap, uint8_t *q_codes, uint8_t *q_scales,
+                                uint8_t *k_codes, uint8_t *k_scales, uint8_t *v_codes, uint8_t *v_scales,
+                                cudaStream_t stream);
 cudaError_t launch_quantize_v4(const void *v, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                                const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
                                cudaStream_t stream);

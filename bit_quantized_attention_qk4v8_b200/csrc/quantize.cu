@@ -50,25 +50,25 @@ __device__ __forceinline__ void fwht_stage_pairs(float2 (&w)[16]) {
     }
 }
 
+// Rows of batch entry b taken by CTA bx of the gx CTAs that share the entry
+// (the body of quantize_qk_kernel, also run by quantize_qkv_kernel).
 template <bool kRotate>
-__global__ void __launch_bounds__(256, kRotate ? 3 : 4) quantize_qk_kernel(const __nv_bfloat16 *__restrict__ x, int B, int S, int H,
-                                                          int64_t sb, int64_t ss, int64_t sh,
-                                                          const int32_t *__restrict__ seqlens, int cap,
-                                                          int row_len, uint8_t *__restrict__ codes,
-                                                          uint8_t *__restrict__ scales) {
+__device__ __forceinline__ void qk_rows(const __nv_bfloat16 *__restrict__ x, int S, int H, int64_t sb, int64_t ss,
+                                        int64_t sh, const int32_t *__restrict__ seqlens, int cap, int row_len,
+                                        uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int b, int bx,
+                                        int gx) {
     const int lane = threadIdx.x & 31;
     const int g = lane & 3;   // MX group (channels 32g .. 32g+31) of this lane
-    const int b = blockIdx.y;
     const int rows = row_len * H;  // rows of this batch entry (the launcher keeps this below 2^30)
     int valid_len = S;
     if (seqlens) {
         const int L = seqlens[b];
         valid_len = L < valid_len ? L : valid_len;
     }
-    const int step = static_cast<int>(gridDim.x) * (blockDim.x >> 5) * 8;  // rows per grid step
+    const int step = gx * (blockDim.x >> 5) * 8;  // rows per grid step
     const int step_t = step / H, step_h = step - step_t * H;
     // The loop bound is taken per warp (8 rows) so every lane reaches the shuffles.
-    int base = (static_cast<int>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 8;
+    int base = (bx * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 8;
     int t = (base + (lane >> 2)) / H;
     int h = (base + (lane >> 2)) - t * H;
     const __nv_bfloat16 *xb = x + b * sb;
@@ -153,6 +153,17 @@ __global__ void __launch_bounds__(256, kRotate ? 3 : 4) quantize_qk_kernel(const
     }
 }
 
+template <bool kRotate>
+__global__ void __launch_bounds__(256, kRotate ? 3 : 4) quantize_qk_kernel(const __nv_bfloat16 *__restrict__ x, int S,
+                                                                           int H, int64_t sb, int64_t ss, int64_t sh,
+                                                                           const int32_t *__restrict__ seqlens,
+                                                                           int cap, int row_len,
+                                                                           uint8_t *__restrict__ codes,
+                                                                           uint8_t *__restrict__ scales) {
+    qk_rows<kRotate>(x, S, H, sb, ss, sh, seqlens, cap, row_len, codes, scales, static_cast<int>(blockIdx.y),
+                     static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x));
+}
+
 // ------------------------------------------------------------------ MXFP8 V
 
 // One CTA per (b, h, 128-token block): stage the bf16 tile in shared memory,
@@ -215,18 +226,18 @@ __device__ __forceinline__ float v_chan(uint32_t w, int k) {
 // the 32 threads of a warp store to consecutive rows.
 __device__ __forceinline__ int v_code_row(int channel) { return (channel >> 1) + (channel & 1) * 64; }
 
-__global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__restrict__ v, int B, int S, int H,
-                                                         int64_t sb, int64_t ss, int64_t sh,
-                                                         const int32_t *__restrict__ seqlens, int cap,
-                                                         uint8_t *__restrict__ codes,
-                                                         uint8_t *__restrict__ scales) {
+// Tile `idx` = (b, h, 128-token block) of V (the body of quantize_v_kernel,
+// also run by quantize_qkv_kernel).
+__device__ __forceinline__ void v_tile(const __nv_bfloat16 *__restrict__ v, int S, int H, int64_t sb, int64_t ss,
+                                       int64_t sh, const int32_t *__restrict__ seqlens, int cap,
+                                       uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int idx) {
     __shared__ __align__(16) uint16_t tile[128 * kVPitch];  // bf16 staging, later the code tile
     __shared__ __align__(16) uint8_t atom[512];
     uint8_t *ctile = reinterpret_cast<uint8_t *>(tile);     // [128 code rows][kCPitch] after the barrier
     const int nblk = cap / 128;
-    const int blk = blockIdx.x % nblk;
-    const int h = (blockIdx.x / nblk) % H;
-    const int b = blockIdx.x / (nblk * H);
+    const int blk = idx % nblk;
+    const int h = (idx / nblk) % H;
+    const int b = idx / (nblk * H);
     const int t0 = blk * 128;
     int valid_len = S;
     if (seqlens) {
@@ -273,6 +284,46 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16 *__
     if (threadIdx.x < 32)
         reinterpret_cast<uint4 *>(scales + (head * nblk + blk) * 512)[threadIdx.x] =
             reinterpret_cast<const uint4 *>(atom)[threadIdx.x];
+}
+
+__global__ void __launch_bounds__(256, 5) quantize_v_kernel(const __nv_bfloat16 *__restrict__ v, int S, int H,
+                                                         int64_t sb, int64_t ss, int64_t sh,
+                                                         const int32_t *__restrict__ seqlens, int cap,
+                                                         uint8_t *__restrict__ codes,
+                                                         uint8_t *__restrict__ scales) {
+    v_tile(v, S, H, sb, ss, sh, seqlens, cap, codes, scales, static_cast<int>(blockIdx.x));
+}
+
+// ------------------------------------------------------------------ Q, K and V in one launch
+
+// CTAs [0, nq) quantize Q (gxq per batch entry), [nq, nq + nk) K (gxk per
+// entry), the rest V (one per (b, h, 128-token block)). Small prefills are
+// launch-bound: one launch instead of three. Every CTA carries the V staging
+// buffer (35 KB), which still allows the four CTAs per SM the registers allow.
+struct QkvArgs {
+    const __nv_bfloat16 *q, *k, *v;
+    int Sq, Sk, Hq, Hkv, q_cap, kv_cap;
+    int64_t qsb, qss, qsh, ksb, kss, ksh;
+    const int32_t *seqlens_k;
+    uint8_t *q_codes, *q_scales, *k_codes, *k_scales, *v_codes, *v_scales;
+    int gxq, gxk, nq, nk;
+};
+
+__global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QkvArgs a) {
+    int i = static_cast<int>(blockIdx.x);
+    if (i < a.nq) {
+        qk_rows<false>(a.q, a.Sq, a.Hq, a.qsb, a.qss, a.qsh, nullptr, a.q_cap, a.q_cap, a.q_codes, a.q_scales,
+                       i / a.gxq, i % a.gxq, a.gxq);
+        return;
+    }
+    i -= a.nq;
+    if (i < a.nk) {
+        qk_rows<false>(a.k, a.Sk, a.Hkv, a.ksb, a.kss, a.ksh, a.seqlens_k, a.kv_cap, a.kv_cap, a.k_codes,
+                       a.k_scales, i / a.gxk, i % a.gxk, a.gxk);
+        return;
+    }
+    i -= a.nk;
+    v_tile(a.v, a.Sk, a.Hkv, a.ksb, a.kss, a.ksh, a.seqlens_k, a.kv_cap, a.v_codes, a.v_scales, i);
 }
 
 // ------------------------------------------------------------------ MXFP4 V
@@ -349,19 +400,22 @@ cudaError_t launch_quantize_v4(const void *v, int B, int S, int H, int64_t sb, i
     return cudaGetLastError();
 }
 
+// CTAs per batch entry of the Q/K part: about one wave over all entries (4 CTAs
+// per SM, 3 with the rotation), 64 rows per CTA per step.
+static int64_t qk_ctas_per_entry(int64_t rows, int B, bool rotate) {
+    int64_t gx = (rows + 63) / 64;
+    const int64_t wave = (148 * (rotate ? 3 : 4) + B - 1) / B;
+    if (gx > wave) gx = wave;
+    return gx < 1 ? 1 : gx;
+}
+
 cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, int64_t ss, int64_t sh,
                                const int32_t *seqlens, int cap, uint8_t *codes, uint8_t *scales,
                                cudaStream_t stream, bool pad_to_cap, bool rotate) {
     const int row_len = pad_to_cap ? cap : S;
     const int64_t rows = static_cast<int64_t>(row_len) * H;  // per batch entry
     if (rows >= (int64_t{1} << 30)) return cudaErrorInvalidValue;
-    // About one wave over all batch entries (4 CTAs per SM, 3 with the rotation),
-    // 64 rows per CTA per step.
-    const int64_t rows_per_cta = 64;
-    int64_t gx = (rows + rows_per_cta - 1) / rows_per_cta;
-    const int64_t wave = (148 * (rotate ? 3 : 4) + B - 1) / B;
-    if (gx > wave) gx = wave;
-    if (gx < 1) gx = 1;
+    const int64_t gx = qk_ctas_per_entry(rows, B, rotate);
     // The grid's y extent is at most 65535: larger batches go in chunks.
     const int64_t codes_per_b = static_cast<int64_t>(H) * cap * 64;
     const int64_t scales_per_b = static_cast<int64_t>(H) * (cap / 128) * 512;
@@ -371,10 +425,10 @@ cudaError_t launch_quantize_qk(const void *x, int B, int S, int H, int64_t sb, i
         const __nv_bfloat16 *xs = static_cast<const __nv_bfloat16 *>(x) + b0 * sb;
         const int32_t *ls = seqlens ? seqlens + b0 : nullptr;
         if (rotate)
-            quantize_qk_kernel<true><<<grid, 256, 0, stream>>>(xs, nb, S, H, sb, ss, sh, ls, cap, row_len,
+            quantize_qk_kernel<true><<<grid, 256, 0, stream>>>(xs, S, H, sb, ss, sh, ls, cap, row_len,
                                                                codes + b0 * codes_per_b, scales + b0 * scales_per_b);
         else
-            quantize_qk_kernel<false><<<grid, 256, 0, stream>>>(xs, nb, S, H, sb, ss, sh, ls, cap, row_len,
+            quantize_qk_kernel<false><<<grid, 256, 0, stream>>>(xs, S, H, sb, ss, sh, ls, cap, row_len,
                                                                 codes + b0 * codes_per_b, scales + b0 * scales_per_b);
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
@@ -387,7 +441,47 @@ cudaError_t launch_quantize_v(const void *v, int B, int S, int H, int64_t sb, in
                               cudaStream_t stream) {
     const int64_t grid = static_cast<int64_t>(B) * H * (cap / 128);
     quantize_v_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(v), B, S, H, sb, ss, sh, seqlens, cap, codes, scales);
+        static_cast<const __nv_bfloat16 *>(v), S, H, sb, ss, sh, seqlens, cap, codes, scales);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_qkv(const void *q, const void *k, const void *v, int B, int Sq, int Sk, int Hq, int Hkv,
+                                const int32_t *seqlens_k, int q_cap, int kv_cap, uint8_t *q_codes, uint8_t *q_scales,
+                                uint8_t *k_codes, uint8_t *k_scales, uint8_t *v_codes, uint8_t *v_scales,
+                                cudaStream_t stream) {
+    const int64_t rows_q = static_cast<int64_t>(q_cap) * Hq, rows_k = static_cast<int64_t>(kv_cap) * Hkv;
+    if (rows_q >= (int64_t{1} << 30) || rows_k >= (int64_t{1} << 30)) return cudaErrorInvalidValue;
+    QkvArgs a{};
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.k = static_cast<const __nv_bfloat16 *>(k);
+    a.v = static_cast<const __nv_bfloat16 *>(v);
+    a.Sq = Sq;
+    a.Sk = Sk;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.q_cap = q_cap;
+    a.kv_cap = kv_cap;
+    a.qsh = 128;
+    a.qss = static_cast<int64_t>(Hq) * 128;
+    a.qsb = a.qss * Sq;
+    a.ksh = 128;
+    a.kss = static_cast<int64_t>(Hkv) * 128;
+    a.ksb = a.kss * Sk;
+    a.seqlens_k = seqlens_k;
+    a.q_codes = q_codes;
+    a.q_scales = q_scales;
+    a.k_codes = k_codes;
+    a.k_scales = k_scales;
+    a.v_codes = v_codes;
+    a.v_scales = v_scales;
+    a.gxq = static_cast<int>(qk_ctas_per_entry(rows_q, B, false));
+    a.gxk = static_cast<int>(qk_ctas_per_entry(rows_k, B, false));
+    const int64_t nq = static_cast<int64_t>(B) * a.gxq, nk = static_cast<int64_t>(B) * a.gxk;
+    const int64_t nv = static_cast<int64_t>(B) * Hkv * (kv_cap / 128);
+    if (nq + nk + nv >= (int64_t{1} << 31)) return cudaErrorInvalidValue;
+    a.nq = static_cast<int>(nq);
+    a.nk = static_cast<int>(nk);
+    quantize_qkv_kernel<<<static_cast<unsigned>(nq + nk + nv), 256, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -136,9 +136,11 @@ QK4V8_API int qk4v8_quantize_v(const void *v, int B, int S, int H, int d,
                      uint8_t *codes, uint8_t *scales, void *stream);
 
 /*
- * Q, K and V in one call (three launches on `stream`): Q [B][Sq][Hq][128] into
- * capacity q_cap, K and V [B][Sk][Hkv][128] into capacity kv_cap. Contiguous
- * [B][T][H][128] inputs; seqlens_k (device, nullable) marks valid KV tokens.
+ * Q, K and V in one call and one launch on `stream` (the same bytes as the three
+ * calls above): Q [B][Sq][Hq][128] into capacity q_cap, K and V
+ * [B][Sk][Hkv][128] into capacity kv_cap. Contiguous [B][T][H][128] inputs;
+ * seqlens_k (device, nullable) marks valid KV tokens. Errors as for the
+ * separate calls; q_cap * Hq and kv_cap * Hkv below 2^30.
  */
 QK4V8_API int qk4v8_quantize(const void *q, const void *k, const void *v,
                    int B, int Sq, int Sk, int Hq, int Hkv, int d,

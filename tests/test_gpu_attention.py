@@ -282,8 +282,12 @@ def test_deterministic():
     assert torch.equal(a, b) and torch.equal(c, d)
 
 
-def test_quantize_entry_point_matches_separate_calls():
-    gen = make_gen(2, 100, 300, 4, 2, seed=12, lens=[300, 150])
+@pytest.mark.parametrize("B,Sq,Sk,Hq,Hkv,lens", [
+    (2, 100, 300, 4, 2, [300, 150]),
+    (5, 1, 1000, 8, 2, [1000, 1, 0, 999, 512]),   # one launch: Q, K and V CTAs of five entries
+])
+def test_quantize_entry_point_matches_separate_calls(B, Sq, Sk, Hq, Hkv, lens):
+    gen = make_gen(B, Sq, Sk, Hq, Hkv, seed=12, lens=lens)
     q, k, v = to_dev(gen["q"]), to_dev(gen["k"]), to_dev(gen["v"])
     sl = torch.from_numpy(gen["seqlens"]).cuda()
     qp, kp, vp = qk.quantize(q, k, v, seqlens_k=sl)
