@@ -546,7 +546,7 @@ def run_paged(gen, steps, hbm_gbs):
         pages = idx[:, i]
         cache.k_codes[pages] = kp.codes[:, :, i * 128:(i + 1) * 128]
         cache.k_scales[pages] = kp.scales[:, :, i]
-        cache.v_codes[pages] = vp.codes[:, :, :, i * 128:(i + 1) * 128]
+        cache.v_codes[pages] = vp.codes[:, :, i]
         cache.v_scales[pages] = vp.scales[:, :, i]
     cache.seqlens.copy_(sl)
     # The staging buffer holds the open V group (none: 8192 is a multiple of 32).

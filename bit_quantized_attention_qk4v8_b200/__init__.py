@@ -51,8 +51,8 @@ class MXFP4:
 
 @dataclass
 class MXFP4V:
-    """Packed MXFP4 V (the QK4V4 comparison point): codes uint8 [B][H][128][cap/2]
-    (two tokens per byte), scales uint8 [B][H][cap/128][512]."""
+    """Packed MXFP4 V (the QK4V4 comparison point): codes uint8 [B][H][cap/128][128][64]
+    (128-token blocks of channel rows, two tokens per byte), scales uint8 [B][H][cap/128][512]."""
     codes: torch.Tensor
     scales: torch.Tensor
     B: int
@@ -63,7 +63,8 @@ class MXFP4V:
 
 @dataclass
 class MXFP8V:
-    """Packed MXFP8-E4M3 V: codes uint8 [B][H][128][cap], scales uint8 [B][H][cap/128][512]."""
+    """Packed MXFP8-E4M3 V: codes uint8 [B][H][cap/128][128][128] (128-token blocks of
+    channel rows), scales uint8 [B][H][cap/128][512]."""
     codes: torch.Tensor
     scales: torch.Tensor
     B: int
@@ -124,7 +125,7 @@ def quantize_v(v: torch.Tensor, cap: Optional[int] = None, seqlens=None, out: Op
     cap = round_cap(T) if cap is None else int(cap)
     sl = _seqlens(seqlens, B, v.device)
     if out is None:
-        out = MXFP8V(torch.empty((B, H, D, cap), dtype=torch.uint8, device=v.device),
+        out = MXFP8V(torch.empty((B, H, cap // 128, D, 128), dtype=torch.uint8, device=v.device),
                      torch.empty((B, H, cap // 128, 512), dtype=torch.uint8, device=v.device), B, H, cap, T)
     check(lib().qk4v8_quantize_v(v.data_ptr(), B, T, H, D, v.stride(0), v.stride(1), v.stride(2), _ptr(sl), cap,
                                  out.codes.data_ptr(), out.scales.data_ptr(), _stream(v.device)), "qk4v8_quantize_v")
@@ -139,7 +140,7 @@ def quantize_v4(v: torch.Tensor, cap: Optional[int] = None, seqlens=None, out: O
     cap = round_cap(T) if cap is None else int(cap)
     sl = _seqlens(seqlens, B, v.device)
     if out is None:
-        out = MXFP4V(torch.empty((B, H, D, cap // 2), dtype=torch.uint8, device=v.device),
+        out = MXFP4V(torch.empty((B, H, cap // 128, D, 64), dtype=torch.uint8, device=v.device),
                      torch.empty((B, H, cap // 128, 512), dtype=torch.uint8, device=v.device), B, H, cap, T)
     check(lib().qk4v8_quantize_v4(v.data_ptr(), B, T, H, D, v.stride(0), v.stride(1), v.stride(2), _ptr(sl), cap,
                                   out.codes.data_ptr(), out.scales.data_ptr(), _stream(v.device)), "qk4v8_quantize_v4")
@@ -172,7 +173,7 @@ def quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seqlens_k=None, 
                torch.empty((B, Hq, q_cap // 128, 512), dtype=torch.uint8, device=dev), B, Hq, q_cap, Sq)
     kp = MXFP4(torch.empty((B, Hkv, kv_cap, 64), dtype=torch.uint8, device=dev),
                torch.empty((B, Hkv, kv_cap // 128, 512), dtype=torch.uint8, device=dev), B, Hkv, kv_cap, Sk)
-    vp = MXFP8V(torch.empty((B, Hkv, D, kv_cap), dtype=torch.uint8, device=dev),
+    vp = MXFP8V(torch.empty((B, Hkv, kv_cap // 128, D, 128), dtype=torch.uint8, device=dev),
                 torch.empty((B, Hkv, kv_cap // 128, 512), dtype=torch.uint8, device=dev), B, Hkv, kv_cap, Sk)
     check(lib().qk4v8_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Sq, Sk, Hq, Hkv, D, _ptr(sl), q_cap,
                                kv_cap, qp.codes.data_ptr(), qp.scales.data_ptr(), kp.codes.data_ptr(),

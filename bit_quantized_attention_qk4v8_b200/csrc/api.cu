@@ -76,13 +76,15 @@ int make_k_map(CUtensorMap *map, const uint8_t *codes, int BH, int cap) {
     return QK4V8_OK;
 }
 
-// V codes [B*Hkv][128][cap] as a 3-D uint8 tensor, 128-token x 128-channel
-// boxes, 128-byte swizzle.
+// V codes [B*Hkv][cap / 128][128][128] (a 128-token block of a channel row
+// after another, each block's 16 KiB contiguous) as a 3-D uint8 tensor of
+// B*Hkv*(cap/128) 128-channel x 128-token tiles: tile z = row * (cap / 128) +
+// block, the index of its scale atom. 128-byte swizzle.
 int make_v_map(CUtensorMap *map, const uint8_t *codes, int BH, int cap) {
     auto enc = get_encode_fn();
     if (!enc) return set_error(QK4V8_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cap), 128, static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(cap), static_cast<cuuint64_t>(cap) * 128};
+    cuuint64_t dims[3] = {128, 128, static_cast<cuuint64_t>(BH) * static_cast<cuuint64_t>(cap / 128)};
+    cuuint64_t strides[2] = {128, 128 * 128};
     cuuint32_t box[3] = {128, 128, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(codes), dims, strides, box, estr,
@@ -92,16 +94,17 @@ int make_v_map(CUtensorMap *map, const uint8_t *codes, int BH, int cap) {
     return QK4V8_OK;
 }
 
-// MXFP4 V codes [B*Hkv][128][cap / 2] (the QK4V4 comparison point): loaded with
-// the 16U4_ALIGN16B element type, which lands each 16 packed codes (8 bytes)
-// in a 16-byte slot of shared memory, the layout the block-scaled f8f6f4 MMA
-// reads for an E2M1 operand. A 128-token x 128-channel box then fills the same
+// MXFP4 V codes [B*Hkv][cap / 128][128][64] (the QK4V4 comparison point; the
+// blocks as for MXFP8 V, 64 bytes per channel row of a block): loaded with the
+// 16U4_ALIGN16B element type, which lands each 16 packed codes (8 bytes) in a
+// 16-byte slot of shared memory, the layout the block-scaled f8f6f4 MMA reads
+// for an E2M1 operand. A 128-token x 128-channel box then fills the same
 // 128 x 128-byte, 128-byte-swizzled tile as an MXFP8 V box.
 int make_v4_map(CUtensorMap *map, const uint8_t *codes, int BH, int cap) {
     auto enc = get_encode_fn();
     if (!enc) return set_error(QK4V8_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cap), 128, static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(cap) / 2, static_cast<cuuint64_t>(cap) / 2 * 128};
+    cuuint64_t dims[3] = {128, 128, static_cast<cuuint64_t>(BH) * static_cast<cuuint64_t>(cap / 128)};
+    cuuint64_t strides[2] = {64, 64 * 128};
     cuuint32_t box[3] = {128, 128, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<uint8_t *>(codes), dims, strides, box,

@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars.kv_full[st], kKBytes + kVTmaBytes + 1024);
                 tma_load_3d(smem + kKOff + st * kKBytes, &tmap_k, 0, tile * 128, kvh, &bars.kv_full[st]);
-                tma_load_3d(smem + kVOff + st * kVBytes, &tmap_v, tile * 128, 0, kvh, &bars.kv_full[st]);
+                tma_load_3d(smem + kVOff + st * kVBytes, &tmap_v, 0, 0, kvh * nblk + tile, &bars.kv_full[st]);
                 const int64_t atom = (static_cast<int64_t>(kvh) * nblk + tile) * 512;
                 bulk_load(smem + kSfKOff + st * 512, p.k_scales + atom, 512, &bars.kv_full[st]);
                 bulk_load(smem + kSfVOff + st * 512, p.v_scales + atom, 512, &bars.kv_full[st]);

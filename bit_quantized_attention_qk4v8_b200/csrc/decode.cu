@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(DecodeLayout<NT, RW, NC, ST>::kThreads, MINB)
                 const int v_bytes = kExt && p.v_fp4 ? Lay::kVBytes / 2 : Lay::kVBytes;
                 mbar_arrive_expect_tx(&kv_full[st], Lay::kKBytes + v_bytes + 1024);
                 tma_load_3d(smem + Lay::kK + st * Lay::kKBytes, &tmap_k, 0, blk * 128, row, &kv_full[st]);
-                tma_load_3d(smem + Lay::kV + st * Lay::kVBytes, &tmap_v, blk * 128, 0, row, &kv_full[st]);
+                tma_load_3d(smem + Lay::kV + st * Lay::kVBytes, &tmap_v, 0, 0, row * nblk + blk, &kv_full[st]);
                 const int64_t atom = (static_cast<int64_t>(row) * nblk + blk) * 512;
                 bulk_load(smem + Lay::kSfK + st * 512, p.k_scales + atom, 512, &kv_full[st]);
                 bulk_load(smem + Lay::kSfV + st * 512, p.v_scales + atom, 512, &kv_full[st]);

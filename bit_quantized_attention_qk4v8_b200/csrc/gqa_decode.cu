@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kGdThreads, 1)
                 if (lane == 0) {
                     // An MXFP4 tile lands unpacked; the copy moves half the bytes.
                     mbar_arrive_expect_tx(&v_full[sv], (kExt && p.v_fp4 ? S::kVTmaBytes / 2 : S::kVTmaBytes) + 512);
-                    tma_load_3d(smem + S::kV + sv * S::kVBytes, &tmap_v, blk * 128, 0, row, &v_full[sv]);
+                    tma_load_3d(smem + S::kV + sv * S::kVBytes, &tmap_v, 0, 0, row * nblk + blk, &v_full[sv]);
                     bulk_load(smem + S::kSfV + sv * 512, p.v_scales + (static_cast<int64_t>(row) * nblk + blk) * 512,
                               512, &v_full[sv]);
                 }

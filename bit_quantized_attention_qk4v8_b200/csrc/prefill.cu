@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     ok = mbar_test_wait(&v_empty[sv], ph ^ 1) || wait_bar(&v_empty[sv], ph ^ 1, abort_flag, p.status);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&v_full[sv], S::kVTmaBytes + 512);
-                    tma_load_3d(smem + S::kV + sv * S::kVBytes, &tmap_v, jt * 128, 0, kvh, &v_full[sv]);
+                    tma_load_3d(smem + S::kV + sv * S::kVBytes, &tmap_v, 0, 0, kvh * nblk + jt, &v_full[sv]);
                     bulk_load(smem + S::kSfV + sv * 512, p.v_scales + (static_cast<int64_t>(kvh) * nblk + jt) * 512,
                               512, &v_full[sv]);
                     gv_issued = gv + 1;

@@ -276,9 +276,10 @@ __device__ __forceinline__ void v_tile(const __nv_bfloat16 *__restrict__ v, int 
     }
     __syncthreads();
     const int64_t head = static_cast<int64_t>(b) * H + h;
+    uint8_t *block = codes + (head * nblk + blk) * (128 * 128);  // the tile's 16 KiB, channel rows of 128 B
     for (int i = threadIdx.x; i < 128 * 8; i += 256) {
         const int row = i >> 3, ch = i & 7;
-        *reinterpret_cast<uint4 *>(codes + (head * 128 + row) * cap + t0 + ch * 16) =
+        *reinterpret_cast<uint4 *>(block + row * 128 + ch * 16) =
             *reinterpret_cast<const uint4 *>(&ctile[v_code_row(row) * kCPitch + ch * 16]);
     }
     if (threadIdx.x < 32)
@@ -381,9 +382,10 @@ __global__ void __launch_bounds__(256) quantize_v4_kernel(const __nv_bfloat16 *_
     }
     __syncthreads();
     const int64_t head = static_cast<int64_t>(b) * H + h;
+    uint8_t *block = codes + (head * nblk + blk) * (128 * 64);  // the tile's 8 KiB, channel rows of 64 B
     for (int i = threadIdx.x; i < 128 * 4; i += 256) {
         const int row = i >> 2, ch = i & 3;
-        *reinterpret_cast<uint4 *>(codes + (head * 128 + row) * (cap / 2) + t0 / 2 + ch * 16) =
+        *reinterpret_cast<uint4 *>(block + row * 64 + ch * 16) =
             *reinterpret_cast<const uint4 *>(&ctile[v_code_row(row) * kC4Pitch + ch * 16]);
     }
     if (threadIdx.x < 32)

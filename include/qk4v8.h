@@ -37,7 +37,11 @@
  *                                        token t, group g (channels 32g..32g+31) is
  *                                        at byte (t%32)*16 + ((t%128)/32)*4 + g.
  *   MXFP8 V tensor, capacity `cap` (a multiple of 128):
- *     codes  uint8 [B][H][128][cap]     E4M3, token-contiguous per channel.
+ *     codes  uint8 [B][H][cap/128][128][128]  E4M3 in 128-token blocks: block n
+ *                                        holds tokens 128n..128n+127 as 128
+ *                                        channel rows of 128 bytes (token t at
+ *                                        byte t%128 of its channel's row), each
+ *                                        block 16 KiB contiguous.
  *     scales uint8 [B][H][cap/128][512] E8M0, one per channel per 32 tokens. In
  *                                        block n, channel c, group g (tokens
  *                                        128n+32g .. 128n+32g+31) is at byte
@@ -259,8 +263,10 @@ QK4V8_API int qk4v8_attention_decode(const uint8_t *q_codes, const uint8_t *q_sc
  * 32 tokens along the sequence, the same OCP MX rule with emax 2), halving
  * V's cache bytes (136 instead of 200 bytes per token and KV head with K).
  *   MXFP4 V tensor, capacity cap (a multiple of 128):
- *     codes  uint8 [B][H][128][cap/2]   two E2M1 codes per byte along the
- *                                        token axis, even token in the low nibble
+ *     codes  uint8 [B][H][cap/128][128][64]  the 128-token blocks of MXFP8 V,
+ *                                        two E2M1 codes per byte along the token
+ *                                        axis (even token in the low nibble), 64
+ *                                        bytes per channel row of a block
  *                                        (qk4v8_mxfp4v_codes_bytes)
  *     scales uint8 [B][H][cap/128][512] as for MXFP8 V
  * qk4v8_quantize_v4: arguments as for qk4v8_quantize_v.

@@ -4,7 +4,7 @@ import torch
 
 import bit_quantized_attention_qk4v8_b200 as qk
 import oracle
-from layouts import qk_scales_logical, unpack_e2m1, v_scales_logical
+from layouts import qk_scales_logical, unpack_e2m1, v_codes_logical, v_scales_logical
 
 MAX_ABS_TOL = 3e-2   # attention output vs the fp64 oracle, unit-variance inputs
 MEAN_ABS_TOL = 3e-3
@@ -30,7 +30,7 @@ def packed_to_logical(qp, kp, vp, Tq, Tk):
     qs = qk_scales_logical(qp.scales.cpu().numpy(), Tq)
     kc = unpack_e2m1(kp.codes.cpu().numpy()[:, :, :Tk])
     ks = qk_scales_logical(kp.scales.cpu().numpy(), Tk)
-    vc = vp.codes.cpu().numpy()[:, :, :, :Tk]
+    vc = v_codes_logical(vp.codes.cpu().numpy())[:, :, :, :Tk]
     vs = v_scales_logical(vp.scales.cpu().numpy(), Tk)
     return dict(qc=qc, qs=qs, kc=kc, ks=ks, vc=vc, vs=vs)
 

@@ -24,6 +24,25 @@ def v_scales_logical(scales: np.ndarray, T: int) -> np.ndarray:
     return scales.reshape(B, H, nblk * 512)[:, :, idx]
 
 
+def v_codes_logical(codes: np.ndarray) -> np.ndarray:
+    """Blocked V codes [B, H, cap/128, 128, w] (w = 128 bytes per channel row of a
+    block for MXFP8, 64 for MXFP4) -> channel rows [B, H, 128, cap/128 * w]."""
+    B, H, nb, C, w = codes.shape
+    return np.transpose(codes, (0, 1, 3, 2, 4)).reshape(B, H, C, nb * w)
+
+
+def fill_v_bytes(codes, b, start, value, stop=None):
+    """Sets the token-axis bytes [start, stop) of batch entry b, every head and
+    channel, of blocked V codes [B, H, cap/128, 128, w] (torch or numpy; bytes are
+    tokens for MXFP8, token pairs for MXFP4). stop defaults to the capacity."""
+    nb, w = codes.shape[2], codes.shape[4]
+    stop = nb * w if stop is None else stop
+    for blk in range(start // w, (stop + w - 1) // w):
+        lo, hi = max(start - blk * w, 0), min(stop - blk * w, w)
+        if lo < hi:
+            codes[b, :, blk, :, lo:hi] = value
+
+
 def unpack_e2m1(packed: np.ndarray) -> np.ndarray:
     """[..., 64] bytes -> [..., 128] codes, element 2i from the low nibble of byte i."""
     out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), dtype=np.uint8)

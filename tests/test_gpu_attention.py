@@ -16,7 +16,7 @@ import oracle
 import synth
 from bit_quantized_attention_qk4v8_b200 import _lib
 from gpu_util import assert_close, err_stats, oracle_attention_from, packed_to_logical, quantize_on_gpu, to_dev
-from layouts import qk_scales_logical, unpack_e2m1
+from layouts import fill_v_bytes, qk_scales_logical, unpack_e2m1
 
 pytestmark = pytest.mark.gpu
 
@@ -188,7 +188,7 @@ def test_decode_poisoned_padding_does_not_leak():
     qp, kp, vp, sl = quantize_on_gpu(gen)
     clean = qk.attention_decode(qp, kp, vp, sl, max_seqlen=300, num_splits=2)
     for b, L in enumerate([300, 45]):
-        vp.codes[b, :, :, L:] = 0xFF          # E4M3 NaN
+        fill_v_bytes(vp.codes, b, L, 0xFF)    # E4M3 NaN
         kp.codes[b, :, L:] = 0xFF
         blk0 = L // 128
         # scale atoms of blocks fully past L, and the groups past L inside block blk0
@@ -213,7 +213,7 @@ def _poison_padding(kp, vp, lens):
     codes, whole scale atoms past the last block, and the scale entries of the
     padding rows and groups inside the last block."""
     for b, L in enumerate(lens):
-        vp.codes[b, :, :, L:] = 0xFF          # E4M3 NaN
+        fill_v_bytes(vp.codes, b, L, 0xFF)    # E4M3 NaN
         kp.codes[b, :, L:] = 0xFF
         blk0 = L // 128
         vp.scales[b, :, blk0 + 1:] = 0xFF

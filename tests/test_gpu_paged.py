@@ -122,7 +122,7 @@ def _paged_from_contiguous(kp, vp, max_pages, num_pages, seed):
         pages = idx[:, i]
         cache.k_codes[pages] = kp.codes[:, :, i * 128:(i + 1) * 128]
         cache.k_scales[pages] = kp.scales[:, :, i]
-        cache.v_codes[pages] = vp.codes[:, :, :, i * 128:(i + 1) * 128]
+        cache.v_codes[pages] = vp.codes[:, :, i]
         cache.v_scales[pages] = vp.scales[:, :, i]
     return cache
 

@@ -14,7 +14,7 @@ import bit_quantized_attention_qk4v8_b200 as qk
 import oracle
 import synth
 from gpu_util import assert_close, to_dev
-from layouts import v_scales_logical
+from layouts import fill_v_bytes, v_codes_logical, v_scales_logical
 
 pytestmark = pytest.mark.gpu
 
@@ -38,7 +38,7 @@ def check_v4(bits, cap=None, seqlens=None):
     sl = None if seqlens is None else torch.tensor(list(seqlens), dtype=torch.int32)
     vp = qk.quantize_v4(to_dev(bits), cap=cap, seqlens=sl)
     torch.cuda.synchronize()
-    codes = unpack_tokens(vp.codes.cpu().numpy())
+    codes = unpack_tokens(v_codes_logical(vp.codes.cpu().numpy()))
     scales = vp.scales.cpu().numpy()
     oc, os_ = oracle.quantize_v(bits, seqlens, fmt=oracle.E2M1)
     assert np.array_equal(codes[..., :T], oc)
@@ -117,7 +117,7 @@ def test_v4_decode_poisoned_scales_past_length():
     for b, L in enumerate(lens):
         blk0 = L // 128
         vp.scales[b, :, blk0 + 1:] = 0xFF
-        vp.codes[b, :, :, (L + 1) // 2:] = 0xFF       # E2M1 -6: finite, and P is zero there
+        fill_v_bytes(vp.codes, b, (L + 1) // 2, 0xFF)   # E2M1 -6: finite, and P is zero there
         jv = L - blk0 * 128
         idx = torch.tensor([(c % 32) * 16 + (c // 32) * 4 + g for c in range(128) for g in range((jv + 31) // 32, 4)],
                            dtype=torch.long, device="cuda")

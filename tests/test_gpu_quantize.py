@@ -12,7 +12,7 @@ import bit_quantized_attention_qk4v8_b200 as qk
 import oracle
 import synth
 from gpu_util import to_dev
-from layouts import qk_scales_logical, unpack_e2m1, v_scales_logical
+from layouts import qk_scales_logical, unpack_e2m1, v_codes_logical, v_scales_logical
 
 pytestmark = pytest.mark.gpu
 
@@ -46,7 +46,7 @@ def check_v(bits, cap=None, seqlens=None):
     sl = None if seqlens is None else torch.tensor(seqlens, dtype=torch.int32)
     vp = qk.quantize_v(to_dev(bits), cap=cap, seqlens=sl)
     torch.cuda.synchronize()
-    codes = vp.codes.cpu().numpy()
+    codes = v_codes_logical(vp.codes.cpu().numpy())
     scales = vp.scales.cpu().numpy()
     oc, os_ = oracle.quantize_v(bits, seqlens)
     assert np.array_equal(codes[..., :T], oc)
@@ -151,7 +151,7 @@ def test_workload_quantize_bit_exact(name):
         assert np.array_equal(unpack_e2m1(kp.codes[b:b + 1].cpu().numpy()[:, :, :wl.Lk]), kc)
         assert np.array_equal(qk_scales_logical(kp.scales[b:b + 1].cpu().numpy(), wl.Lk), ks)
         vc, vs = oracle.quantize_v(gen["v"][b:b + 1], lens[b:b + 1])
-        assert np.array_equal(vp.codes[b:b + 1].cpu().numpy()[..., :wl.Lk], vc)
+        assert np.array_equal(v_codes_logical(vp.codes[b:b + 1].cpu().numpy())[..., :wl.Lk], vc)
         assert np.array_equal(v_scales_logical(vp.scales[b:b + 1].cpu().numpy(), wl.Lk), vs)
 
 

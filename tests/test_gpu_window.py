@@ -17,6 +17,7 @@ import bit_quantized_attention_qk4v8_b200 as qk
 import oracle
 import synth
 from gpu_util import assert_close, quantize_on_gpu, to_dev
+from layouts import fill_v_bytes
 
 pytestmark = pytest.mark.gpu
 
@@ -87,7 +88,7 @@ def test_window_streams_only_the_window():
     for b, L in enumerate(lens):
         t0 = (L - nq - W) // 128          # first tile of the window
         kp.codes[b, :, :t0 * 128] = 0xFF
-        vp.codes[b, :, :, :t0 * 128] = 0xFF
+        fill_v_bytes(vp.codes, b, 0, 0xFF, stop=t0 * 128)
         kp.scales[b, :, :t0] = 0xFF
         vp.scales[b, :, :t0] = 0xFF
     dirty = qk.attention_decode(qp, kp, vp, sl, max_seqlen=4000, causal_in_block=False, window=W)
