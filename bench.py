@@ -76,8 +76,8 @@ L2_BYTES = 126 * 2 ** 20
 # kernel, from its committed ncu capture; None until a capture of the kernel as
 # it stands exists.
 NCU_TRAFFIC = {
-    DECODE_WORKLOAD: (423917568, "profiles/decode_attention_b32_hq32_hkv8_l8192.md (dram read 419.77 MB + write "
-                                 "4.15 MB, qk4v8_decode_kernel<16,4,4,4,2,false>)"),
+    DECODE_WORKLOAD: (423641088, "profiles/decode_attention_b32_hq32_hkv8_l8192.md (dram read 419.78 MB + write "
+                                 "3.86 MB, qk4v8_decode_kernel<16,4,4,4,2,false>, blocked V)"),
 }
 
 
