@@ -611,7 +611,9 @@ def run_draft_block(gen, hbm_gbs, window=1024, reps=20):
     splits = qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, wl.Lk, window)
     ws = torch.empty((max(16, qk.decode_bf16_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, splits)),),
                      dtype=torch.uint8, device="cuda")
-    flush = torch.empty((256 * 2 ** 20,), dtype=torch.uint8, device="cuda")
+    # 1 GiB: larger than L2, and its write (~160 us) outlasts the host's enqueue of
+    # the timed launches, so the start event fires when the device reaches them.
+    flush = torch.empty((1024 * 2 ** 20,), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step():
@@ -638,7 +640,7 @@ def run_draft_block(gen, hbm_gbs, window=1024, reps=20):
     return dict(res={"workload": f"draft block on {VERIFY_WORKLOAD}: 8 non-causal rows, window {window}",
                      "ms_per_step": ms, "value": gbs, "unit": "GB/s", "roofline_frac": gbs / hbm_gbs,
                      "visible_kv_bytes": vis_bytes, "kv_splits": splits, "steps": reps,
-                     "l2": "flushed (256 MB write) before each timed step",
+                     "l2": "flushed (1 GiB write) before each timed step",
                      "tokens_per_s": wl.B * wl.Sq / (ms * 1e-3)},
                 out=out.float().cpu().numpy(), window=window)
 
@@ -755,13 +757,15 @@ def run_prefill_small(steps=200):
 
 def run_quantize_kernels(hbm_gbs, gen, reps=10):
     """HBM throughput of the quantize kernels on the S=8192 prefill workload's
-    tensors (`gen`); L2 is flushed (a 256 MB write) before every timed launch."""
+    tensors (`gen`); L2 is flushed (a 1 GiB write) before every timed launch."""
     import torch
     import bit_quantized_attention_qk4v8_b200 as qk
     import synth
     wl = synth.WORKLOADS[PREFILL_WORKLOAD]
     q, k, v = to_dev(gen["q"]), to_dev(gen["k"]), to_dev(gen["v"])
-    flush = torch.empty((256 * 2 ** 20,), dtype=torch.uint8, device="cuda")
+    # 1 GiB: larger than L2, and its write (~160 us) outlasts the host's enqueue of
+    # the timed launches, so the start event fires when the device reaches them.
+    flush = torch.empty((1024 * 2 ** 20,), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     qp = qk.quantize_qk(q)
     kp = qk.quantize_qk(k)
@@ -779,7 +783,7 @@ def run_quantize_kernels(hbm_gbs, gen, reps=10):
     res = {"workload": PREFILL_WORKLOAD, "unit": "GB/s", "peak_gbs": hbm_gbs,
            "bytes": "algorithmic: 256 B bf16 read + 64 B codes + 4 B scales written per Q/K token-head row; "
                     "256 B read + 128 B codes + 4 B scales per V token-head",
-           "l2": "flushed (256 MB write) before each timed launch"}
+           "l2": "flushed (1 GiB write) before each timed launch"}
     for key, kname, fn, nbytes in cases:
         fn()
         torch.cuda.synchronize()
