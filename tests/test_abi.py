@@ -99,6 +99,9 @@ def test_plan_splits(lib):
         return lib.qk4v8_decode_plan_splits(B, Hq, Hkv, nq, a.ctypes.data_as(ctypes.c_void_p), window)
 
     assert plan(2, 4, 1, 1, [1280, 128]) == 10
+    # Window 128: the tiles are counted from the window's first key, 2 and 1 here:
+    # s=1 ends at 2/1.5 + 17 = 18.3, s=2 (three 1-tile CTAs) at 1/1.5 + 17 + 4 = 21.7.
+    assert plan(2, 4, 1, 1, [1280, 128], window=128) == 1
     assert plan(32, 32, 8, 1, [8192] * 32) == 1
     assert plan(64, 64, 8, 8, [16384] * 64) == lib.qk4v8_decode_default_splits(64, 64, 8, 8, 16384)
     assert plan(0, 4, 1, 1, [1]) == 1

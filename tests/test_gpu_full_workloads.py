@@ -53,7 +53,8 @@ def test_decode_workload_full_size(name):
     vp = qk.quantize_v(to_dev(gen["v"]), cap=cap, seqlens=sl)
     q = to_dev(gen["q"])
     max_len = int(lens.max())
-    splits = qk.decode_default_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, max_len)
+    # The split count bench.py times: the plan from the host-side lengths.
+    splits = qk.decode_plan_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, lens)
     out, lse = qk.attention_decode_bf16(q, kp, vp, sl, max_seqlen=max_len, num_splits=splits, return_lse=True)
     torch.cuda.synchronize()
     out = out.float().cpu().numpy()   # [B, nq, Hq, d]
@@ -95,7 +96,7 @@ def test_prefill_workload_full_size():
 @pytest.mark.parametrize("name", ["decode_gqa_b32_hq32_hkv8_l8192", "decode_long_b8_hq64_hkv8_l64k_128k",
                                   "verify_b64_nq8_hq64_hkv8_l16384"])
 def test_qk4v4_workload_full_size(name):
-    """QK4V4 (V in MXFP4) at full size, as bench.py runs it: bf16 queries, default splits."""
+    """QK4V4 (V in MXFP4) at full size, as bench.py runs it: bf16 queries, the planned splits."""
     wl = synth.WORKLOADS[name]
     gen = wl.generate()
     lens = gen["seqlens"]
@@ -104,7 +105,9 @@ def test_qk4v4_workload_full_size(name):
     kp = qk.quantize_qk(to_dev(gen["k"]), cap=cap, seqlens=sl)
     vp = qk.quantize_v4(to_dev(gen["v"]), cap=cap, seqlens=sl)
     max_len = int(lens.max())
-    out, lse = qk.attention_decode_bf16(to_dev(gen["q"]), kp, vp, sl, max_seqlen=max_len, return_lse=True)
+    splits = qk.decode_plan_splits(wl.B, wl.Hq, wl.Hkv, wl.Sq, lens)
+    out, lse = qk.attention_decode_bf16(to_dev(gen["q"]), kp, vp, sl, max_seqlen=max_len, num_splits=splits,
+                                        return_lse=True)
     torch.cuda.synchronize()
     out = out.float().cpu().numpy()
     lse = lse.cpu().numpy()
