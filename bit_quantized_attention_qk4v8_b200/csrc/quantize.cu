@@ -167,8 +167,9 @@ __global__ void __launch_bounds__(256, kRotate ? 3 : 4) quantize_qk_kernel(const
 // ------------------------------------------------------------------ MXFP8 V
 
 // One CTA per (b, h, 128-token block): stage the bf16 tile in shared memory,
-// quantize each channel's four 32-token groups, and write the token-contiguous
-// codes plus the block's 512-byte scale atom.
+// quantize each channel's four 32-token groups, and write the block's codes
+// (128 channel rows of 128 tokens, 16 KiB contiguous) plus its 512-byte scale
+// atom.
 constexpr int kVPitch = 136;  // bf16 elements per staged token row (16-byte padding)
 constexpr int kCPitch = 144;  // bytes per staged code row
 
