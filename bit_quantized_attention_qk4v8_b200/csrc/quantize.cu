@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(256, 4) quantize_qkv_kernel(const QkvArgs a) {
 // groups of 32 along the token axis like the MXFP8 V. Same staging as
 // quantize_v_kernel; each thread encodes the 32-token group of two channels to
 // 16 bytes of packed E2M1 each (even token in the low nibble), and the
-// 128-token tile of a channel row is 64 bytes of codes [B][H][128][cap / 2].
+// 128-token block of a channel row is 64 bytes of codes [B][H][cap / 128][128][64].
 constexpr int kC4Pitch = 80;  // bytes per staged code row (64 + 16 padding)
 
 __global__ void __launch_bounds__(256) quantize_v4_kernel(const __nv_bfloat16 *__restrict__ v, int B, int S, int H,
